@@ -1,0 +1,444 @@
+"""Pins of the CPU oracle to facts fixed outside it: the pages' printed numbers,
+closed forms, independent library routines, exact rational brute force and
+algebraic identities.  CPU only."""
+
+import json
+import math
+import os
+import statistics
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import oracle as O
+
+F32 = np.float32
+
+
+# ---------------------------------------------------------------------------
+# Normal quantile (AS241)
+# ---------------------------------------------------------------------------
+def test_ppf_matches_two_independent_libraries():
+    # statistics.NormalDist and scipy (Cephes ndtri) are separate implementations.
+    nd = statistics.NormalDist()
+    ps = np.concatenate([np.linspace(1e-6, 1 - 1e-6, 4001), [1e-300, 1e-20, 1e-10, 0.02, 0.075, 0.925,
+                                                            0.9677083, 0.5 + 1e-12, 1 - 1e-12]])
+    for p in ps:
+        got = O.norm_ppf(float(p))
+        ref1 = nd.inv_cdf(float(p))
+        ref2 = float(scipy.special.ndtri(p))
+        tol = 4e-16 * max(1.0, abs(ref1))
+        assert abs(got - ref1) <= tol + 1e-300, (p, got, ref1)
+        assert abs(got - ref2) <= 1e-13 * max(1.0, abs(ref2)), (p, got, ref2)
+
+
+def test_ppf_inverts_erf_cdf():
+    # Phi(x) = (1 + erf(x / sqrt 2)) / 2 from the C library, a different route.
+    for x in np.linspace(-6, 6, 241):
+        p = 0.5 * (1.0 + math.erf(x / math.sqrt(2.0)))
+        if 1e-12 < p < 1 - 1e-12:
+            assert abs(O.norm_ppf(p) - x) < 1e-7 * max(1.0, abs(x)) + 1e-9
+    assert O.norm_ppf(0.5) == 0.0
+
+
+# ---------------------------------------------------------------------------
+# NF4 level table
+# ---------------------------------------------------------------------------
+def test_levels_structure():
+    lv = O.nf4_levels()
+    assert lv.dtype == np.float32 and lv.shape == (16,)
+    assert np.all(np.diff(lv) > 0)                    # 16 sorted, distinct levels
+    assert lv[7] == 0.0 and np.signbit(lv[7]) == 0    # exact zero
+    assert lv[0] == -1.0 and lv[15] == 1.0            # endpoints +-1
+    assert np.sum(lv > 0) == 8 and np.sum(lv < 0) == 7  # 8 positive, 7 negative
+    assert float(np.min(np.diff(lv))) == pytest.approx(0.0795803, abs=1e-7)
+
+
+def _torch_fp32_levels():
+    """The glossary snippet's construction, re-expressed in torch float32."""
+    nrm = torch.distributions.Normal(0.0, 1.0)
+    up = nrm.icdf(torch.linspace(0.9677083, 0.5, 9)[:-1])
+    dn = -nrm.icdf(torch.linspace(0.9677083, 0.5, 8)[:-1])
+    t = torch.cat([dn, torch.zeros(1), up]).sort().values
+    return (t / t.max()).numpy()
+
+
+def test_levels_close_to_snippet_float32_build():
+    # The snippet builds the table with several float32 roundings (linspace, icdf,
+    # the division by the max); the oracle rounds the exact values once.  The two
+    # agree to float32 working precision (a few ulp on the small levels).
+    ours = O.nf4_levels().view(np.int32).astype(np.int64)
+    theirs = _torch_fp32_levels().view(np.int32).astype(np.int64)
+    assert np.max(np.abs(ours - theirs)) <= 8
+    assert np.sum(ours != theirs) <= 12
+
+
+# ---------------------------------------------------------------------------
+# The page's worked example
+# ---------------------------------------------------------------------------
+def _snippet_weights():
+    torch.manual_seed(0)
+    return (torch.randn(4096, 64) * 0.02).numpy()
+
+
+def _mse(w, lv):
+    s = O.block_absmax(w)
+    c = O.assign_codes(w, s, lv)
+    rest = (lv[c].reshape(-1, 64) * s[:, None]).astype(F32)
+    return float(np.mean((rest.astype(np.float64) - w.reshape(-1, 64).astype(np.float64)) ** 2)), c
+
+
+def test_page_example_printed_mse(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "ul_snippet_mse.json")))
+    w = _snippet_weights()
+    assert w.shape == (g["blocks"], g["block"])
+    nf4, _ = _mse(w, O.nf4_levels())
+    uni, _ = _mse(w, O.uniform4_levels())
+    assert f"{nf4:.3e}" == g["nf4_mse_printed"]
+    assert f"{uni:.3e}" == g["uniform4_mse_printed"]
+    assert abs((1 - nf4 / uni) - g["relative_reduction_stated"]) < 0.01
+
+
+def test_page_example_codes_match_torch_argmin():
+    # Same data through torch's own float32 argmin with the snippet's level table:
+    # every one of the 262144 codes agrees (argmin semantics, ties, float32 math).
+    w = _snippet_weights()
+    _, ours = _mse(w, O.nf4_levels())
+    wt = torch.from_numpy(w)
+    am = wt.abs().amax(dim=1, keepdim=True)
+    lv = torch.from_numpy(_torch_fp32_levels())
+    theirs = ((wt / am)[..., None] - lv).abs().argmin(dim=-1).reshape(-1).numpy()
+    assert np.array_equal(ours.astype(np.int64), theirs)
+
+
+@pytest.mark.parametrize("seed", [1, 2, 3])
+def test_nf4_beats_uniform_by_about_16_percent(seed):
+    g = torch.Generator().manual_seed(seed)
+    w = (torch.randn(8192, 64, generator=g) * 0.02).numpy()
+    nf4, _ = _mse(w, O.nf4_levels())
+    uni, _ = _mse(w, O.uniform4_levels())
+    assert 0.14 < 1 - nf4 / uni < 0.18
+
+
+# ---------------------------------------------------------------------------
+# Code assignment: exact-rational brute force of the float32 definition
+# ---------------------------------------------------------------------------
+def _fl32(q: Fraction) -> Fraction:
+    """Round a rational to the nearest float32 (ties to even), normal/subnormal."""
+    if q == 0:
+        return Fraction(0)
+    sign = -1 if q < 0 else 1
+    a = abs(q)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1
+    e = max(e, -126)
+    ulp = Fraction(2) ** (e - 23)
+    n = a / ulp
+    fl = n.numerator // n.denominator
+    rem = n - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1):
+        fl += 1
+    return sign * fl * ulp
+
+
+def _brute_codes(block, levels):
+    ws = [Fraction(float(v)) for v in block]
+    s = max(abs(v) for v in ws)
+    lv = [Fraction(float(v)) for v in levels]
+    out = []
+    for w in ws:
+        if s == 0:
+            out.append(7)
+            continue
+        x = _fl32(w / s)
+        d = [abs(_fl32(x - l)) for l in lv]
+        out.append(min(range(16), key=lambda j: (d[j], j)))
+    return out
+
+
+def test_codes_exact_rational_bruteforce():
+    rng = np.random.default_rng(7)
+    w = (rng.standard_normal((24, 64)) * 0.02).astype(F32)
+    w[3] = 0.0                                          # all-zero block
+    w[5, :] = np.float32(1e-30) * rng.standard_normal(64).astype(F32)  # tiny scale
+    lv = O.nf4_levels()
+    got = O.assign_codes(w, O.block_absmax(w), lv).reshape(24, 64)
+    for b in range(24):
+        assert list(got[b]) == _brute_codes(w[b], lv), b
+
+
+def _tie_points(levels):
+    """float32 x in (L_j, L_j+1) with fl32(x - L_j) == fl32(L_j+1 - x)."""
+    pts = []
+    for j in range(15):
+        lo, hi = Fraction(float(levels[j])), Fraction(float(levels[j + 1]))
+        mid = np.float32(float((lo + hi) / 2))
+        cand = mid
+        for _ in range(8):
+            cand = np.nextafter(cand, np.float32(-2))
+        for _ in range(17):
+            x = Fraction(float(cand))
+            if _fl32(x - lo) == _fl32(hi - x):
+                pts.append((j, np.float32(cand)))
+            cand = np.nextafter(cand, np.float32(2))
+    return pts
+
+
+def test_ties_go_to_lower_level():
+    lv = O.nf4_levels()
+    ties = _tie_points(lv)
+    assert len(ties) >= 3
+    for j, x in ties:
+        blk = np.zeros(64, F32)
+        blk[0] = 1.0                                    # S = 1, so w / S = w exactly
+        blk[1] = x
+        c = O.assign_codes(blk, O.block_absmax(blk), lv)
+        assert c[1] == j, (j, x)
+
+
+def test_exact_levels_map_to_themselves():
+    lv = O.nf4_levels()
+    for s in (F32(1.0), F32(0.037), F32(3.5e-4)):
+        blk = np.zeros(64, F32)
+        blk[:16] = (lv * s).astype(F32)
+        blk[16:32] = (lv * s).astype(F32)[::-1]
+        c = O.assign_codes(blk, O.block_absmax(blk), lv)
+        if s == 1.0:
+            assert list(c[:16]) == list(range(16))
+        assert c[0] == 0 and c[15] == 15 and c[7] == 7
+
+
+def test_zero_block_and_zero_group():
+    w = np.zeros((2, 64 * 300), F32)                    # 600 blocks -> groups of 256, 256, 88
+    w[1, 5] = 0.5
+    q = O.quantize(w, 2, 64 * 300)
+    codes = O.unpack_codes(q["codes"])
+    assert np.all(codes[:300 * 64] == 7)
+    assert np.all(q["absmax"][:300] == 0)
+    assert q["c2"][0] == 0 and np.all(q["scale_codes"][:256] == 0)
+    wd = O.dequantize(q["codes"], q["scale_codes"], q["c2"], 2, 64 * 300)
+    assert np.all(wd[0] == 0) and not np.any(np.signbit(wd[0]))
+    assert wd[1, 5] == 0.5
+
+
+def test_pack_layout():
+    codes = np.array([1, 2, 3, 4, 15, 0], np.uint8)
+    p = O.pack_codes(codes)
+    assert list(p) == [0x21, 0x43, 0x0F]
+    assert np.array_equal(O.unpack_codes(p), codes)
+
+
+# ---------------------------------------------------------------------------
+# OCP FP8 E4M3
+# ---------------------------------------------------------------------------
+def test_e4m3_spec_points():
+    # max normal 1.75*2^8, min normal 2^-6, min subnormal 2^-9, one, ties to even
+    assert O.e4m3_encode([448.0])[0] == 0x7E
+    assert O.e4m3_encode([2.0 ** -6])[0] == 0x08
+    assert O.e4m3_encode([2.0 ** -9])[0] == 0x01
+    assert O.e4m3_encode([1.0])[0] == 0x38
+    assert O.e4m3_encode([0.0])[0] == 0x00
+    assert O.e4m3_encode([1.0625])[0] == 0x38     # halfway 1 .. 1.125 -> even (1.0)
+    assert O.e4m3_encode([1.1875])[0] == 0x3A     # halfway 1.125 .. 1.25 -> even (1.25)
+    assert O.e4m3_encode([2.0 ** -10])[0] == 0x00  # halfway 0 .. 2^-9 -> even (0)
+    assert O.e4m3_encode([1000.0])[0] == 0x7E     # saturates
+    assert O.e4m3_decode(0x7E) == 448.0 and np.isnan(O.e4m3_decode(0x7F))
+    assert O.e4m3_decode(0x01) == 2.0 ** -9 and O.e4m3_decode(0xB8) == -1.0
+
+
+def test_e4m3_decode_all_codes_vs_torch():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+    got = O.e4m3_decode(codes)
+    nan = np.isnan(ref)
+    assert np.array_equal(nan, np.isnan(got))
+    assert np.array_equal(ref[~nan], got[~nan])
+
+
+def _torch_e4m3(x):
+    return torch.from_numpy(np.asarray(x, F32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def test_e4m3_encode_vs_torch():
+    pos = O.e4m3_decode(np.arange(0x7F)).astype(np.float64)
+    mids = ((pos[1:] + pos[:-1]) / 2).astype(F32)
+    around = [mids]
+    for k in range(1, 4):
+        around += [np.nextafter(mids, np.float32(1e9)), np.nextafter(mids, np.float32(-1))]
+        mids = around[-2]
+    probe = np.concatenate(around + [pos.astype(F32)])
+    rng = np.random.default_rng(3)
+    probe = np.concatenate([probe, np.exp(rng.uniform(np.log(1e-4), np.log(448.0), 400000)).astype(F32),
+                            rng.uniform(0, 448.0, 100000).astype(F32)])
+    probe = probe[(probe >= 0) & (probe <= 448.0)]
+    assert np.array_equal(O.e4m3_encode(probe), _torch_e4m3(probe))
+
+
+# ---------------------------------------------------------------------------
+# Double quantisation and storage size
+# ---------------------------------------------------------------------------
+def test_double_quant_scale_error_bound():
+    rng = np.random.default_rng(11)
+    w = (rng.standard_normal(64 * 256 * 3 + 64 * 17) * 0.02).astype(F32)
+    q = O.quantize(w, 1, w.size)
+    s, sp = q["absmax"], O.dequantize_scales(q["scale_codes"], q["c2"])
+    g = np.arange(s.size) // 256
+    normal_range = s / q["c2"][g] >= 2.0 ** -6
+    rel = np.abs(sp - s) / s
+    assert np.all(rel[normal_range] <= 2.0 ** -4 * (1 + 1e-6))
+    # the group maximum is encoded at the top of the E4M3 range
+    for gi in range(q["c2"].size):
+        blk = slice(gi * 256, (gi + 1) * 256)
+        assert q["scale_codes"][blk].max() == 0x7E
+
+
+def test_storage_overhead_closed_form(golden_dir):
+    figs = {f["what"]: f["value"] for f in json.load(open(os.path.join(golden_dir, "memory_figures.json")))["figures"]}
+    rows, cols = 4096, 4096
+    cb, sb, c2b = O.storage_bytes(rows, cols)
+    bits = 8.0 * (cb + sb + c2b) / (rows * cols)
+    assert bits == 4 + 8 / 64 + 32 / (64 * 256)                    # 4.126953125 exactly
+    overhead = bits - 4
+    no_dq = 32 / 64
+    assert no_dq == figs["first-level scale overhead without double quantisation, bits per parameter"]
+    assert round(overhead, 3) == figs["scale overhead with double quantisation, bits per parameter (about)"]
+    saving = no_dq - overhead
+    assert round(saving, 2) == figs["saving from double quantisation, bits per parameter (about)"]
+    assert round(saving, 1) == figs["saving from nested quantisation, bits per parameter"]
+    p65 = 65e9
+    assert round(p65 * saving / 8 / 1e9) == figs["saving from double quantisation at 65B parameters, GB (about)"]
+    assert round(p65 * 2 / 1e9) == figs["65B weights at 16 bit, GB (about)"]
+    gb = p65 * bits / 8 / 1e9                                        # 33.5 GB
+    assert abs(gb - figs["65B 4-bit weights plus double-quantised scales, GB (about)"]) <= 0.5
+    # the two pages round the same quantity differently (34 vs 33); 33.5 lies between
+    assert abs(gb - figs["65B base model in NF4, GB (about)"]) <= 1.0
+
+
+def test_requantise_is_idempotent():
+    rng = np.random.default_rng(5)
+    rows, cols = 96, 640
+    w = (rng.standard_normal((rows, cols)) * 0.02).astype(F32)
+    q = O.quantize(w, rows, cols)
+    wd = O.dequantize(q["codes"], q["scale_codes"], q["c2"], rows, cols)
+    q2 = O.quantize(wd, rows, cols)
+    assert np.array_equal(q["codes"], q2["codes"])
+
+
+def test_dequantize_is_level_times_scale_rounded_once():
+    rng = np.random.default_rng(9)
+    rows, cols = 8, 256
+    w = (rng.standard_normal((rows, cols)) * 0.02).astype(F32)
+    q = O.quantize(w, rows, cols)
+    wd = O.dequantize(q["codes"], q["scale_codes"], q["c2"], rows, cols).reshape(-1)
+    codes = O.unpack_codes(q["codes"])
+    lv = O.nf4_levels()
+    for i in range(0, rows * cols, 37):                 # exact rational re-derivation
+        b = i // 64
+        sp = _fl32(Fraction(float(O.e4m3_decode(q["scale_codes"][b]))) * Fraction(float(q["c2"][b // 256])))
+        prod = _fl32(Fraction(float(lv[codes[i]])) * sp)
+        # bf16 RNE of a float32: keep 8 significant bits
+        v = float(prod)
+        ref = float(torch.tensor(v, dtype=torch.float32).to(torch.bfloat16).float())
+        assert wd[i] == ref
+
+
+# ---------------------------------------------------------------------------
+# Linear layer with LoRA
+# ---------------------------------------------------------------------------
+def _tiny_linear(seed=0, m=4, n=8, k=16, r=2):
+    rng = np.random.default_rng(seed)
+    w = rng.standard_normal((n, k))
+    a = rng.standard_normal((r, k))
+    b = rng.standard_normal((n, r))
+    x = rng.standard_normal((m, k))
+    dy = rng.standard_normal((m, n))
+    return w, a, b, x, dy
+
+
+def test_linear_fwd_bruteforce_loops():
+    w, a, b, x, _ = _tiny_linear()
+    m, k = x.shape
+    n, r = b.shape
+    alpha = 3.0
+    s = alpha / r
+    y, t = O.linear_fwd(w, a, b, x, alpha, r)
+    for i in range(m):
+        for jr in range(r):
+            assert abs(t[i, jr] - sum(x[i, kk] * a[jr, kk] for kk in range(k))) < 1e-12
+        for j in range(n):
+            base = sum(x[i, kk] * w[j, kk] for kk in range(k))
+            lora = sum(sum(x[i, kk] * a[jr, kk] for kk in range(k)) * b[j, jr] for jr in range(r))
+            assert abs(y[i, j] - (base + s * lora)) < 1e-11
+
+
+def test_linear_bwd_bruteforce_loops():
+    w, a, b, x, dy = _tiny_linear(1)
+    m, k = x.shape
+    n, r = b.shape
+    alpha = 4.0
+    s = alpha / r
+    dx, da, db = O.linear_bwd(w, a, b, x, dy, alpha, r)
+    u = [[sum(dy[i, j] * b[j, jr] for j in range(n)) for jr in range(r)] for i in range(m)]
+    t = [[sum(x[i, kk] * a[jr, kk] for kk in range(k)) for jr in range(r)] for i in range(m)]
+    for i in range(m):
+        for kk in range(k):
+            ref = sum(dy[i, j] * w[j, kk] for j in range(n)) + s * sum(u[i][jr] * a[jr, kk] for jr in range(r))
+            assert abs(dx[i, kk] - ref) < 1e-11
+    for jr in range(r):
+        for kk in range(k):
+            assert abs(da[jr, kk] - s * sum(u[i][jr] * x[i, kk] for i in range(m))) < 1e-11
+    for j in range(n):
+        for jr in range(r):
+            assert abs(db[j, jr] - s * sum(dy[i, j] * t[i][jr] for i in range(m))) < 1e-11
+
+
+def test_gradients_by_central_differences():
+    w, a, b, x, dy = _tiny_linear(2, m=3, n=5, k=7, r=2)
+    alpha, r = 2.0, 2
+
+    def loss(xx, aa, bb):
+        y, _ = O.linear_fwd(w, aa, bb, xx, alpha, r)
+        return float(np.sum(dy * y))
+
+    dx, da, db = O.linear_bwd(w, a, b, x, dy, alpha, r)
+    h = 1e-3
+    for arr, grad, which in ((x, dx, 0), (a, da, 1), (b, db, 2)):
+        for idx in np.ndindex(arr.shape):
+            p, mi = [x.copy(), a.copy(), b.copy()], [x.copy(), a.copy(), b.copy()]
+            p[which][idx] += h
+            mi[which][idx] -= h
+            fd = (loss(*p) - loss(*mi)) / (2 * h)
+            assert abs(fd - grad[idx]) < 1e-8 * max(1.0, abs(fd))
+
+
+def test_b_zero_reduces_to_base_layer():
+    w, a, b, x, dy = _tiny_linear(3)
+    b0 = np.zeros_like(b)
+    y, _ = O.linear_fwd(w, a, b0, x, 16.0, 2)
+    assert np.array_equal(y, x @ w.T)
+    dx, da, db = O.linear_bwd(w, a, b0, x, dy, 16.0, 2)
+    assert np.all(da == 0)
+    assert np.array_equal(dx, dy @ w)
+
+
+def test_w_zero_isolates_lora_path():
+    w, a, b, x, _ = _tiny_linear(4)
+    y, t = O.linear_fwd(np.zeros_like(w), a, b, x, 16.0, 2)
+    assert np.allclose(y, 8.0 * (x @ a.T) @ b.T, rtol=0, atol=1e-12)
+
+
+def test_merged_form_agrees():
+    w, a, b, x, _ = _tiny_linear(5, m=6, n=9, k=20, r=3)
+    y, _ = O.linear_fwd(w, a, b, x, 6.0, 3)
+    wm = O.merged_weight(w, a, b, 6.0, 3)
+    assert np.allclose(y, x @ wm.T, rtol=1e-13, atol=1e-13)
+
+
+def test_lora_scale_float32():
+    assert O.lora_scale(16.0, 8) == 2.0
+    assert O.lora_scale(16.0, 64) == 0.25
+    assert O.lora_scale(1.0, 3) == float(np.float32(1.0) / np.float32(3.0))
