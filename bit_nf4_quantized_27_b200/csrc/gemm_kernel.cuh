@@ -1,0 +1,460 @@
+// Persistent warp-specialised tcgen05 GEMM for sm_100a, with an NF4-dequantising
+// producer for the frozen weight operand and the rank-r LoRA product folded in as
+// extra K steps of the same accumulator.
+//
+//   D[M_rows, N_cols] = A (.) B^T  (+ A2 (.) B2^T)      fp32 accumulate in TMEM
+//
+// Operands are bf16 in 128-byte-swizzled shared memory.  A is always loaded by TMA
+// (K-major or MN-major); B is either loaded by TMA or produced by 8 "dequant"
+// warps from packed NF4 codes (TMA-staged) and the E4M3 block scales:
+//   w' = bf16_rne(fl32(L[code] * fl32(E4M3(q) * c2)))
+// exactly the dequantised weight of the glossary page's forward rule ("How QLoRA
+// works": dequantise to bfloat16 right before the matmul).  The forward pass uses
+// W' as a K-major B operand (rows = out features); the backward dX pass uses the
+// same tile as an MN-major B operand (rows = in features), so one decode routine
+// serves both.
+//
+// Roles (warp index):  0 TMA producer | 1 MMA issuer + TMEM owner |
+//                      4..7 epilogue (TMEM lane quadrants 0..3) | 8..15 dequant.
+// Every wait is bounded; a wait that gives up raises QLORA_ERR_TIMEOUT in the
+// status word, sets a CTA abort flag so the other roles leave too, drains the
+// copies and MMAs this CTA has in flight (again bounded) and frees TMEM.
+#pragma once
+
+#include "nf4_device.cuh"
+#include "sm100_ptx.cuh"
+
+namespace qlora {
+
+struct GemmArgs {
+  int M_rows;        // rows of D (tiles of 128 * MT)
+  int N_cols;        // cols of D (tiles of BN)
+  int k_steps;       // main K steps of 64
+  int lora_steps;    // extra K steps of 64 for the LoRA block (0 = none)
+  int lora_r;        // LoRA rank (bounds the B2 rows/cols read by the dequant warps)
+  // output 1 (required) and output 2 (optional, bf16)
+  void *out;
+  int64_t ldo;
+  int out_f32;       // 1: float32, 0: bf16
+  int out_transpose; // 1: out[col * ldo + row]
+  float out_scale;
+  void *out2;
+  int64_t ldo2;
+  float out2_scale;
+  // NF4 operand (B from dequant)
+  const uint8_t *scale_codes;
+  const float *c2;
+  int64_t w_rows;    // N of W
+  int64_t w_cols;    // K of W
+  const __nv_bfloat16 *lora_b2;  // B2 source read by the dequant warps (fwd: B [N, r]; bwd: A [r, K])
+  int64_t lora_ld;   // row stride of lora_b2 (elements)
+  uint32_t *status;
+};
+
+template <bool A_MN, bool B_MN, bool NF4, int BN, int MT>
+struct GemmCfg {
+  static constexpr int BM = 128;
+  static constexpr int BK = 64;
+  static constexpr int A_STAGE = MT * BM * BK * 2;
+  static constexpr int B_STAGE = BN * BK * 2;
+  static constexpr int C_STAGE = NF4 ? BN * 32 : 0;  // codes: 64 weights (32 B) per B row
+  static constexpr int SA = NF4 ? (MT == 1 ? 4 : 3) : 6;
+  static constexpr int SB = NF4 ? (MT == 1 ? 3 : 2) : SA;
+  static constexpr int SC = NF4 ? 4 : 1;
+  static constexpr int NUM_ACC = (2 * MT * BN <= 512) ? 2 : 1;
+  static constexpr int ACC_COLS = MT * BN;
+  static constexpr int TMEM_COLS = (NUM_ACC * ACC_COLS <= 32) ? 32 : (NUM_ACC * ACC_COLS <= 64) ? 64
+                                   : (NUM_ACC * ACC_COLS <= 128) ? 128 : (NUM_ACC * ACC_COLS <= 256) ? 256 : 512;
+  static constexpr int THREADS = NF4 ? 512 : 256;
+  static constexpr int SMEM_DATA = SA * A_STAGE + SB * B_STAGE + SC * C_STAGE;
+  static constexpr int SMEM_BYTES = SMEM_DATA + 1024 /*align*/ + 512 /*barriers*/;
+  static constexpr uint32_t IDESC = ptx::idesc_bf16(BM, BN, A_MN ? 1 : 0, B_MN ? 1 : 0);
+  static_assert(BN % 64 == 0 || (!NF4 && BN >= 16), "tile");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+
+// Byte offset of the 16-byte chunk `c` (0..7) of the 128-byte row `row` inside a
+// 1024-byte SW128 atom.
+__device__ __forceinline__ uint32_t sw128_row_chunk(uint32_t row, uint32_t c) {
+  return (row & 7u) * 128u + ((c ^ (row & 7u)) << 4);
+}
+
+// Decode 64 NF4 codes (two uint4 of packed nibbles) with block scale S into 32
+// packed bf16x2 words, via a per-block table of the 16 products split into byte
+// planes and looked up with byte permutes.
+__device__ __forceinline__ void nf4_decode64(const uint4 &c0, const uint4 &c1, float S, const float (&lv)[16],
+                                             uint32_t (&o)[32]) {
+  uint32_t p[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) p[j] = pack_bf16x2(__fmul_rn(lv[2 * j], S), __fmul_rn(lv[2 * j + 1], S));
+  // lo/hi byte planes of entries 0-3, 4-7, 8-11, 12-15
+  uint32_t lo[4], hi[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    lo[j] = __byte_perm(p[2 * j], p[2 * j + 1], 0x6420);
+    hi[j] = __byte_perm(p[2 * j], p[2 * j + 1], 0x7531);
+  }
+  const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const uint32_t sel32 = w[q] & 0x77777777u;
+    const uint32_t msel32 = 0x32103210u | ((w[q] >> 1) & 0x44444444u);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t sel = h ? (sel32 >> 16) : sel32;
+      const uint32_t msel = h ? (msel32 >> 16) : msel32;
+      const uint32_t la = __byte_perm(lo[0], lo[1], sel), lb = __byte_perm(lo[2], lo[3], sel);
+      const uint32_t ha = __byte_perm(hi[0], hi[1], sel), hb = __byte_perm(hi[2], hi[3], sel);
+      const uint32_t l = __byte_perm(la, lb, msel), hh = __byte_perm(ha, hb, msel);
+      o[q * 4 + h * 2 + 0] = __byte_perm(l, hh, 0x5140);
+      o[q * 4 + h * 2 + 1] = __byte_perm(l, hh, 0x7362);
+    }
+  }
+}
+
+__device__ __forceinline__ void store_row128(uint8_t *atom_base, uint32_t row, const uint32_t (&o)[32]) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    *reinterpret_cast<uint4 *>(atom_base + sw128_row_chunk(row, c)) =
+        make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+  }
+}
+
+// 64 bf16 (128 bytes) from global, zero where col >= ncols or !valid.
+__device__ __forceinline__ void load_row128(const __nv_bfloat16 *src, int valid_cols, uint32_t (&o)[32]) {
+  if (valid_cols >= 64) {
+    const uint4 *s = reinterpret_cast<const uint4 *>(src);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint4 v = __ldg(s + c);
+      o[4 * c] = v.x; o[4 * c + 1] = v.y; o[4 * c + 2] = v.z; o[4 * c + 3] = v.w;
+    }
+  } else {
+    const uint16_t *s = reinterpret_cast<const uint16_t *>(src);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const uint32_t a = (2 * i < valid_cols) ? __ldg(s + 2 * i) : 0u;
+      const uint32_t b = (2 * i + 1 < valid_cols) ? __ldg(s + 2 * i + 1) : 0u;
+      o[i] = a | (b << 16);
+    }
+  }
+}
+
+template <bool A_MN, bool B_MN, bool NF4, int BN, int MT>
+__global__ void __launch_bounds__(GemmCfg<A_MN, B_MN, NF4, BN, MT>::THREADS, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmCodes,
+               const GemmArgs args) {
+  using C = GemmCfg<A_MN, B_MN, NF4, BN, MT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sA = smem;
+  uint8_t *sB = sA + C::SA * C::A_STAGE;
+  uint8_t *sC = sB + C::SB * C::B_STAGE;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sC + C::SC * C::C_STAGE);
+  uint64_t *full_a = bars;
+  uint64_t *empty_a = full_a + C::SA;
+  uint64_t *full_b = empty_a + C::SA;
+  uint64_t *empty_b = full_b + C::SB;
+  uint64_t *full_c = empty_b + C::SB;
+  uint64_t *empty_c = full_c + C::SC;
+  uint64_t *acc_full = empty_c + C::SC;
+  uint64_t *acc_empty = acc_full + 2;
+  uint64_t *drain = acc_empty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::SA; ++s) { ptx::mbar_init(&full_a[s], 1); ptx::mbar_init(&empty_a[s], 1); }
+    for (int s = 0; s < C::SB; ++s) {
+      ptx::mbar_init(&full_b[s], NF4 ? 8 : 1);
+      ptx::mbar_init(&empty_b[s], 1);
+    }
+    for (int s = 0; s < C::SC; ++s) { ptx::mbar_init(&full_c[s], 1); ptx::mbar_init(&empty_c[s], 8); }
+    for (int s = 0; s < 2; ++s) { ptx::mbar_init(&acc_full[s], 1); ptx::mbar_init(&acc_empty[s], 4); }
+    ptx::mbar_init(drain, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    ptx::prefetch_tmap(&tmA);
+    if (!NF4) ptx::prefetch_tmap(&tmB);
+    if (args.lora_steps) ptx::prefetch_tmap(&tmA2);
+    if (NF4) ptx::prefetch_tmap(&tmCodes);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, C::TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_m = (args.M_rows + C::BM * MT - 1) / (C::BM * MT);
+  const int num_n = (args.N_cols + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
+  const int steps = args.k_steps + args.lora_steps;
+
+  auto fail = [&]() {
+    raise_status(args.status, QLORA_ERR_TIMEOUT);
+    *abort_flag = 1;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (ptx::elect_one()) {
+      uint32_t sa = 0, pa = 0, sc = 0, pc = 0;
+      int issued_a = 0, issued_c = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int m0 = (tile % num_m) * C::BM * MT;
+        const int n0 = (tile / num_m) * BN;
+        for (int ks = 0; ks < steps && ok; ++ks) {
+          const bool lora = ks >= args.k_steps;
+          if (NF4 && !lora) {
+            if (!ptx::mbar_wait(&empty_c[sc], pc ^ 1, abort_flag)) { ok = false; break; }
+            ptx::mbar_arrive_expect_tx(&full_c[sc], C::C_STAGE);
+            // fwd: rows n0.., 32 code bytes of K step ks; bwd: 64 rows of W, BN/2 code bytes
+            if (!B_MN) ptx::tma_load_2d(sC + sc * C::C_STAGE, &tmCodes, &full_c[sc], ks * 32, n0);
+            else ptx::tma_load_2d(sC + sc * C::C_STAGE, &tmCodes, &full_c[sc], n0 / 2, ks * 64);
+            ++issued_c;
+            if (++sc == C::SC) { sc = 0; pc ^= 1; }
+          }
+          if (!ptx::mbar_wait(&empty_a[sa], pa ^ 1, abort_flag)) { ok = false; break; }
+          const uint32_t bytes = C::A_STAGE + (NF4 ? 0 : C::B_STAGE);
+          ptx::mbar_arrive_expect_tx(&full_a[sa], bytes);
+          uint8_t *dA = sA + sa * C::A_STAGE;
+          if (lora) {
+            const int kk = (ks - args.k_steps) * 64;
+            for (int t = 0; t < MT; ++t) ptx::tma_load_2d(dA + t * 16384, &tmA2, &full_a[sa], kk, m0 + t * 128);
+          } else if (!A_MN) {
+            for (int t = 0; t < MT; ++t) ptx::tma_load_2d(dA + t * 16384, &tmA, &full_a[sa], ks * 64, m0 + t * 128);
+          } else {
+            for (int t = 0; t < MT * 2; ++t) ptx::tma_load_2d(dA + t * 8192, &tmA, &full_a[sa], m0 + t * 64, ks * 64);
+          }
+          if (!NF4) {
+            uint8_t *dB = sB + sa * C::B_STAGE;
+            if (!B_MN) {
+              ptx::tma_load_2d(dB, &tmB, &full_a[sa], ks * 64, n0);
+            } else {
+              for (int t = 0; t < BN / 64; ++t) ptx::tma_load_2d(dB + t * 8192, &tmB, &full_a[sa], n0 + t * 64, ks * 64);
+            }
+          }
+          ++issued_a;
+          if (++sa == C::SA) { sa = 0; pa ^= 1; }
+        }
+      }
+      if (!ok) {
+        fail();
+        // Drain: every issued copy completes its full barrier phase; wait for the
+        // last `SA` / `SC` of them (older ones were consumed already).
+        for (int i = 0; i < C::SA && i < issued_a; ++i) {
+          sa = (sa + C::SA - 1) % C::SA;
+          if (sa == C::SA - 1) pa ^= 1;
+          ptx::mbar_wait(&full_a[sa], pa, nullptr);
+        }
+        for (int i = 0; NF4 && i < C::SC && i < issued_c; ++i) {
+          sc = (sc + C::SC - 1) % C::SC;
+          if (sc == C::SC - 1) pc ^= 1;
+          ptx::mbar_wait(&full_c[sc], pc, nullptr);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (ptx::elect_one()) {
+      uint32_t sa = 0, pa = 0, sb = 0, pb = 0;
+      int it = 0;
+      bool ok = true;
+      const uint32_t sA0 = ptx::smem_addr(sA), sB0 = ptx::smem_addr(sB);
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+        const int acc = it % C::NUM_ACC;
+        const uint32_t acc_phase = (it / C::NUM_ACC) & 1;
+        if (!ptx::mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag)) { ok = false; break; }
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * C::ACC_COLS;
+        for (int ks = 0; ks < steps && ok; ++ks) {
+          const bool lora = ks >= args.k_steps;
+          if (!ptx::mbar_wait(&full_a[sa], pa, abort_flag)) { ok = false; break; }
+          if (NF4 && !ptx::mbar_wait(&full_b[sb], pb, abort_flag)) { ok = false; break; }
+          ptx::tc_fence_after();
+          const uint32_t a_base = sA0 + sa * C::A_STAGE;
+          const uint32_t b_base = sB0 + (NF4 ? sb : sa) * C::B_STAGE;
+          const bool a_mn = A_MN && !lora;  // the LoRA A2 block is K-major
+#pragma unroll
+          for (int k16 = 0; k16 < 4; ++k16) {
+            const uint64_t bd = B_MN ? ptx::smem_desc_sw128(b_base + k16 * 2048, 8192, 1024)
+                                     : ptx::smem_desc_sw128(b_base + k16 * 32, 16, 1024);
+#pragma unroll
+            for (int t = 0; t < MT; ++t) {
+              const uint64_t ad = a_mn ? ptx::smem_desc_sw128(a_base + t * 16384 + k16 * 2048, 8192, 1024)
+                                       : ptx::smem_desc_sw128(a_base + t * 16384 + k16 * 32, 16, 1024);
+              const uint32_t idesc = a_mn ? C::IDESC : (C::IDESC & ~(1u << 15));
+              ptx::mma_bf16(d_tmem + t * BN, ad, bd, idesc, (ks | k16) ? 1u : 0u);
+            }
+          }
+          ptx::mma_commit(&empty_a[sa]);
+          if (NF4) ptx::mma_commit(&empty_b[sb]);
+          if (++sa == C::SA) { sa = 0; pa ^= 1; }
+          if (NF4 && ++sb == C::SB) { sb = 0; pb ^= 1; }
+        }
+        if (ok) ptx::mma_commit(&acc_full[acc]);
+      }
+      if (!ok) fail();
+      // Wait until every MMA this thread issued has completed.
+      ptx::mma_commit(drain);
+      ptx::mbar_wait(drain, 0, nullptr);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp - 4;  // TMEM lane quadrant (warp % 4)
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      const int acc = it % C::NUM_ACC;
+      const uint32_t acc_phase = (it / C::NUM_ACC) & 1;
+      if (!ptx::mbar_wait(&acc_full[acc], acc_phase, abort_flag)) {
+        if (lane == 0) fail();
+        break;
+      }
+      ptx::tc_fence_after();
+      const int m0 = (tile % num_m) * C::BM * MT;
+      const int n0 = (tile / num_m) * BN;
+      for (int t = 0; t < MT; ++t) {
+        const int row = m0 + t * 128 + q * 32 + lane;
+        for (int cb = 0; cb < BN; cb += 32) {
+          uint32_t v[32];
+          ptx::tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS + t * BN + cb, v);
+          ptx::tmem_ld_wait();
+          const int col0 = n0 + cb;
+          if (row >= args.M_rows || col0 >= args.N_cols) continue;
+          const int ncol = min(32, args.N_cols - col0);
+          if (!args.out_transpose) {
+            if (args.out_f32) {
+              float *o = reinterpret_cast<float *>(args.out) + (int64_t)row * args.ldo + col0;
+              if (ncol == 32) {
+#pragma unroll
+                for (int j = 0; j < 32; j += 4)
+                  *reinterpret_cast<float4 *>(o + j) =
+                      make_float4(__uint_as_float(v[j]) * args.out_scale, __uint_as_float(v[j + 1]) * args.out_scale,
+                                  __uint_as_float(v[j + 2]) * args.out_scale, __uint_as_float(v[j + 3]) * args.out_scale);
+              } else {
+                for (int j = 0; j < ncol; ++j) o[j] = __uint_as_float(v[j]) * args.out_scale;
+              }
+            } else {
+              __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(args.out) + (int64_t)row * args.ldo + col0;
+              uint32_t pk[16];
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]) * args.out_scale,
+                                    __uint_as_float(v[2 * j + 1]) * args.out_scale);
+              if (ncol == 32) {
+#pragma unroll
+                for (int j = 0; j < 16; j += 4)
+                  *reinterpret_cast<uint4 *>(o + 2 * j) = make_uint4(pk[j], pk[j + 1], pk[j + 2], pk[j + 3]);
+              } else {
+                uint16_t *o16 = reinterpret_cast<uint16_t *>(o);
+                for (int j = 0; j < ncol; ++j) o16[j] = (j & 1) ? (pk[j >> 1] >> 16) : (pk[j >> 1] & 0xffffu);
+              }
+            }
+            if (args.out2) {
+              uint16_t *o2 = reinterpret_cast<uint16_t *>(args.out2) + (int64_t)row * args.ldo2 + col0;
+              for (int j = 0; j < ncol; j += 2) {
+                const uint32_t pk = pack_bf16x2(__uint_as_float(v[j]) * args.out2_scale,
+                                                __uint_as_float(v[min(j + 1, 31)]) * args.out2_scale);
+                o2[j] = pk & 0xffffu;
+                if (j + 1 < ncol) o2[j + 1] = pk >> 16;
+              }
+            }
+          } else {
+            // out[col * ldo + row]: lanes write consecutive rows of each column.
+            for (int j = 0; j < ncol; ++j) {
+              const float x = __uint_as_float(v[j]) * args.out_scale;
+              if (args.out_f32) reinterpret_cast<float *>(args.out)[(int64_t)(col0 + j) * args.ldo + row] = x;
+              else reinterpret_cast<__nv_bfloat16 *>(args.out)[(int64_t)(col0 + j) * args.ldo + row] = __float2bfloat16_rn(x);
+            }
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&acc_empty[acc]);
+    }
+  } else if (NF4 && warp >= 8) {
+    // ------------------------------------------------------------ dequant producer
+    const int d = threadIdx.x - 256;  // 0..255
+    float lv[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) lv[j] = __uint_as_float(kNf4LevelBits[j]);
+    const int64_t kblocks = args.w_cols / 64;
+    uint32_t sb = 0, pb = 0, sc = 0, pc = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      const int n0 = (tile / num_m) * BN;
+      for (int ks = 0; ks < steps && ok; ++ks) {
+        const bool lora = ks >= args.k_steps;
+        uint32_t o[32];
+        // Which 128-byte row of which SW128 atom this thread fills.
+        uint32_t atom_off, row_in;
+        if (!B_MN) {  // B[n, k]: thread = W row n0 + d, one 64-code block (K step ks)
+          atom_off = (d >> 3) * 1024;
+          row_in = d & 7;
+        } else {      // B[kf, n]: thread = (W row ks*64 + d/4, 64 in-features block d%4)
+          const int nl = d >> 2, a = d & 3;
+          atom_off = a * 8192 + (nl >> 3) * 1024;
+          row_in = nl & 7;
+        }
+        if (!lora) {
+          if (!ptx::mbar_wait(&full_c[sc], pc, abort_flag)) { ok = false; break; }
+          const uint8_t *cs = sC + sc * C::C_STAGE + d * 32;
+          const uint4 c0 = *reinterpret_cast<const uint4 *>(cs);
+          const uint4 c1 = *reinterpret_cast<const uint4 *>(cs + 16);
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&empty_c[sc]);
+          if (++sc == C::SC) { sc = 0; pc ^= 1; }
+          int64_t wrow, kblk;
+          if (!B_MN) { wrow = n0 + d; kblk = ks; }
+          else { wrow = (int64_t)ks * 64 + (d >> 2); kblk = n0 / 64 + (d & 3); }
+          if (wrow < args.w_rows && kblk < kblocks) {
+            const float S = block_scale(args.scale_codes, args.c2, wrow * kblocks + kblk);
+            nf4_decode64(c0, c1, S, lv, o);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = 0u;
+          }
+        } else {
+          const int j0 = (ks - args.k_steps) * 64;
+          if (!B_MN) {  // fwd: B2 = lora B [N, r], row n0 + d, cols j0..j0+63
+            const int64_t n = n0 + d;
+            if (n < args.w_rows) load_row128(args.lora_b2 + n * args.lora_ld + j0, args.lora_r - j0, o);
+            else for (int j = 0; j < 32; ++j) o[j] = 0u;
+          } else {      // bwd: B2 = lora A [r, K], row j0 + d/4, cols n0 + 64*(d%4) ..
+            const int jr = j0 + (d >> 2);
+            const int64_t kf = n0 + 64 * (d & 3);
+            if (jr < args.lora_r && kf < args.w_cols) load_row128(args.lora_b2 + (int64_t)jr * args.lora_ld + kf, 64, o);
+            else for (int j = 0; j < 32; ++j) o[j] = 0u;
+          }
+        }
+        if (!ptx::mbar_wait(&empty_b[sb], pb ^ 1, abort_flag)) { ok = false; break; }
+        store_row128(sB + sb * C::B_STAGE + atom_off, row_in, o);
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&full_b[sb]);
+        if (++sb == C::SB) { sb = 0; pb ^= 1; }
+      }
+    }
+    if (!ok && lane == 0) fail();
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace qlora

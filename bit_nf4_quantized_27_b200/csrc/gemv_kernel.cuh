@@ -1,0 +1,332 @@
+// Small-M (decode-shaped) forward of the NF4 linear layer with LoRA, M <= 16:
+//   Y [M, N] = X W'^T + (s T) B^T,   T = X A^T computed by lora_down_small_kernel.
+//
+// HBM-bound: the packed codes (0.5 B/weight) dominate the traffic, so the kernel
+// streams them straight from HBM into registers with 8-byte vector loads and
+// decodes in registers.  Each byte (two codes) indexes a 256-entry table of bf16
+// level pairs (L[lo], L[hi]) kept in shared memory with one copy per lane (each
+// lane reads its own bank, so lookups never conflict); the pair is directly one
+// register of an m16n8k16 tensor-core A fragment (rows = 16 weight rows).  The
+// per-block scale S' = E4M3(q) * c2 multiplies the fp32 partial of each 64-weight
+// block after its four MMAs, so the sum equals X W'^T up to the bf16 rounding of
+// the products L * S' (the dequantised weight is bf16(L * S'); here L is exact in
+// the table and S' is applied in fp32).
+//
+// Work split: 16 warps per CTA; warp w owns the w-th 256-wide slice of each
+// 4096-wide K chunk and keeps that slice of X as MMA B fragments in registers.  The
+// mapping of fragment registers to k inside a 64-block is permuted (thread quad q
+// owns k in [16q, 16q+16) of every block) identically for W and X, which leaves
+// the dot products unchanged and lets each thread load 8 contiguous code bytes per
+// row and block.  Each CTA owns a set of 16-row groups; per-warp partials land in
+// shared memory and are summed in a fixed order (deterministic).
+#pragma once
+
+#include "nf4_device.cuh"
+
+namespace qlora {
+
+constexpr int kGemvMaxM = 16;
+constexpr int kGemvWarps = 16;
+constexpr int kGemvThreads = kGemvWarps * 32;
+constexpr int kGemvMaxRG = 10;  // row groups of 16 per CTA
+
+struct GemvArgs {
+  const uint8_t *codes;
+  const uint8_t *scale_codes;
+  const float *c2;
+  int64_t N, K;
+  int M;
+  const __nv_bfloat16 *X;   // [M, K]
+  const __nv_bfloat16 *sT;  // [M, r]  s * X A^T
+  const __nv_bfloat16 *B;   // [N, r]
+  int r;
+  void *Y;
+  int y_f32;
+  float *partial;           // unused scratch slot (reserved)
+  uint32_t *status;
+  int rg_per_cta;
+};
+
+inline size_t gemv_workspace_bytes(int64_t, int64_t, int64_t) { return 0; }
+
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// smem: table [256][32] u32 | red [rg][16 warps][16 rows][16 tokens] f32
+template <int NG>
+__global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_lora_kernel(const GemvArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint32_t *lut = reinterpret_cast<uint32_t *>(smem_raw);
+  float *red = reinterpret_cast<float *>(smem_raw + 256 * 32 * 4);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, q = lane & 3;
+
+  // Pair table: entry v = (bf16 L[v & 15]) | (bf16 L[v >> 4]) << 16, one copy per lane.
+  for (int i = tid; i < 256 * 32; i += kGemvThreads) {
+    const int v = i >> 5;
+    const float lo = __uint_as_float(kNf4LevelBits[v & 15]), hi = __uint_as_float(kNf4LevelBits[v >> 4]);
+    lut[i] = pack_bf16x2(lo, hi);
+  }
+  const int num_rg = static_cast<int>((a.N + 15) / 16);
+  const int rg0 = blockIdx.x * a.rg_per_cta;
+  const int my_rg = max(0, min(a.rg_per_cta, num_rg - rg0));
+  for (int i = tid; i < my_rg * kGemvWarps * 256; i += kGemvThreads) red[i] = 0.0f;
+  __syncthreads();
+
+  const int64_t nbk = a.K / 64;            // blocks per row
+  const int64_t row_bytes = a.K / 2;
+  const uint32_t lut_lane = static_cast<uint32_t>(__cvta_generic_to_shared(lut)) + lane * 4;
+  const int nchunks = static_cast<int>((nbk + 63) / 64);
+
+  for (int ch = 0; ch < nchunks; ++ch) {
+    const int64_t kb0 = (int64_t)ch * 64 + warp * 4;  // first block of this warp's quad
+    if (kb0 >= nbk) continue;
+    const int nblk = static_cast<int>(nbk - kb0 < 4 ? nbk - kb0 : 4);
+    // X fragments: token (g + 8*ng), k = kb*64 + 16q + 4s + {0..3}
+    uint32_t xf[4][4][NG][2];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int ng = 0; ng < NG; ++ng) {
+        const int t = g + 8 * ng;
+        uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+        if (j < nblk && t < a.M) {
+          const uint4 *src = reinterpret_cast<const uint4 *>(a.X + (int64_t)t * a.K + (kb0 + j) * 64 + 16 * q);
+          v0 = __ldg(src);
+          v1 = __ldg(src + 1);
+        }
+        xf[j][0][ng][0] = v0.x; xf[j][0][ng][1] = v0.y;
+        xf[j][1][ng][0] = v0.z; xf[j][1][ng][1] = v0.w;
+        xf[j][2][ng][0] = v1.x; xf[j][2][ng][1] = v1.y;
+        xf[j][3][ng][0] = v1.z; xf[j][3][ng][1] = v1.w;
+      }
+
+    // Software pipeline over this CTA's row groups: codes of the next group are
+    // loaded while the current one is decoded.
+    uint2 cur[4][2], nxt[4][2];
+    auto load_codes = [&](int i, uint2 (&dst)[4][2]) {
+      const int64_t n0 = (int64_t)(rg0 + i) * 16;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int64_t row = n0 + g + 8 * h;
+          if (j < nblk && row < a.N)
+            dst[j][h] = __ldg(reinterpret_cast<const uint2 *>(a.codes + row * row_bytes + (kb0 + j) * 32 + 8 * q));
+          else
+            dst[j][h] = make_uint2(0x77777777u, 0x77777777u);
+        }
+    };
+    if (my_rg > 0) load_codes(0, cur);
+    for (int i = 0; i < my_rg; ++i) {
+      if (i + 1 < my_rg) load_codes(i + 1, nxt);
+      const int64_t n0 = (int64_t)(rg0 + i) * 16;
+      float part[NG][4];
+#pragma unroll
+      for (int ng = 0; ng < NG; ++ng) part[ng][0] = part[ng][1] = part[ng][2] = part[ng][3] = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (j >= nblk) break;
+        float S[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int64_t row = n0 + g + 8 * h;
+          S[h] = row < a.N ? block_scale(a.scale_codes, a.c2, row * nbk + kb0 + j) : 0.0f;
+        }
+        float acc[NG][4];
+#pragma unroll
+        for (int ng = 0; ng < NG; ++ng) acc[ng][0] = acc[ng][1] = acc[ng][2] = acc[ng][3] = 0.0f;
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          // bytes 2s, 2s+1 of the 8 code bytes of rows g (h=0) and g+8 (h=1)
+          const uint32_t w0 = (s < 2) ? cur[j][0].x : cur[j][0].y;
+          const uint32_t w1 = (s < 2) ? cur[j][1].x : cur[j][1].y;
+          const int sh = (s & 1) * 16;
+          const uint32_t b00 = (w0 >> sh) & 0xffu, b01 = (w0 >> (sh + 8)) & 0xffu;
+          const uint32_t b10 = (w1 >> sh) & 0xffu, b11 = (w1 >> (sh + 8)) & 0xffu;
+          uint32_t a0, a1, a2, a3;
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a0) : "r"(lut_lane + (b00 << 7)));
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a1) : "r"(lut_lane + (b10 << 7)));
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a2) : "r"(lut_lane + (b01 << 7)));
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a3) : "r"(lut_lane + (b11 << 7)));
+#pragma unroll
+          for (int ng = 0; ng < NG; ++ng) mma_16816(acc[ng], a0, a1, a2, a3, xf[j][s][ng][0], xf[j][s][ng][1]);
+        }
+#pragma unroll
+        for (int ng = 0; ng < NG; ++ng) {
+          part[ng][0] = fmaf(S[0], acc[ng][0], part[ng][0]);
+          part[ng][1] = fmaf(S[0], acc[ng][1], part[ng][1]);
+          part[ng][2] = fmaf(S[1], acc[ng][2], part[ng][2]);
+          part[ng][3] = fmaf(S[1], acc[ng][3], part[ng][3]);
+        }
+      }
+      // red[i][warp][row][token] += partial (this warp is the only writer)
+      float *rb = red + ((size_t)i * kGemvWarps + warp) * 256;
+#pragma unroll
+      for (int ng = 0; ng < NG; ++ng) {
+        const int t = 2 * q + 8 * ng;
+        rb[g * 16 + t] += part[ng][0];
+        rb[g * 16 + t + 1] += part[ng][1];
+        rb[(g + 8) * 16 + t] += part[ng][2];
+        rb[(g + 8) * 16 + t + 1] += part[ng][3];
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) { cur[j][0] = nxt[j][0]; cur[j][1] = nxt[j][1]; }
+    }
+  }
+
+  // LoRA up-projection on tensor cores: rows = 16 weight rows (A = B_lora rows),
+  // cols = tokens (B = (s T)^T), K = r.  Needs s T from the preceding kernel.
+  griddep_wait();
+  for (int i = warp; i < my_rg; i += kGemvWarps) {
+    const int64_t n0 = (int64_t)(rg0 + i) * 16;
+    float acc[NG][4];
+#pragma unroll
+    for (int ng = 0; ng < NG; ++ng) acc[ng][0] = acc[ng][1] = acc[ng][2] = acc[ng][3] = 0.0f;
+    for (int j0 = 0; j0 < a.r; j0 += 16) {
+      // A fragment: rows g / g+8, k = j0 + 2q + {0,1} and j0 + 8 + 2q + {0,1}
+      uint32_t af[4];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int64_t row = n0 + g + 8 * h;
+        const uint32_t *src = reinterpret_cast<const uint32_t *>(a.B + row * a.r + j0 + 2 * q);
+        af[h] = row < a.N ? __ldg(src) : 0u;
+        af[2 + h] = row < a.N ? __ldg(src + 4) : 0u;
+      }
+#pragma unroll
+      for (int ng = 0; ng < NG; ++ng) {
+        const int t = g + 8 * ng;
+        uint32_t b0 = 0, b1 = 0;
+        if (t < a.M) {
+          const uint32_t *src = reinterpret_cast<const uint32_t *>(a.sT + (int64_t)t * a.r + j0 + 2 * q);
+          b0 = __ldg(src);
+          b1 = __ldg(src + 4);
+        }
+        mma_16816(acc[ng], af[0], af[1], af[2], af[3], b0, b1);
+      }
+    }
+    float *rb = red + ((size_t)i * kGemvWarps + warp) * 256;
+#pragma unroll
+    for (int ng = 0; ng < NG; ++ng) {
+      const int t = 2 * q + 8 * ng;
+      rb[g * 16 + t] += acc[ng][0];
+      rb[g * 16 + t + 1] += acc[ng][1];
+      rb[(g + 8) * 16 + t] += acc[ng][2];
+      rb[(g + 8) * 16 + t + 1] += acc[ng][3];
+    }
+  }
+  __syncthreads();
+
+  // Deterministic reduction over the 16 warps and store.
+  for (int idx = tid; idx < my_rg * 256; idx += kGemvThreads) {
+    const int i = idx >> 8, e = idx & 255, row = e >> 4, t = e & 15;
+    const int64_t n = (int64_t)(rg0 + i) * 16 + row;
+    if (t >= a.M || n >= a.N) continue;
+    const float *rb = red + (size_t)i * kGemvWarps * 256 + e;
+    float sum = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kGemvWarps; ++w) sum += rb[w * 256];
+    if (a.y_f32) reinterpret_cast<float *>(a.Y)[(int64_t)t * a.N + n] = sum;
+    else reinterpret_cast<__nv_bfloat16 *>(a.Y)[(int64_t)t * a.N + n] = __float2bfloat16_rn(sum);
+  }
+}
+
+// T = X A^T for M <= 16 tokens: one CTA per LoRA rank row j; the CTA's threads
+// stride over K, then reduce.  Writes s*T (bf16) and optionally T (bf16).
+__global__ void __launch_bounds__(256) lora_down_small_kernel(const __nv_bfloat16 *__restrict__ X,
+                                                              const __nv_bfloat16 *__restrict__ A, int M,
+                                                              int64_t K, int r, float s,
+                                                              __nv_bfloat16 *__restrict__ sT,
+                                                              __nv_bfloat16 *__restrict__ T_out) {
+  griddep_launch_dependents();
+  __shared__ float red[8][kGemvMaxM];
+  const int j = blockIdx.x;
+  const int tid = threadIdx.x;
+  float acc[kGemvMaxM];
+#pragma unroll
+  for (int t = 0; t < kGemvMaxM; ++t) acc[t] = 0.0f;
+  for (int64_t k = (int64_t)tid * 8; k < K; k += 256 * 8) {
+    const uint4 av = __ldg(reinterpret_cast<const uint4 *>(A + (int64_t)j * K + k));
+    const float af[8] = {bf16lo_to_f32(av.x), bf16hi_to_f32(av.x), bf16lo_to_f32(av.y), bf16hi_to_f32(av.y),
+                         bf16lo_to_f32(av.z), bf16hi_to_f32(av.z), bf16lo_to_f32(av.w), bf16hi_to_f32(av.w)};
+#pragma unroll
+    for (int t = 0; t < kGemvMaxM; ++t) {
+      if (t < M) {
+        const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(X + (int64_t)t * K + k));
+        acc[t] = fmaf(af[0], bf16lo_to_f32(xv.x), acc[t]);
+        acc[t] = fmaf(af[1], bf16hi_to_f32(xv.x), acc[t]);
+        acc[t] = fmaf(af[2], bf16lo_to_f32(xv.y), acc[t]);
+        acc[t] = fmaf(af[3], bf16hi_to_f32(xv.y), acc[t]);
+        acc[t] = fmaf(af[4], bf16lo_to_f32(xv.z), acc[t]);
+        acc[t] = fmaf(af[5], bf16hi_to_f32(xv.z), acc[t]);
+        acc[t] = fmaf(af[6], bf16lo_to_f32(xv.w), acc[t]);
+        acc[t] = fmaf(af[7], bf16hi_to_f32(xv.w), acc[t]);
+      }
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < kGemvMaxM; ++t) {
+    float v = acc[t];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if ((tid & 31) == 0) red[tid >> 5][t] = v;
+  }
+  __syncthreads();
+  if (tid < M) {
+    float v = 0.0f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) v += red[w][tid];
+    sT[(int64_t)tid * r + j] = __float2bfloat16_rn(v * s);
+    if (T_out) T_out[(int64_t)tid * r + j] = __float2bfloat16_rn(v);
+  }
+}
+
+inline qlora_status launch_gemv(GemvArgs g, int dev, int sms, cudaStream_t st) {
+  const int num_rg = static_cast<int>((g.N + 15) / 16);
+  int per = (num_rg + sms - 1) / sms;
+  if (per > kGemvMaxRG) per = kGemvMaxRG;
+  g.rg_per_cta = per;
+  const int grid = (num_rg + per - 1) / per;
+  const int smem = 256 * 32 * 4 + per * kGemvWarps * 256 * 4;
+  static std::once_flag flags[2][64];
+  static qlora_status results[2][64];
+  const bool two = g.M > 8;
+  auto kernel = two ? nf4_gemv_lora_kernel<2> : nf4_gemv_lora_kernel<1>;
+  std::call_once(flags[two][dev], [&] {
+    results[two][dev] = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             256 * 32 * 4 + kGemvMaxRG * kGemvWarps * 256 * 4) == cudaSuccess
+                            ? QLORA_OK
+                            : QLORA_ERR_CUDA;
+    cudaGetLastError();
+  });
+  if (results[two][dev] != QLORA_OK) return results[two][dev];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGemvThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, g);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  return QLORA_OK;
+}
+
+}  // namespace qlora

@@ -1,0 +1,56 @@
+// Device-side helpers shared by the NF4 kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "qlora_nf4.h"
+
+namespace qlora {
+
+constexpr int kBlock = QLORA_BLOCK;  // weights per absmax block
+constexpr int kGroup = QLORA_GROUP;  // blocks per second-level group
+
+// The 16 NF4 levels as float32 bit patterns: Phi^-1 at the quantile offsets of the
+// QLoRA glossary page's snippet ("How QLoRA works"; offset 0.9677083, 8 positive and
+// 7 negative quantiles plus an exact zero, sorted, divided by the largest), each
+// evaluated in exact arithmetic and rounded once to float32.
+__constant__ uint32_t kNf4LevelBits[16] = {
+    0xbf800000u, 0xbf3239b3u, 0xbf066b30u, 0xbeca32a0u, 0xbe91a24cu, 0xbe3d353fu,
+    0xbdba786bu, 0x00000000u, 0x3da2fb03u, 0x3e24cae1u, 0x3e7c04dcu, 0x3ead0338u,
+    0x3ee1a4b7u, 0x3f1007aau, 0x3f3913b1u, 0x3f800000u};
+
+// Device status word flags (bit k set <=> status code k was raised).
+__device__ __forceinline__ void raise_status(uint32_t *status, qlora_status code) {
+  if (status) atomicOr(status, 1u << static_cast<uint32_t>(code));
+}
+
+// E4M3 byte -> float32 (exact: every E4M3 value is a half value).
+__device__ __forceinline__ float e4m3_to_f32(uint8_t q) {
+  __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(q), __NV_E4M3);
+  return __half2float(__half(h));
+}
+
+// float32 -> E4M3 byte, round to nearest even, saturating to +-448.
+__device__ __forceinline__ uint8_t f32_to_e4m3(float x) {
+  return static_cast<uint8_t>(__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3));
+}
+
+// Two float32 -> packed bf16x2 (lo in bits 0..15), round to nearest even.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ float bf16lo_to_f32(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16hi_to_f32(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+// Dequantised block scale S' = fl32(E4M3(q) * c2).
+__device__ __forceinline__ float block_scale(const uint8_t *scale_codes, const float *c2, int64_t b) {
+  return __fmul_rn(e4m3_to_f32(__ldg(scale_codes + b)), __ldg(c2 + (b >> 8)));
+}
+
+}  // namespace qlora

@@ -1,0 +1,410 @@
+// C ABI of the NF4 frozen-linear + LoRA library (see include/qlora_nf4.h).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "gemm_kernel.cuh"
+#include "gemv_kernel.cuh"
+#include "host_common.h"
+#include "qlora_nf4.h"
+#include "quant_kernels.cuh"
+
+using namespace qlora;
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// Tensor maps (driver entry point fetched through the runtime: no link-time
+// dependency on libcuda).
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void *p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [outer, inner] with row stride `ld` elements.
+bool make_tmap(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, uint32_t esize, uint64_t inner,
+               uint64_t outer, uint64_t ld, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  std::memset(m, 0, sizeof(*m));
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {ld * esize};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool tmap_bf16(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
+               uint32_t box_outer) {
+  return make_tmap(m, ptr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, inner, outer, inner, box_inner, box_outer, true);
+}
+
+// Once per device and kernel: allow the kernel's dynamic shared memory.
+template <typename F>
+qlora_status set_smem(F kernel, int bytes, int dev, std::once_flag *flags, qlora_status *results) {
+  std::call_once(flags[dev], [&] {
+    results[dev] = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess
+                       ? QLORA_OK
+                       : QLORA_ERR_CUDA;
+    cudaGetLastError();
+  });
+  return results[dev];
+}
+
+template <bool A_MN, bool B_MN, bool NF4, int BN, int MT>
+qlora_status launch_gemm(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmA2,
+                         const CUtensorMap &tmCodes, const GemmArgs &args, int dev, int sms, cudaStream_t st) {
+  using C = GemmCfg<A_MN, B_MN, NF4, BN, MT>;
+  auto kernel = gemm_tc_kernel<A_MN, B_MN, NF4, BN, MT>;
+  static std::once_flag flags[64];
+  static qlora_status results[64];
+  qlora_status s = set_smem(kernel, C::SMEM_BYTES, dev, flags, results);
+  if (s != QLORA_OK) return s;
+  const int num_m = (args.M_rows + C::BM * MT - 1) / (C::BM * MT);
+  const int num_n = (args.N_cols + BN - 1) / BN;
+  const int tiles = num_m * num_n;
+  const int grid = std::max(1, std::min(tiles, sms));
+  kernel<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tmA, tmB, tmA2, tmCodes, args);
+  return launch_status();
+}
+
+uint32_t *status_ptr(void *ws) { return reinterpret_cast<uint32_t *>(ws); }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+qlora_status check_lora(const qlora_lora *ad) {
+  if (!ad || !ad->A || !ad->B) return QLORA_ERR_INVALID_ARGUMENT;
+  if (ad->r < 8 || ad->r > QLORA_MAX_RANK || ad->r % 8) return QLORA_ERR_INVALID_ARGUMENT;
+  if (!std::isfinite(ad->alpha)) return QLORA_ERR_INVALID_ARGUMENT;
+  if (!aligned(ad->A, 16) || !aligned(ad->B, 16)) return QLORA_ERR_MISALIGNED;
+  return QLORA_OK;
+}
+
+bool valid_dtype(qlora_dtype d) { return d == QLORA_F32 || d == QLORA_BF16; }
+
+// T = X A^T for the tokens: writes s*T (bf16) to sT and, if T_out, T (bf16).
+qlora_status run_lora_down(const void *X, const qlora_lora *ad, int64_t M, int64_t K, float s, void *sT,
+                           void *T_out, uint32_t *status, int dev, int sms, cudaStream_t st) {
+  CUtensorMap tmX, tmA;
+  if (!tmap_bf16(&tmX, X, K, M, 64, 128) || !tmap_bf16(&tmA, ad->A, K, ad->r, 64, 64)) return QLORA_ERR_CUDA;
+  GemmArgs g{};
+  g.M_rows = (int)M;
+  g.N_cols = ad->r;
+  g.k_steps = (int)(K / 64);
+  g.out = sT;
+  g.ldo = ad->r;
+  g.out_f32 = 0;
+  g.out_scale = s;
+  g.out2 = T_out;
+  g.ldo2 = ad->r;
+  g.out2_scale = 1.0f;
+  g.status = status;
+  return launch_gemm<false, false, false, 64, 1>(tmX, tmA, tmX, tmX, g, dev, sms, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int qlora_abi_version(void) { return QLORA_NF4_ABI_VERSION; }
+
+void qlora_nf4_codebook(float out[16]) {
+  if (!out) return;
+  const float *lv = nf4_levels_host();
+  for (int i = 0; i < 16; ++i) out[i] = lv[i];
+}
+
+size_t qlora_nf4_storage_bytes(int64_t rows, int64_t cols, size_t *codes_bytes, size_t *scale_codes_bytes,
+                               size_t *c2_bytes) {
+  if (rows <= 0 || cols <= 0 || cols % QLORA_BLOCK) return 0;
+  const size_t n = static_cast<size_t>(rows) * static_cast<size_t>(cols);
+  const size_t nb = n / QLORA_BLOCK;
+  const size_t ng = (nb + QLORA_GROUP - 1) / QLORA_GROUP;
+  if (codes_bytes) *codes_bytes = n / 2;
+  if (scale_codes_bytes) *scale_codes_bytes = nb;
+  if (c2_bytes) *c2_bytes = ng * sizeof(float);
+  return n / 2 + nb + ng * sizeof(float);
+}
+
+size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r, int for_backward) {
+  if (M <= 0 || N <= 0 || K <= 0 || r <= 0 || r > QLORA_MAX_RANK) return 0;
+  const size_t mr = align256(static_cast<size_t>(M) * r * 2);  // one bf16 [M, r] buffer
+  size_t bytes = QLORA_STATUS_BYTES;
+  if (!for_backward) {
+    bytes += mr;                                    // s*T
+    if (M <= kGemvMaxM) bytes += gemv_workspace_bytes(M, N, K);
+  } else {
+    bytes += 2 * mr;                                // s*U, recomputed T
+  }
+  return bytes;
+}
+
+qlora_status qlora_nf4_quantize(const void *W, qlora_dtype w_dtype, const qlora_nf4_tensor *out, void *ws,
+                                qlora_stream_t stream) {
+  qlora_status s = check_nf4(out);
+  if (s != QLORA_OK) return s;
+  if (!W || !ws) return QLORA_ERR_INVALID_ARGUMENT;
+  if (!valid_dtype(w_dtype)) return QLORA_ERR_INVALID_ARGUMENT;
+  if (!aligned(W, 16) || !aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
+  int dev, sms;
+  if ((s = check_device(&dev, &sms)) != QLORA_OK) return s;
+  const HostCellTable &ht = cell_table();
+  if (!ht.ok) return QLORA_ERR_CUDA;
+  CodeCellTable t;
+  std::memcpy(t.thr, ht.thr, sizeof(t.thr));
+  std::memcpy(t.base, ht.base, sizeof(t.base));
+  const int64_t nb = out->rows * out->cols / QLORA_BLOCK;
+  const int64_t ng = (nb + QLORA_GROUP - 1) / QLORA_GROUP;
+  if (ng > 0x7fffffff) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (w_dtype == QLORA_BF16)
+    nf4_quantize_kernel<__nv_bfloat16><<<(unsigned)ng, kQuantThreads, 0, st>>>(
+        static_cast<const __nv_bfloat16 *>(W), nb, out->codes, out->scale_codes, out->c2, status_ptr(ws), t);
+  else
+    nf4_quantize_kernel<float><<<(unsigned)ng, kQuantThreads, 0, st>>>(
+        static_cast<const float *>(W), nb, out->codes, out->scale_codes, out->c2, status_ptr(ws), t);
+  return launch_status();
+}
+
+qlora_status qlora_nf4_dequantize(const qlora_nf4_tensor *w, void *W_out, qlora_dtype out_dtype,
+                                  qlora_stream_t stream) {
+  qlora_status s = check_nf4(w);
+  if (s != QLORA_OK) return s;
+  if (!W_out || !valid_dtype(out_dtype)) return QLORA_ERR_INVALID_ARGUMENT;
+  if (!aligned(W_out, 16)) return QLORA_ERR_MISALIGNED;
+  int dev, sms;
+  if ((s = check_device(&dev, &sms)) != QLORA_OK) return s;
+  const int64_t nchunks = w->rows * w->cols / 32;
+  const int64_t want = (nchunks + kDequantThreads - 1) / kDequantThreads;
+  const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)sms * 16));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (out_dtype == QLORA_BF16)
+    nf4_dequantize_kernel<__nv_bfloat16><<<grid, kDequantThreads, 0, st>>>(
+        w->codes, w->scale_codes, w->c2, nchunks, static_cast<__nv_bfloat16 *>(W_out));
+  else
+    nf4_dequantize_kernel<float><<<grid, kDequantThreads, 0, st>>>(w->codes, w->scale_codes, w->c2, nchunks,
+                                                                   static_cast<float *>(W_out));
+  return launch_status();
+}
+
+qlora_status qlora_linear_fwd(const qlora_nf4_tensor *W, const qlora_lora *ad, const void *X, int64_t M, void *Y,
+                              qlora_dtype y_dtype, void *T_save, void *ws, size_t ws_bytes,
+                              qlora_stream_t stream) {
+  qlora_status s = check_nf4(W);
+  if (s != QLORA_OK) return s;
+  if ((s = check_lora(ad)) != QLORA_OK) return s;
+  if (!X || !Y || !ws || M < 1 || M > (int64_t(1) << 30) || !valid_dtype(y_dtype)) return QLORA_ERR_INVALID_ARGUMENT;
+  if (W->rows % 8) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(ws, 256) || (T_save && !aligned(T_save, 16)))
+    return QLORA_ERR_MISALIGNED;
+  const int64_t N = W->rows, K = W->cols;
+  if (ws_bytes < qlora_workspace_bytes(M, N, K, ad->r, 0)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  int dev, sms;
+  if ((s = check_device(&dev, &sms)) != QLORA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const float sc = ad->alpha / static_cast<float>(ad->r);
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  void *sT = wsb + QLORA_STATUS_BYTES;
+  const size_t mr = align256(static_cast<size_t>(M) * ad->r * 2);
+
+  if (M <= kGemvMaxM) {
+    lora_down_small_kernel<<<ad->r, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(X),
+                                                  static_cast<const __nv_bfloat16 *>(ad->A), (int)M, K, ad->r, sc,
+                                                  static_cast<__nv_bfloat16 *>(sT),
+                                                  static_cast<__nv_bfloat16 *>(T_save));
+    if ((s = launch_status()) != QLORA_OK) return s;
+    GemvArgs g{};
+    g.codes = W->codes; g.scale_codes = W->scale_codes; g.c2 = W->c2;
+    g.N = N; g.K = K; g.M = (int)M;
+    g.X = static_cast<const __nv_bfloat16 *>(X);
+    g.sT = static_cast<const __nv_bfloat16 *>(sT);
+    g.B = static_cast<const __nv_bfloat16 *>(ad->B);
+    g.r = ad->r;
+    g.Y = Y; g.y_f32 = y_dtype == QLORA_F32;
+    g.partial = reinterpret_cast<float *>(wsb + QLORA_STATUS_BYTES + mr);
+    g.status = status_ptr(ws);
+    return launch_gemv(g, dev, sms, st);
+  }
+
+  if ((s = run_lora_down(X, ad, M, K, sc, sT, T_save, status_ptr(ws), dev, sms, st)) != QLORA_OK) return s;
+
+  CUtensorMap tmX, tmCodes, tmT;
+  if (!tmap_bf16(&tmX, X, K, M, 64, 128) || !tmap_bf16(&tmT, sT, ad->r, M, 64, 128) ||
+      !make_tmap(&tmCodes, W->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, K / 2, 32, 256, false))
+    return QLORA_ERR_CUDA;
+  GemmArgs g{};
+  g.M_rows = (int)M;
+  g.N_cols = (int)N;
+  g.k_steps = (int)(K / 64);
+  g.lora_steps = (ad->r + 63) / 64;
+  g.lora_r = ad->r;
+  g.out = Y;
+  g.ldo = N;
+  g.out_f32 = y_dtype == QLORA_F32;
+  g.out_scale = 1.0f;
+  g.scale_codes = W->scale_codes;
+  g.c2 = W->c2;
+  g.w_rows = N;
+  g.w_cols = K;
+  g.lora_b2 = static_cast<const __nv_bfloat16 *>(ad->B);
+  g.lora_ld = ad->r;
+  g.status = status_ptr(ws);
+  return launch_gemm<false, false, true, 256, 1>(tmX, tmX, tmT, tmCodes, g, dev, sms, st);
+}
+
+qlora_status qlora_linear_bwd(const qlora_nf4_tensor *W, const qlora_lora *ad, const void *X, const void *dY,
+                              int64_t M, const void *T_saved, void *dX, qlora_dtype dx_dtype, void *dA, void *dB,
+                              qlora_dtype grad_dtype, void *ws, size_t ws_bytes, qlora_stream_t stream) {
+  qlora_status s = check_nf4(W);
+  if (s != QLORA_OK) return s;
+  if ((s = check_lora(ad)) != QLORA_OK) return s;
+  if (!X || !dY || !dX || !dA || !dB || !ws || M < 1 || M > (int64_t(1) << 30)) return QLORA_ERR_INVALID_ARGUMENT;
+  if (!valid_dtype(dx_dtype) || !valid_dtype(grad_dtype)) return QLORA_ERR_INVALID_ARGUMENT;
+  if (W->rows % 8) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(X, 16) || !aligned(dY, 16) || !aligned(dX, 16) || !aligned(dA, 16) || !aligned(dB, 16) ||
+      !aligned(ws, 256) || (T_saved && !aligned(T_saved, 16)))
+    return QLORA_ERR_MISALIGNED;
+  const int64_t N = W->rows, K = W->cols;
+  if (ws_bytes < qlora_workspace_bytes(M, N, K, ad->r, 1)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  int dev, sms;
+  if ((s = check_device(&dev, &sms)) != QLORA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const float sc = ad->alpha / static_cast<float>(ad->r);
+  const int r = ad->r;
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  const size_t mr = align256(static_cast<size_t>(M) * r * 2);
+  void *sU = wsb + QLORA_STATUS_BYTES;
+  void *Tbuf = wsb + QLORA_STATUS_BYTES + mr;
+  uint32_t *status = status_ptr(ws);
+
+  const void *T = T_saved;
+  if (!T) {
+    // recompute T (unscaled) into the workspace; sU's slot serves as scratch for s*T
+    if ((s = run_lora_down(X, ad, M, K, sc, sU, Tbuf, status, dev, sms, st)) != QLORA_OK) return s;
+    T = Tbuf;
+  }
+  // U = dY B, stored as s*U (bf16)
+  {
+    CUtensorMap tmDY, tmB;
+    if (!tmap_bf16(&tmDY, dY, N, M, 64, 128) || !tmap_bf16(&tmB, ad->B, r, N, 64, 64)) return QLORA_ERR_CUDA;
+    GemmArgs g{};
+    g.M_rows = (int)M;
+    g.N_cols = r;
+    g.k_steps = (int)((N + 63) / 64);
+    g.out = sU;
+    g.ldo = r;
+    g.out_scale = sc;
+    g.status = status;
+    if ((s = launch_gemm<false, true, false, 64, 1>(tmDY, tmB, tmDY, tmDY, g, dev, sms, st)) != QLORA_OK) return s;
+  }
+  // dX = dY W' + (s U) A
+  {
+    CUtensorMap tmDY, tmU, tmCodes;
+    if (!tmap_bf16(&tmDY, dY, N, M, 64, 128) || !tmap_bf16(&tmU, sU, r, M, 64, 128) ||
+        !make_tmap(&tmCodes, W->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, K / 2, 128, 64, false))
+      return QLORA_ERR_CUDA;
+    GemmArgs g{};
+    g.M_rows = (int)M;
+    g.N_cols = (int)K;
+    g.k_steps = (int)((N + 63) / 64);
+    g.lora_steps = (r + 63) / 64;
+    g.lora_r = r;
+    g.out = dX;
+    g.ldo = K;
+    g.out_f32 = dx_dtype == QLORA_F32;
+    g.out_scale = 1.0f;
+    g.scale_codes = W->scale_codes;
+    g.c2 = W->c2;
+    g.w_rows = N;
+    g.w_cols = K;
+    g.lora_b2 = static_cast<const __nv_bfloat16 *>(ad->A);
+    g.lora_ld = K;
+    g.status = status;
+    if ((s = launch_gemm<false, true, true, 256, 1>(tmDY, tmDY, tmU, tmCodes, g, dev, sms, st)) != QLORA_OK)
+      return s;
+  }
+  // dA^T [K, r] = X^T (s U)  -> stored transposed into dA [r, K]
+  {
+    CUtensorMap tmXt, tmU;
+    if (!tmap_bf16(&tmXt, X, K, M, 64, 64) || !tmap_bf16(&tmU, sU, r, M, 64, 64)) return QLORA_ERR_CUDA;
+    GemmArgs g{};
+    g.M_rows = (int)K;
+    g.N_cols = r;
+    g.k_steps = (int)((M + 63) / 64);
+    g.out = dA;
+    g.ldo = K;
+    g.out_f32 = grad_dtype == QLORA_F32;
+    g.out_transpose = 1;
+    g.out_scale = 1.0f;
+    g.status = status;
+    if ((s = launch_gemm<true, true, false, 64, 1>(tmXt, tmU, tmXt, tmXt, g, dev, sms, st)) != QLORA_OK) return s;
+  }
+  // dB [N, r] = s dY^T T
+  {
+    CUtensorMap tmDYt, tmT;
+    if (!tmap_bf16(&tmDYt, dY, N, M, 64, 64) || !tmap_bf16(&tmT, T, r, M, 64, 64)) return QLORA_ERR_CUDA;
+    GemmArgs g{};
+    g.M_rows = (int)N;
+    g.N_cols = r;
+    g.k_steps = (int)((M + 63) / 64);
+    g.out = dB;
+    g.ldo = r;
+    g.out_f32 = grad_dtype == QLORA_F32;
+    g.out_scale = sc;
+    g.status = status;
+    if ((s = launch_gemm<true, true, false, 64, 1>(tmDYt, tmT, tmDYt, tmDYt, g, dev, sms, st)) != QLORA_OK) return s;
+  }
+  return QLORA_OK;
+}
+
+qlora_status qlora_clear_status(void *ws, qlora_stream_t stream) {
+  if (!ws) return QLORA_ERR_INVALID_ARGUMENT;
+  return cudaMemsetAsync(ws, 0, sizeof(uint32_t), reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? QLORA_OK
+             : QLORA_ERR_CUDA;
+}
+
+qlora_status qlora_read_status(const void *ws, qlora_stream_t stream) {
+  if (!ws) return QLORA_ERR_INVALID_ARGUMENT;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return QLORA_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpy(&word, ws, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return QLORA_ERR_CUDA;
+  for (int code = 1; code < 32; ++code)
+    if (word & (1u << code)) return static_cast<qlora_status>(code);
+  return QLORA_OK;
+}
+
+const char *qlora_status_string(qlora_status status) {
+  switch (status) {
+    case QLORA_OK: return "ok";
+    case QLORA_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case QLORA_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case QLORA_ERR_MISALIGNED: return "misaligned pointer";
+    case QLORA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case QLORA_ERR_NONFINITE: return "non-finite weight";
+    case QLORA_ERR_TIMEOUT: return "device wait timed out";
+    case QLORA_ERR_CUDA: return "CUDA error";
+    case QLORA_ERR_NO_DEVICE: return "no sm_100 device";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,223 @@
+// NF4 quantise (absmax per 64-block, codes, packing, E4M3 double quantisation of
+// the block scales per group of 256) and dequantise kernels.
+//
+// Quantiser: "QLoRA" (Ultralytics glossary), "How QLoRA works": NF4 bullet (one
+// absmax per 64 weights, 4-bit code into 16 normal-quantile levels) and the
+// double-quantisation bullet (the block scales quantised to 8 bits in blocks of
+// 256); "Grokking QLoRA" (vnread), "Double Quantization": the 8-bit format is FP8.
+//
+// One CTA owns one whole group (256 blocks = 16384 weights), so the group maximum
+// needed by the second level is a CTA-local reduction and no scratch memory or
+// second pass is needed.  Loads are 16-byte vectors; lanes 8 (bf16) or 16 (f32)
+// at a time share a block and reduce its absmax with warp shuffles.
+//
+// Code search.  The code of x = fl32(w / S) is argmin_j fl32(|x - L_j|), lowest j
+// on ties.  It is a non-decreasing step function of x with 15 switch points t_j
+// (the largest float32 whose code is <= j).  The kernel cuts [-1, 1] into 65 cells
+// of width 1/32 (cell = trunc(fl32(x * 32 + 32))), narrower than the closest pair
+// of switch points, and keeps per cell the switch point nearest to it and the code
+// just below that point: code = base + (x > thr).  The table is built on the host
+// from the same float32 definition.  To avoid a division per weight, the fast path
+// uses x' = w * fl32(1/S), which is within 2 ulp of fl32(w / S); whenever x' lies
+// within 4 ulp of the cell's switch point, the exact quotient (IEEE division) is
+// used instead, so the result is always the code of fl32(w / S).
+#pragma once
+
+#include "nf4_device.cuh"
+
+namespace qlora {
+
+constexpr int kCells = 65;
+
+struct CodeCellTable {
+  float thr[kCells];      // switch point nearest to the cell
+  uint32_t base[kCells];  // code of x <= thr
+};
+
+// Exact code of a normalised weight x in [-1, 1] (x already equal to fl32(w / S)).
+__device__ __forceinline__ uint32_t code_from_table(float x, const float *s_thr, const uint32_t *s_base) {
+  const int cell = __float2int_rz(__fmaf_rn(x, 32.0f, 32.0f));
+  return s_base[cell] + (x > s_thr[cell] ? 1u : 0u);
+}
+
+template <typename TIn>
+struct QuantTraits;
+template <>
+struct QuantTraits<__nv_bfloat16> {
+  static constexpr int kElemsPerLane = 8;  // one 16-byte vector
+};
+template <>
+struct QuantTraits<float> {
+  static constexpr int kElemsPerLane = 4;
+};
+
+// Unpacks the 16-byte vector of this lane to float32 values.
+__device__ __forceinline__ void unpack_vec(const uint4 &v, float (&w)[8]) {
+  w[0] = bf16lo_to_f32(v.x); w[1] = bf16hi_to_f32(v.x);
+  w[2] = bf16lo_to_f32(v.y); w[3] = bf16hi_to_f32(v.y);
+  w[4] = bf16lo_to_f32(v.z); w[5] = bf16hi_to_f32(v.z);
+  w[6] = bf16lo_to_f32(v.w); w[7] = bf16hi_to_f32(v.w);
+}
+__device__ __forceinline__ void unpack_vec(const uint4 &v, float (&w)[4]) {
+  w[0] = __uint_as_float(v.x); w[1] = __uint_as_float(v.y);
+  w[2] = __uint_as_float(v.z); w[3] = __uint_as_float(v.w);
+}
+
+// |w| bit pattern maximum; NaN and infinities compare above every finite value.
+__device__ __forceinline__ uint32_t absbits_max(const uint4 &v, __nv_bfloat16 *) {
+  const uint32_t a = __vmaxu2(v.x & 0x7fff7fffu, v.y & 0x7fff7fffu);
+  const uint32_t b = __vmaxu2(v.z & 0x7fff7fffu, v.w & 0x7fff7fffu);
+  const uint32_t m = __vmaxu2(a, b);
+  return max(m & 0xffffu, m >> 16) << 16;  // as float32 bits
+}
+__device__ __forceinline__ uint32_t absbits_max(const uint4 &v, float *) {
+  return max(max(v.x & 0x7fffffffu, v.y & 0x7fffffffu), max(v.z & 0x7fffffffu, v.w & 0x7fffffffu));
+}
+
+constexpr int kQuantThreads = 256;
+
+// grid.x = number of groups; one CTA per group of 256 blocks.
+template <typename TIn>
+__global__ void __launch_bounds__(kQuantThreads)
+nf4_quantize_kernel(const TIn *__restrict__ W, int64_t nblocks, uint8_t *__restrict__ codes,
+                    uint8_t *__restrict__ scale_codes, float *__restrict__ c2_out,
+                    uint32_t *__restrict__ status, const CodeCellTable table) {
+  constexpr int EPL = QuantTraits<TIn>::kElemsPerLane;
+  constexpr int LPB = kBlock / EPL;                      // lanes per block
+  constexpr int BPI = kQuantThreads / LPB;               // blocks per CTA iteration
+  constexpr int ITERS = kGroup / BPI;
+
+  __shared__ float s_thr[kCells];
+  __shared__ uint32_t s_base[kCells];
+  __shared__ float s_absmax[kGroup];
+  __shared__ float s_wmax[kQuantThreads / 32];
+
+  const int tid = threadIdx.x;
+  if (tid < kCells) {
+    s_thr[tid] = table.thr[tid];
+    s_base[tid] = table.base[tid];
+  }
+  const int64_t g = blockIdx.x;
+  const int64_t blk0 = g * kGroup;
+  const int nblk = static_cast<int>(nblocks - blk0 < kGroup ? nblocks - blk0 : kGroup);
+
+  // Issue every load of this thread first (ITERS x 16 bytes in flight).
+  uint4 v[ITERS];
+#pragma unroll
+  for (int it = 0; it < ITERS; ++it) {
+    const int lb = it * BPI + tid / LPB;  // block within group
+    if (lb < nblk) {
+      const int64_t e0 = (blk0 + lb) * kBlock + (tid % LPB) * EPL;
+      v[it] = __ldg(reinterpret_cast<const uint4 *>(W + e0));
+    } else {
+      v[it] = make_uint4(0, 0, 0, 0);
+    }
+  }
+  __syncthreads();
+
+#pragma unroll
+  for (int it = 0; it < ITERS; ++it) {
+    const int lb = it * BPI + tid / LPB;
+    uint32_t mb = absbits_max(v[it], static_cast<TIn *>(nullptr));
+#pragma unroll
+    for (int o = LPB / 2; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+    if (lb >= nblk) continue;
+    const bool finite = mb < 0x7f800000u;
+    const float S = __uint_as_float(mb);
+    if (!finite && (tid % LPB) == 0) raise_status(status, QLORA_ERR_NONFINITE);
+    if ((tid % LPB) == 0) s_absmax[lb] = finite ? S : 0.0f;
+
+    float w[EPL];
+    unpack_vec(v[it], w);
+    uint32_t packed = 0;
+    if (S == 0.0f || !finite) {
+      packed = 0x77777777u & ((1ull << (4 * EPL)) - 1);  // exact-zero level everywhere
+    } else {
+      const float rS = __frcp_rn(S);
+      bool slow = !(rS < 3.0e38f);  // subnormal S: reciprocal overflows
+      uint32_t c[EPL];
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const float xa = __fmul_rn(w[i], rS);
+        const int cell = __float2int_rz(__fmaf_rn(xa, 32.0f, 32.0f));
+        const float t = s_thr[min(max(cell, 0), kCells - 1)];
+        c[i] = s_base[min(max(cell, 0), kCells - 1)] + (xa > t ? 1u : 0u);
+        slow |= (__float_as_uint(xa) - __float_as_uint(t) + 4u) <= 8u;
+      }
+      if (slow) {
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) c[i] = code_from_table(__fdiv_rn(w[i], S), s_thr, s_base);
+      }
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) packed |= c[i] << (4 * i);
+    }
+    const int64_t e0 = (blk0 + lb) * kBlock + (tid % LPB) * EPL;
+    if constexpr (EPL == 8) {
+      *reinterpret_cast<uint32_t *>(codes + e0 / 2) = packed;
+    } else {
+      *reinterpret_cast<uint16_t *>(codes + e0 / 2) = static_cast<uint16_t>(packed);
+    }
+  }
+  __syncthreads();
+
+  // Second level: c2 = fl32(max S / 448), q = E4M3(fl32(S / c2)).
+  float m = tid < nblk ? s_absmax[tid] : 0.0f;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((tid & 31) == 0) s_wmax[tid >> 5] = m;
+  __syncthreads();
+  m = s_wmax[0];
+#pragma unroll
+  for (int i = 1; i < kQuantThreads / 32; ++i) m = fmaxf(m, s_wmax[i]);
+  const float c2 = m == 0.0f ? 0.0f : __fdiv_rn(m, 448.0f);
+  if (tid < nblk) scale_codes[blk0 + tid] = c2 == 0.0f ? 0 : f32_to_e4m3(__fdiv_rn(s_absmax[tid], c2));
+  if (tid == 0) c2_out[g] = c2;
+}
+
+// ---------------------------------------------------------------------------
+// Dequantise: w' = bf16_rne(fl32(L[c] * S')), S' = fl32(E4M3(q) * c2).
+// One thread per 16 bytes of codes (32 weights, half a block).
+// ---------------------------------------------------------------------------
+constexpr int kDequantThreads = 256;
+
+template <typename TOut>
+__global__ void __launch_bounds__(kDequantThreads)
+nf4_dequantize_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scale_codes,
+                      const float *__restrict__ c2, int64_t nchunks, TOut *__restrict__ out) {
+  __shared__ float s_lv[16];
+  if (threadIdx.x < 16) s_lv[threadIdx.x] = __uint_as_float(kNf4LevelBits[threadIdx.x]);
+  __syncthreads();
+  for (int64_t ch = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; ch < nchunks;
+       ch += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 cv = __ldg(reinterpret_cast<const uint4 *>(codes) + ch);
+    const float S = block_scale(scale_codes, c2, ch >> 1);
+    const uint32_t words[4] = {cv.x, cv.y, cv.z, cv.w};
+    if constexpr (sizeof(TOut) == 2) {
+      uint32_t o[16];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t byte = (words[q] >> (8 * j)) & 0xffu;
+          o[q * 4 + j] = pack_bf16x2(__fmul_rn(s_lv[byte & 0xf], S), __fmul_rn(s_lv[byte >> 4], S));
+        }
+      uint4 *dst = reinterpret_cast<uint4 *>(out + ch * 32);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) dst[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+    } else {
+      float o[32];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float p = __fmul_rn(s_lv[(words[q] >> (4 * j)) & 0xfu], S);
+          o[q * 8 + j] = __uint_as_float(pack_bf16x2(p, 0.0f) << 16);
+        }
+      float4 *dst = reinterpret_cast<float4 *>(out + ch * 32);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+    }
+  }
+}
+
+}  // namespace qlora

@@ -1,0 +1,175 @@
+/*
+ * qlora_nf4.h -- C ABI of the B200 (sm_100a) library for the frozen NF4 linear
+ * layer with a LoRA adapter, as the QLoRA pages define it.
+ *
+ * What the layer computes (sources named by page title and section):
+ *   - "QLoRA" (Ultralytics glossary), "How QLoRA works": every frozen weight is a
+ *     4-bit code into 16 levels placed at normal quantiles, with one absmax scale
+ *     per block of 64 weights; the block scales are themselves quantised to 8 bits
+ *     in blocks of 256; the forward pass dequantises NF4 to bfloat16 right before
+ *     the matmul and adds the LoRA path; the backward pass computes gradients
+ *     through the dequantised weights and updates only the two LoRA matrices.
+ *   - "Grokking QLoRA" (vnread), "Double Quantization": the 8-bit second level is FP8.
+ *   - "What is LoRA?" (IBM) and "Mastering model fine-tuning" (ezsol.ir),
+ *     "Low-Rank Adaptation (LoRA)": Delta W = B A with rank r; lora_alpha scales it.
+ *
+ * Notation: W [N, K] row-major (nn.Linear convention y = X W^T), N = rows =
+ * out_features, K = cols = in_features; X [M, K]; A [r, K]; B [N, r]; s = alpha / r
+ * (float32).  Block = 64 consecutive elements of row-major W (K % 64 == 0, so a
+ * block never crosses a row); group = 256 consecutive blocks (the last group of a
+ * tensor may be short; groups may cross rows).  nb = N*K/64, ng = ceil(nb/256).
+ *
+ * Formats fixed by this library (readings of the pages):
+ *   codes        N*K/2 bytes; byte i = code[2i] | code[2i+1] << 4 (row-major order)
+ *   scale_codes  nb bytes, OCP FP8 E4M3 (sign bit 0): q = E4M3_rne_sat(S / c2)
+ *   c2           ng float32: c2 = max(S over the group) / 448 (0 for an all-zero group)
+ *   code         argmin_j |fl32(w / S) - L_j| in float32, lowest j on ties; S == 0 -> 7
+ *   dequantised  w' = bf16_rne(fl32(L[code] * fl32(E4M3(q) * c2)))
+ *
+ * Conventions shared by every entry point:
+ *   - Pointers named in a qlora_nf4_tensor, qlora_lora or as X/Y/dY/dX/dA/dB/ws
+ *     are DEVICE pointers, allocated and owned by the caller.  Tensor pointers must
+ *     be 16-byte aligned; ws must be 256-byte aligned.
+ *   - The library never allocates, frees or synchronises (except
+ *     qlora_read_status, which synchronises the stream it is given).  All scratch
+ *     comes from the caller's workspace ws of at least qlora_workspace_bytes().
+ *     The first QLORA_STATUS_BYTES of ws hold a device status word.
+ *   - Argument checks run on the host before any launch; a failed check returns an
+ *     error code and launches nothing.  A failed launch returns QLORA_ERR_CUDA.
+ *     Errors found on the device (non-finite weights, a bounded wait that timed
+ *     out) are OR-ed into the status word; qlora_read_status() returns them.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *   - Entry points are thread-safe and keep no per-call state.  Nothing is printed
+ *     and no C++ exception crosses this boundary.
+ *   - Only sm_100 devices are supported (QLORA_ERR_NO_DEVICE otherwise).
+ */
+#ifndef QLORA_NF4_H
+#define QLORA_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define QLORA_NF4_ABI_VERSION 1
+#define QLORA_BLOCK 64          /* weights per first-level absmax block */
+#define QLORA_GROUP 256         /* first-level scales per second-level group */
+#define QLORA_STATUS_BYTES 256  /* bytes at the start of ws reserved for the status word */
+#define QLORA_MAX_RANK 256
+
+#if defined(__GNUC__)
+#define QLORA_API __attribute__((visibility("default")))
+#else
+#define QLORA_API
+#endif
+
+typedef struct CUstream_st *qlora_stream_t; /* same handle type as cudaStream_t */
+
+typedef enum {
+  QLORA_OK = 0,
+  QLORA_ERR_INVALID_ARGUMENT = 1,   /* null pointer, bad enum, bad rank or M */
+  QLORA_ERR_UNSUPPORTED_SHAPE = 2,  /* K % 64 != 0, or a dimension out of range */
+  QLORA_ERR_MISALIGNED = 3,         /* a tensor pointer is not 16-byte aligned (ws: 256) */
+  QLORA_ERR_WORKSPACE_TOO_SMALL = 4,
+  QLORA_ERR_NONFINITE = 5,          /* device: a block held a NaN or an infinity */
+  QLORA_ERR_TIMEOUT = 6,            /* device: a bounded wait gave up */
+  QLORA_ERR_CUDA = 7,               /* a CUDA runtime call or launch failed */
+  QLORA_ERR_NO_DEVICE = 8           /* the current device is not an sm_100 GPU */
+} qlora_status;
+
+typedef enum { QLORA_F32 = 0, QLORA_BF16 = 1 } qlora_dtype;
+
+/* Quantised weight W [rows, cols]; three caller-owned device buffers, sized by
+ * qlora_nf4_storage_bytes(). */
+typedef struct {
+  int64_t rows;          /* N */
+  int64_t cols;          /* K, a multiple of 64 */
+  uint8_t *codes;        /* rows*cols/2 bytes, packed nibbles */
+  uint8_t *scale_codes;  /* nb bytes, E4M3 */
+  float *c2;             /* ng float32 second-level constants */
+} qlora_nf4_tensor;
+
+/* LoRA adapter: A [r, K] and B [N, r], both bf16 row-major device buffers.
+ * r in [8, 256] and a multiple of 8. */
+typedef struct {
+  int32_t r;
+  float alpha;
+  const void *A;
+  const void *B;
+} qlora_lora;
+
+/* Version of this ABI (QLORA_NF4_ABI_VERSION). */
+QLORA_API int qlora_abi_version(void);
+
+/* Copies the 16 float32 NF4 levels the kernels use into out[0..15] (host memory).
+ * They are the normal-quantile levels of the glossary page's snippet ("How QLoRA
+ * works"), each rounded once to float32. */
+QLORA_API void qlora_nf4_codebook(float out[16]);
+
+/* Bytes of the three buffers of a quantised [rows, cols] tensor.  Any of the
+ * out-pointers may be NULL.  Returns their sum, or 0 if cols % 64 != 0 or a
+ * dimension is not positive. */
+QLORA_API size_t qlora_nf4_storage_bytes(int64_t rows, int64_t cols, size_t *codes_bytes,
+                               size_t *scale_codes_bytes, size_t *c2_bytes);
+
+/* Workspace bytes needed by qlora_linear_fwd (for_backward = 0) or
+ * qlora_linear_bwd (for_backward = 1) for M tokens, W [N, K] and rank r;
+ * at least QLORA_STATUS_BYTES.  0 for invalid sizes. */
+QLORA_API size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r, int for_backward);
+
+/* Quantise W [out->rows, out->cols] (float32 or bf16, row-major, device) to NF4
+ * with double-quantised scales (glossary page, "How QLoRA works": NF4 and double
+ * quantisation bullets).  Writes out->codes, out->scale_codes, out->c2.
+ * ws: device workspace of at least QLORA_STATUS_BYTES (status word).  A block
+ * holding a NaN or an infinity sets QLORA_ERR_NONFINITE in the status word; the
+ * contents of that block's outputs are then unspecified. */
+QLORA_API qlora_status qlora_nf4_quantize(const void *W, qlora_dtype w_dtype, const qlora_nf4_tensor *out,
+                                void *ws, qlora_stream_t stream);
+
+/* Dequantise to W_out [rows, cols] row-major (bf16; float32 holds the same
+ * bf16-exact values, for tests), the step the glossary page places right
+ * before the matmul. */
+QLORA_API qlora_status qlora_nf4_dequantize(const qlora_nf4_tensor *w, void *W_out, qlora_dtype out_dtype,
+                                  qlora_stream_t stream);
+
+/* Forward of the frozen linear layer with LoRA (glossary page, "How QLoRA
+ * works", forward rule):  Y [M, N] = X W'^T + s (X A^T) B^T.
+ *   X      bf16 [M, K] device
+ *   Y      [M, N] device, bf16 or float32 (y_dtype)
+ *   T_save nullable bf16 [M, r] device: receives T = X A^T for the backward pass
+ *   ws     device workspace of ws_bytes >= qlora_workspace_bytes(M, N, K, r, 0)
+ * M >= 1.  M <= 16 takes the decode (GEMV) path; larger M the tensor-core path. */
+QLORA_API qlora_status qlora_linear_fwd(const qlora_nf4_tensor *W, const qlora_lora *adapter, const void *X,
+                              int64_t M, void *Y, qlora_dtype y_dtype, void *T_save, void *ws,
+                              size_t ws_bytes, qlora_stream_t stream);
+
+/* Backward (glossary page, "How QLoRA works": gradients through the dequantised
+ * weights, only the LoRA matrices updated).  With U = dY B:
+ *   dX [M, K] = dY W' + s U A          (dx_dtype: bf16 or float32)
+ *   dA [r, K] = s U^T X                (grad_dtype: bf16 or float32)
+ *   dB [N, r] = s dY^T T,  T = X A^T   (grad_dtype)
+ * T_saved: nullable bf16 [M, r] from qlora_linear_fwd; NULL recomputes it.
+ * dY bf16 [M, N].  dX, dA, dB are overwritten (not accumulated).  W gets no
+ * gradient. */
+QLORA_API qlora_status qlora_linear_bwd(const qlora_nf4_tensor *W, const qlora_lora *adapter, const void *X,
+                              const void *dY, int64_t M, const void *T_saved, void *dX,
+                              qlora_dtype dx_dtype, void *dA, void *dB, qlora_dtype grad_dtype,
+                              void *ws, size_t ws_bytes, qlora_stream_t stream);
+
+/* Zero the status word at the start of ws (enqueued on stream). */
+QLORA_API qlora_status qlora_clear_status(void *ws, qlora_stream_t stream);
+
+/* Synchronise `stream`, read the status word at the start of ws and return the
+ * first error it records (QLORA_OK if none).  The word is left unchanged. */
+QLORA_API qlora_status qlora_read_status(const void *ws, qlora_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+QLORA_API const char *qlora_status_string(qlora_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_NF4_H */

@@ -1,0 +1,91 @@
+"""The C-ABI library loads, exports every declared symbol, and its host-side
+logic (sizes, table, argument checks) behaves without a GPU."""
+
+import ctypes
+
+import numpy as np
+import pytest
+
+import oracle as O
+from bit_nf4_quantized_27_b200 import binding as bd
+from bit_nf4_quantized_27_b200.build import build
+
+
+@pytest.fixture(scope="module")
+def L():
+    build()
+    return bd.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = bd.header_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_abi_version(L):
+    assert L.qlora_abi_version() == 1
+
+
+def test_codebook_equals_oracle_bit_for_bit(L):
+    got = np.array(bd.codebook(), dtype=np.float32)
+    assert np.array_equal(got.view(np.uint32), O.nf4_levels().view(np.uint32))
+
+
+@pytest.mark.parametrize("rows,cols", [(256, 256), (4096, 4096), (11008, 4096), (3, 64), (1, 64 * 300)])
+def test_storage_bytes_match_oracle(L, rows, cols):
+    total, c, s, g = bd.storage_bytes(rows, cols)
+    oc, os_, og = O.storage_bytes(rows, cols)
+    assert (c, s, g) == (oc, os_, og) and total == c + s + g
+
+
+def test_storage_bytes_rejects_bad_cols(L):
+    assert bd.storage_bytes(4, 65)[0] == 0
+    assert bd.storage_bytes(0, 64)[0] == 0
+
+
+def test_workspace_bytes(L):
+    assert bd.workspace_bytes(16, 11008, 4096, 64, False) >= 256 + 16 * 64 * 2
+    assert bd.workspace_bytes(2048, 4096, 4096, 64, True) >= 256 + 2 * 2048 * 64 * 2
+    assert bd.workspace_bytes(0, 1, 64, 8, False) == 0
+    assert bd.workspace_bytes(1, 1, 64, 512, False) == 0
+
+
+def _t(rows, cols, codes=0x1000, sc=0x2000, c2=0x3000):
+    return bd.NF4TensorC(rows, cols, codes, sc, c2)
+
+
+def test_argument_checks_without_gpu(L):
+    # Every check runs before any device work; fake (never dereferenced) pointers.
+    W, ws = ctypes.c_void_p(0x10000), ctypes.c_void_p(0x20000)
+    good = _t(64, 64)
+    assert L.qlora_nf4_quantize(W, 1, ctypes.byref(_t(64, 65)), ws, None) == 2
+    assert L.qlora_nf4_quantize(W, 1, ctypes.byref(_t(64, 64, codes=0)), ws, None) == 1
+    assert L.qlora_nf4_quantize(None, 1, ctypes.byref(good), ws, None) == 1
+    assert L.qlora_nf4_quantize(W, 7, ctypes.byref(good), ws, None) == 1
+    assert L.qlora_nf4_quantize(ctypes.c_void_p(0x10008), 1, ctypes.byref(good), ws, None) == 3
+    assert L.qlora_nf4_quantize(W, 1, ctypes.byref(_t(64, 64, codes=0x1004)), ws, None) == 3
+    ad = bd.LoraC(64, 16.0, 0x4000, 0x5000)
+    X, Y = ctypes.c_void_p(0x6000), ctypes.c_void_p(0x7000)
+    assert L.qlora_linear_fwd(ctypes.byref(good), ctypes.byref(bd.LoraC(12, 16.0, 0x4000, 0x5000)), X, 4, Y, 1,
+                              None, ws, 1 << 20, None) == 1
+    assert L.qlora_linear_fwd(ctypes.byref(good), ctypes.byref(ad), X, 0, Y, 1, None, ws, 1 << 20, None) == 1
+    assert L.qlora_linear_fwd(ctypes.byref(good), ctypes.byref(ad), X, 4, Y, 1, None, ws, 16, None) == 4
+    assert L.qlora_linear_fwd(ctypes.byref(_t(60, 64)), ctypes.byref(ad), X, 4, Y, 1, None, ws, 1 << 20, None) == 2
+    assert L.qlora_linear_bwd(ctypes.byref(good), ctypes.byref(ad), X, None, 4, None, X, 1, X, X, 1, ws, 1 << 20,
+                              None) == 1
+
+
+def test_valid_call_without_gpu_reports_no_device(L):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    W, ws = ctypes.c_void_p(0x10000), ctypes.c_void_p(0x20000)
+    assert L.qlora_nf4_quantize(W, 1, ctypes.byref(_t(64, 64)), ws, None) == 8
+
+
+def test_status_strings(L):
+    for code in range(9):
+        assert L.qlora_status_string(code)
+    assert L.qlora_status_string(0) == b"ok"

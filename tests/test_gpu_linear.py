@@ -1,0 +1,216 @@
+"""GPU forward/backward of the NF4 linear layer with LoRA against the CPU oracle.
+
+Tolerance (the stated bar for outputs and gradients): max |gpu - oracle| <=
+1e-2 * RMS(oracle).  Float32 outputs are held to exactly that; bf16 outputs may in
+addition carry their own rounding, one bf16 ulp of the oracle value.  The oracle
+quantises the raw weights itself; nothing it uses comes from the GPU."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from bit_nf4_quantized_27_b200 import binding as bd
+from bit_nf4_quantized_27_b200 import inputs as I
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-2
+
+
+def _ulp_bf16(v):
+    a = np.abs(v)
+    e = np.floor(np.log2(np.where(a > 0, a, 1e-38)))
+    return np.where(a > 0, 2.0 ** (e - 7), 2.0 ** -133)
+
+
+def check(name, got: torch.Tensor, ref: np.ndarray, rms: float | None = None):
+    g = got.float().cpu().numpy().astype(np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert g.shape == ref.shape, (name, g.shape, ref.shape)
+    rms = float(np.sqrt(np.mean(ref ** 2))) if rms is None else rms
+    err = np.abs(g - ref)
+    bound = TOL * rms + (_ulp_bf16(ref) if got.dtype == torch.bfloat16 else 0.0)
+    worst = float(np.max(err - bound))
+    assert np.all(np.isfinite(g)), name
+    assert worst <= 0, f"{name}: max err {err.max():.3e} vs bound {TOL * rms:.3e} (rms {rms:.3e})"
+    return float(err.max() / rms) if rms > 0 else 0.0
+
+
+class Case:
+    """Inputs + oracle for one layer."""
+
+    def __init__(self, w, x, a, b, dy, alpha):
+        self.w, self.x, self.a, self.b, self.dy, self.alpha = w, x, a, b, dy, alpha
+        self.n, self.k = w.shape
+        self.m, self.r = x.shape[0], a.shape[0]
+        q = O.quantize(w.float().numpy(), self.n, self.k)
+        self.wd = O.dequantize(q["codes"], q["scale_codes"], q["c2"], self.n, self.k)
+        self.xf, self.af, self.bf, self.dyf = (t.float().numpy() for t in (x, a, b, dy))
+
+    def gpu(self):
+        qg = bd.quantize(self.w.cuda())
+        return qg, self.a.cuda(), self.b.cuda(), self.x.cuda(), self.dy.cuda()
+
+    def ref_fwd(self, rows=None):
+        x = self.xf if rows is None else self.xf[rows]
+        return O.linear_fwd(self.wd, self.af, self.bf, x, self.alpha, self.r)
+
+    def ref_bwd(self):
+        return O.linear_bwd(self.wd, self.af, self.bf, self.xf, self.dyf, self.alpha, self.r)
+
+
+def _custom(n, k, m, r, seed, alpha=16.0, w_dtype=torch.bfloat16, b_std=0.01):
+    return Case(*I.custom(n, k, m, r, seed, w_dtype=w_dtype, b_std=b_std), alpha)
+
+
+def _run_fwd_bwd(c: Case, y_dtype, g_dtype, save_t=True):
+    qg, a, b, x, dy = c.gpu()
+    y, t = bd.linear_fwd(qg, a, b, c.alpha, x, y_dtype=y_dtype, save_t=save_t)
+    dx, da, db = bd.linear_bwd(qg, a, b, c.alpha, x, dy, t, dx_dtype=g_dtype, grad_dtype=g_dtype)
+    torch.cuda.synchronize()
+    return y, t, dx, da, db
+
+
+def _check_all(c: Case, y, t, dx, da, db):
+    yr, tr = c.ref_fwd()
+    check("y", y, yr)
+    if t is not None:
+        check("T", t, tr)
+    dxr, dar, dbr = c.ref_bwd()
+    check("dX", dx, dxr)
+    check("dA", da, dar)
+    check("dB", db, dbr)
+
+
+def test_tiny_workload():
+    wl = I.TINY
+    c = Case(I.weight(wl), I.activations(wl), I.lora_a(wl), I.lora_b(wl), I.grad_output(wl), wl.alpha)
+    for dt in (torch.float32, torch.bfloat16):
+        _check_all(c, *_run_fwd_bwd(c, dt, dt))
+
+
+@pytest.mark.parametrize("m", [1, 3, 4, 9, 16])
+def test_gemv_path_small_shapes(m):
+    c = _custom(328, 576, m, 64, 1000 + m)
+    for dt in (torch.float32, torch.bfloat16):
+        qg, a, b, x, _ = c.gpu()
+        y, t = bd.linear_fwd(qg, a, b, c.alpha, x, y_dtype=dt)
+        yr, tr = c.ref_fwd()
+        check(f"y m={m}", y, yr)
+        check(f"T m={m}", t, tr)
+
+
+@pytest.mark.parametrize("m", [1, 4, 16])
+def test_gemv_workload_11008x4096(m):
+    wl = I.GEMV
+    c = Case(I.weight(wl), I.activations(wl, m=m), I.lora_a(wl), I.lora_b(wl), I.grad_output(wl, m=m), wl.alpha)
+    qg, a, b, x, _ = c.gpu()
+    y, _ = bd.linear_fwd(qg, a, b, c.alpha, x, y_dtype=torch.float32)
+    yr, _ = c.ref_fwd()
+    check("y", y, yr)
+    # LoRA contribution alone must be right too (it is ~1.5% of y's RMS)
+    y0, _ = bd.linear_fwd(qg, a, torch.zeros_like(b), c.alpha, x, y_dtype=torch.float32)
+    lora_ref = yr - (c.xf.astype(np.float64) @ c.wd.astype(np.float64).T)
+    check("lora part", y - y0, lora_ref)
+
+
+@pytest.mark.parametrize("n,k,m,r", [(256, 256, 17, 8), (328, 320, 200, 16), (1024, 1024, 512, 64),
+                                     (264, 640, 129, 128), (512, 192, 300, 256), (4104, 128, 64, 64)])
+def test_tensor_core_path_ragged(n, k, m, r):
+    c = _custom(n, k, m, r, 7 * n + k + m + r)
+    for dt in (torch.float32, torch.bfloat16):
+        _check_all(c, *_run_fwd_bwd(c, dt, dt))
+
+
+def test_backward_recomputes_t():
+    c = _custom(512, 512, 96, 64, 55)
+    qg, a, b, x, dy = c.gpu()
+    dx, da, db = bd.linear_bwd(qg, a, b, c.alpha, x, dy, None, dx_dtype=torch.float32, grad_dtype=torch.float32)
+    dxr, dar, dbr = c.ref_bwd()
+    check("dX", dx, dxr)
+    check("dA", da, dar)
+    check("dB", db, dbr)
+
+
+@pytest.mark.parametrize("m", [4, 300])
+def test_b_zero_is_base_layer(m):
+    c = _custom(512, 512, m, 64, 77, b_std=0.0)
+    y, t, dx, da, db = _run_fwd_bwd(c, torch.float32, torch.float32)
+    base = c.xf.astype(np.float64) @ c.wd.astype(np.float64).T
+    check("y", y, base)
+    assert torch.count_nonzero(da) == 0
+
+
+@pytest.mark.parametrize("m", [4, 300])
+def test_w_zero_isolates_lora(m):
+    w, x, a, b, dy = I.custom(512, 512, m, 64, 88)
+    c = Case(torch.zeros_like(w), x, a, b, dy, 16.0)
+    y, t, dx, da, db = _run_fwd_bwd(c, torch.float32, torch.float32)
+    yr, _ = c.ref_fwd()
+    check("y", y, yr)
+    dxr, dar, dbr = c.ref_bwd()
+    check("dX", dx, dxr)
+
+
+def test_merged_form():
+    c = _custom(512, 512, 64, 64, 99)
+    qg, a, b, x, _ = c.gpu()
+    y, _ = bd.linear_fwd(qg, a, b, c.alpha, x, y_dtype=torch.float32)
+    wm = O.merged_weight(c.wd, c.af, c.bf, c.alpha, c.r)
+    check("y", y, c.xf.astype(np.float64) @ wm.T)
+
+
+def test_autograd_wrapper():
+    c = _custom(256, 256, 32, 16, 5)
+    qg, a, b, x, dy = c.gpu()
+    x = x.clone().requires_grad_(True)
+    a = a.clone().requires_grad_(True)
+    b = b.clone().requires_grad_(True)
+    y = bd.QLoRALinearFunction.apply(x, a, b, qg, c.alpha)
+    y.backward(dy)
+    dxr, dar, dbr = c.ref_bwd()
+    check("dX", x.grad, dxr)
+    check("dA", a.grad, dar)
+    check("dB", b.grad, dbr)
+
+
+def test_deterministic():
+    c = _custom(1024, 1024, 256, 64, 3)
+    r1 = _run_fwd_bwd(c, torch.float32, torch.float32)
+    r2 = _run_fwd_bwd(c, torch.float32, torch.float32)
+    for u, v in zip(r1, r2):
+        assert torch.equal(u, v)
+
+
+def _sampled(wl, layer, nrows=48):
+    c = Case(I.weight(wl, layer), I.activations(wl, layer), I.lora_a(wl, layer), I.lora_b(wl, layer),
+             I.grad_output(wl, layer), wl.alpha)
+    qg, a, b, x, dy = c.gpu()
+    y, t = bd.linear_fwd(qg, a, b, c.alpha, x, y_dtype=torch.bfloat16)
+    dx, da, db = bd.linear_bwd(qg, a, b, c.alpha, x, dy, t, dx_dtype=torch.bfloat16, grad_dtype=torch.float32)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(layer)
+    rows = np.sort(rng.choice(c.m, nrows, replace=False))
+    rows[-1] = c.m - 1
+    yr, tr = c.ref_fwd(rows)
+    check("y rows", y[torch.from_numpy(rows)], yr)
+    s = O.lora_scale(c.alpha, c.r)
+    x64, dy64, a64, b64 = (np.asarray(v, np.float64) for v in (c.xf, c.dyf, c.af, c.bf))
+    u = dy64 @ b64
+    dxr = dy64[rows] @ c.wd.astype(np.float64) + s * (u[rows] @ a64)
+    check("dX rows", dx[torch.from_numpy(rows)], dxr)
+    t64 = x64 @ a64.T
+    check("dA", da, s * (u.T @ x64))
+    check("dB", db, s * (dy64.T @ t64))
+
+
+@pytest.mark.parametrize("layer", [0, 4, 6], ids=["q", "gate", "down"])
+def test_llama7b_block_layers_full_size(layer):
+    _sampled(I.LLAMA7B_BLOCK, layer)
+
+
+def test_65b_block_q_full_size():
+    _sampled(I.L65B_BLOCK, 0, nrows=24)
