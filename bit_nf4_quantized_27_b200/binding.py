@@ -179,12 +179,13 @@ def _lora(A: torch.Tensor, B: torch.Tensor, alpha: float) -> LoraC:
 
 def linear_fwd(q: NF4Weight, A, B, alpha: float, X, y_dtype=torch.bfloat16, save_t: bool = True,
                ws: torch.Tensor | None = None, out: torch.Tensor | None = None, t_out=None, stream=None):
-    """Y = X W'^T + (alpha/r) (X A^T) B^T.  Returns (Y, T or None)."""
+    """Y = X W'^T + (alpha/r) (X A^T) B^T.  Returns (Y, T or None); T is the
+    [2, M, r] bf16 pair (hi, lo) with hi + lo = X A^T."""
     M = X.shape[0]
     r = A.shape[0]
     assert X.dtype == torch.bfloat16 and X.is_contiguous() and X.shape[1] == q.cols
     Y = out if out is not None else torch.empty(M, q.rows, dtype=y_dtype, device=X.device)
-    T = t_out if t_out is not None else (torch.empty(M, r, dtype=torch.bfloat16, device=X.device) if save_t else None)
+    T = t_out if t_out is not None else (torch.empty(2, M, r, dtype=torch.bfloat16, device=X.device) if save_t else None)
     need = workspace_bytes(M, q.rows, q.cols, r, False)
     if ws is None:
         ws = new_workspace(need, X.device)

@@ -30,17 +30,20 @@ struct GemmArgs {
   int M_rows;        // rows of D (tiles of 128 * MT)
   int N_cols;        // cols of D (tiles of BN)
   int k_steps;       // main K steps of 64
+  int hilo;          // 1: a second pass of k_steps reuses A with B taken from tmB2
   int lora_steps;    // extra K steps of 64 for the LoRA block (0 = none)
   int lora_r;        // LoRA rank (bounds the B2 rows/cols read by the dequant warps)
-  // output 1 (required) and output 2 (optional, bf16)
+  // outputs (each optional): `out` (f32 or bf16, scaled by out_scale, optionally
+  // transposed) and a bf16 pair hi = bf16(v * hl_scale), lo = bf16(v * hl_scale - hi)
   void *out;
   int64_t ldo;
   int out_f32;       // 1: float32, 0: bf16
   int out_transpose; // 1: out[col * ldo + row]
   float out_scale;
-  void *out2;
-  int64_t ldo2;
-  float out2_scale;
+  __nv_bfloat16 *out_hi;
+  __nv_bfloat16 *out_lo;
+  int64_t ld_hl;
+  float hl_scale;
   // NF4 operand (B from dequant)
   const uint8_t *scale_codes;
   const float *c2;
@@ -140,11 +143,95 @@ __device__ __forceinline__ void load_row128(const __nv_bfloat16 *src, int valid_
   }
 }
 
+constexpr int kGemmDequantThreads = 256;  // NF4 producer threads (warps 8..15)
+
+// Stores one 32-column chunk of accumulator row `row` (v = fp32 bit patterns).
+__device__ __forceinline__ void store_chunk32(const GemmArgs &args, int row, int col0, int ncol,
+                                              const uint32_t (&v)[32]) {
+  const bool full = ncol == 32;
+  if (args.out) {
+    if (!args.out_transpose) {
+      if (args.out_f32) {
+        float *o = reinterpret_cast<float *>(args.out) + (int64_t)row * args.ldo + col0;
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+          const float4 f = make_float4(__uint_as_float(v[j]) * args.out_scale, __uint_as_float(v[j + 1]) * args.out_scale,
+                                       __uint_as_float(v[j + 2]) * args.out_scale,
+                                       __uint_as_float(v[j + 3]) * args.out_scale);
+          if (full) {
+            *reinterpret_cast<float4 *>(o + j) = f;
+          } else {
+            if (j < ncol) o[j] = f.x;
+            if (j + 1 < ncol) o[j + 1] = f.y;
+            if (j + 2 < ncol) o[j + 2] = f.z;
+            if (j + 3 < ncol) o[j + 3] = f.w;
+          }
+        }
+      } else {
+        __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(args.out) + (int64_t)row * args.ldo + col0;
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            pk[i] = pack_bf16x2(__uint_as_float(v[j + 2 * i]) * args.out_scale,
+                                __uint_as_float(v[j + 2 * i + 1]) * args.out_scale);
+          if (full) {
+            *reinterpret_cast<uint4 *>(o + j) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          } else {
+            uint16_t *o16 = reinterpret_cast<uint16_t *>(o);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              if (j + i < ncol) o16[j + i] = (i & 1) ? (pk[i >> 1] >> 16) : (pk[i >> 1] & 0xffffu);
+          }
+        }
+      }
+    } else {
+      // out[col * ldo + row]: lanes write consecutive rows of each column.
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (j < ncol) {
+          const float x = __uint_as_float(v[j]) * args.out_scale;
+          if (args.out_f32) reinterpret_cast<float *>(args.out)[(int64_t)(col0 + j) * args.ldo + row] = x;
+          else reinterpret_cast<__nv_bfloat16 *>(args.out)[(int64_t)(col0 + j) * args.ldo + row] = __float2bfloat16_rn(x);
+        }
+      }
+    }
+  }
+  if (args.out_hi) {
+    uint16_t *oh = reinterpret_cast<uint16_t *>(args.out_hi) + (int64_t)row * args.ld_hl + col0;
+    uint16_t *ol = reinterpret_cast<uint16_t *>(args.out_lo) + (int64_t)row * args.ld_hl + col0;
+#pragma unroll
+    for (int j = 0; j < 32; j += 8) {
+      uint32_t h[4], l[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float a = __uint_as_float(v[j + 2 * i]) * args.hl_scale;
+        const float b = __uint_as_float(v[j + 2 * i + 1]) * args.hl_scale;
+        h[i] = pack_bf16x2(a, b);
+        l[i] = pack_bf16x2(a - bf16lo_to_f32(h[i]), b - bf16hi_to_f32(h[i]));
+      }
+      if (full) {
+        *reinterpret_cast<uint4 *>(oh + j) = make_uint4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<uint4 *>(ol + j) = make_uint4(l[0], l[1], l[2], l[3]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (j + i < ncol) {
+            oh[j + i] = (i & 1) ? (h[i >> 1] >> 16) : (h[i >> 1] & 0xffffu);
+            ol[j + i] = (i & 1) ? (l[i >> 1] >> 16) : (l[i >> 1] & 0xffffu);
+          }
+        }
+      }
+    }
+  }
+}
+
 template <bool A_MN, bool B_MN, bool NF4, int BN, int MT>
 __global__ void __launch_bounds__(GemmCfg<A_MN, B_MN, NF4, BN, MT>::THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-               const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmCodes,
-               const GemmArgs args) {
+               const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
+               const __grid_constant__ CUtensorMap tmCodes, const GemmArgs args) {
   using C = GemmCfg<A_MN, B_MN, NF4, BN, MT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -170,10 +257,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::SA; ++s) { ptx::mbar_init(&full_a[s], 1); ptx::mbar_init(&empty_a[s], 1); }
     for (int s = 0; s < C::SB; ++s) {
-      ptx::mbar_init(&full_b[s], NF4 ? 8 : 1);
+      ptx::mbar_init(&full_b[s], NF4 ? kGemmDequantThreads : 1);
       ptx::mbar_init(&empty_b[s], 1);
     }
-    for (int s = 0; s < C::SC; ++s) { ptx::mbar_init(&full_c[s], 1); ptx::mbar_init(&empty_c[s], 8); }
+    for (int s = 0; s < C::SC; ++s) { ptx::mbar_init(&full_c[s], 1); ptx::mbar_init(&empty_c[s], kGemmDequantThreads); }
     for (int s = 0; s < 2; ++s) { ptx::mbar_init(&acc_full[s], 1); ptx::mbar_init(&acc_empty[s], 4); }
     ptx::mbar_init(drain, 1);
     *abort_flag = 0;
@@ -182,6 +269,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   if (warp == 0 && lane == 0) {
     ptx::prefetch_tmap(&tmA);
     if (!NF4) ptx::prefetch_tmap(&tmB);
+    if (args.hilo) ptx::prefetch_tmap(&tmB2);
     if (args.lora_steps) ptx::prefetch_tmap(&tmA2);
     if (NF4) ptx::prefetch_tmap(&tmCodes);
   }
@@ -197,7 +285,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const int num_m = (args.M_rows + C::BM * MT - 1) / (C::BM * MT);
   const int num_n = (args.N_cols + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
-  const int steps = args.k_steps + args.lora_steps;
+  const int main_steps = args.k_steps * (args.hilo ? 2 : 1);
+  const int steps = main_steps + args.lora_steps;
 
   auto fail = [&]() {
     raise_status(args.status, QLORA_ERR_TIMEOUT);
@@ -214,7 +303,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const int m0 = (tile % num_m) * C::BM * MT;
         const int n0 = (tile / num_m) * BN;
         for (int ks = 0; ks < steps && ok; ++ks) {
-          const bool lora = ks >= args.k_steps;
+          const bool lora = ks >= main_steps;
+          const bool second = !lora && ks >= args.k_steps;  // hi/lo second pass
+          const int kk = second ? ks - args.k_steps : ks;
           if (NF4 && !lora) {
             if (!ptx::mbar_wait(&empty_c[sc], pc ^ 1, abort_flag)) { ok = false; break; }
             ptx::mbar_arrive_expect_tx(&full_c[sc], C::C_STAGE);
@@ -229,39 +320,36 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           ptx::mbar_arrive_expect_tx(&full_a[sa], bytes);
           uint8_t *dA = sA + sa * C::A_STAGE;
           if (lora) {
-            const int kk = (ks - args.k_steps) * 64;
-            for (int t = 0; t < MT; ++t) ptx::tma_load_2d(dA + t * 16384, &tmA2, &full_a[sa], kk, m0 + t * 128);
+            const int k2 = (ks - main_steps) * 64;
+            for (int t = 0; t < MT; ++t) ptx::tma_load_2d(dA + t * 16384, &tmA2, &full_a[sa], k2, m0 + t * 128);
           } else if (!A_MN) {
-            for (int t = 0; t < MT; ++t) ptx::tma_load_2d(dA + t * 16384, &tmA, &full_a[sa], ks * 64, m0 + t * 128);
+            for (int t = 0; t < MT; ++t) ptx::tma_load_2d(dA + t * 16384, &tmA, &full_a[sa], kk * 64, m0 + t * 128);
           } else {
-            for (int t = 0; t < MT * 2; ++t) ptx::tma_load_2d(dA + t * 8192, &tmA, &full_a[sa], m0 + t * 64, ks * 64);
+            for (int t = 0; t < MT * 2; ++t) ptx::tma_load_2d(dA + t * 8192, &tmA, &full_a[sa], m0 + t * 64, kk * 64);
           }
           if (!NF4) {
             uint8_t *dB = sB + sa * C::B_STAGE;
+            const CUtensorMap *mb = second ? &tmB2 : &tmB;
             if (!B_MN) {
-              ptx::tma_load_2d(dB, &tmB, &full_a[sa], ks * 64, n0);
+              ptx::tma_load_2d(dB, mb, &full_a[sa], kk * 64, n0);
             } else {
-              for (int t = 0; t < BN / 64; ++t) ptx::tma_load_2d(dB + t * 8192, &tmB, &full_a[sa], n0 + t * 64, ks * 64);
+              for (int t = 0; t < BN / 64; ++t) ptx::tma_load_2d(dB + t * 8192, mb, &full_a[sa], n0 + t * 64, kk * 64);
             }
           }
           ++issued_a;
           if (++sa == C::SA) { sa = 0; pa ^= 1; }
         }
       }
-      if (!ok) {
-        fail();
-        // Drain: every issued copy completes its full barrier phase; wait for the
-        // last `SA` / `SC` of them (older ones were consumed already).
-        for (int i = 0; i < C::SA && i < issued_a; ++i) {
-          sa = (sa + C::SA - 1) % C::SA;
-          if (sa == C::SA - 1) pa ^= 1;
-          ptx::mbar_wait(&full_a[sa], pa, nullptr);
-        }
-        for (int i = 0; NF4 && i < C::SC && i < issued_c; ++i) {
-          sc = (sc + C::SC - 1) % C::SC;
-          if (sc == C::SC - 1) pc ^= 1;
-          ptx::mbar_wait(&full_c[sc], pc, nullptr);
-        }
+      if (!ok) fail();
+      // Drain: the last (up to) SA / SC copies issued must have landed before the
+      // CTA may exit (older ones were consumed already).
+      for (int i = 0; i < C::SA && i < issued_a; ++i) {
+        if (sa == 0) { sa = C::SA - 1; pa ^= 1; } else { --sa; }
+        ptx::mbar_wait(&full_a[sa], pa, nullptr);
+      }
+      for (int i = 0; NF4 && i < C::SC && i < issued_c; ++i) {
+        if (sc == 0) { sc = C::SC - 1; pc ^= 1; } else { --sc; }
+        ptx::mbar_wait(&full_c[sc], pc, nullptr);
       }
     }
   } else if (warp == 1) {
@@ -278,7 +366,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * C::ACC_COLS;
         for (int ks = 0; ks < steps && ok; ++ks) {
-          const bool lora = ks >= args.k_steps;
+          const bool lora = ks >= main_steps;
           if (!ptx::mbar_wait(&full_a[sa], pa, abort_flag)) { ok = false; break; }
           if (NF4 && !ptx::mbar_wait(&full_b[sb], pb, abort_flag)) { ok = false; break; }
           ptx::tc_fence_after();
@@ -330,53 +418,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           ptx::tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS + t * BN + cb, v);
           ptx::tmem_ld_wait();
           const int col0 = n0 + cb;
-          if (row >= args.M_rows || col0 >= args.N_cols) continue;
-          const int ncol = min(32, args.N_cols - col0);
-          if (!args.out_transpose) {
-            if (args.out_f32) {
-              float *o = reinterpret_cast<float *>(args.out) + (int64_t)row * args.ldo + col0;
-              if (ncol == 32) {
-#pragma unroll
-                for (int j = 0; j < 32; j += 4)
-                  *reinterpret_cast<float4 *>(o + j) =
-                      make_float4(__uint_as_float(v[j]) * args.out_scale, __uint_as_float(v[j + 1]) * args.out_scale,
-                                  __uint_as_float(v[j + 2]) * args.out_scale, __uint_as_float(v[j + 3]) * args.out_scale);
-              } else {
-                for (int j = 0; j < ncol; ++j) o[j] = __uint_as_float(v[j]) * args.out_scale;
-              }
-            } else {
-              __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(args.out) + (int64_t)row * args.ldo + col0;
-              uint32_t pk[16];
-#pragma unroll
-              for (int j = 0; j < 16; ++j)
-                pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]) * args.out_scale,
-                                    __uint_as_float(v[2 * j + 1]) * args.out_scale);
-              if (ncol == 32) {
-#pragma unroll
-                for (int j = 0; j < 16; j += 4)
-                  *reinterpret_cast<uint4 *>(o + 2 * j) = make_uint4(pk[j], pk[j + 1], pk[j + 2], pk[j + 3]);
-              } else {
-                uint16_t *o16 = reinterpret_cast<uint16_t *>(o);
-                for (int j = 0; j < ncol; ++j) o16[j] = (j & 1) ? (pk[j >> 1] >> 16) : (pk[j >> 1] & 0xffffu);
-              }
-            }
-            if (args.out2) {
-              uint16_t *o2 = reinterpret_cast<uint16_t *>(args.out2) + (int64_t)row * args.ldo2 + col0;
-              for (int j = 0; j < ncol; j += 2) {
-                const uint32_t pk = pack_bf16x2(__uint_as_float(v[j]) * args.out2_scale,
-                                                __uint_as_float(v[min(j + 1, 31)]) * args.out2_scale);
-                o2[j] = pk & 0xffffu;
-                if (j + 1 < ncol) o2[j + 1] = pk >> 16;
-              }
-            }
-          } else {
-            // out[col * ldo + row]: lanes write consecutive rows of each column.
-            for (int j = 0; j < ncol; ++j) {
-              const float x = __uint_as_float(v[j]) * args.out_scale;
-              if (args.out_f32) reinterpret_cast<float *>(args.out)[(int64_t)(col0 + j) * args.ldo + row] = x;
-              else reinterpret_cast<__nv_bfloat16 *>(args.out)[(int64_t)(col0 + j) * args.ldo + row] = __float2bfloat16_rn(x);
-            }
-          }
+          if (row < args.M_rows && col0 < args.N_cols) store_chunk32(args, row, col0, min(32, args.N_cols - col0), v);
         }
       }
       ptx::tc_fence_before();
@@ -395,7 +437,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
       const int n0 = (tile / num_m) * BN;
       for (int ks = 0; ks < steps && ok; ++ks) {
-        const bool lora = ks >= args.k_steps;
+        const bool lora = ks >= main_steps;
         uint32_t o[32];
         // Which 128-byte row of which SW128 atom this thread fills.
         uint32_t atom_off, row_in;
@@ -412,8 +454,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           const uint8_t *cs = sC + sc * C::C_STAGE + d * 32;
           const uint4 c0 = *reinterpret_cast<const uint4 *>(cs);
           const uint4 c1 = *reinterpret_cast<const uint4 *>(cs + 16);
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(&empty_c[sc]);
+          ptx::mbar_arrive(&empty_c[sc]);
           if (++sc == C::SC) { sc = 0; pc ^= 1; }
           int64_t wrow, kblk;
           if (!B_MN) { wrow = n0 + d; kblk = ks; }
@@ -426,23 +467,32 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             for (int j = 0; j < 32; ++j) o[j] = 0u;
           }
         } else {
-          const int j0 = (ks - args.k_steps) * 64;
+          const int j0 = (ks - main_steps) * 64;
           if (!B_MN) {  // fwd: B2 = lora B [N, r], row n0 + d, cols j0..j0+63
             const int64_t n = n0 + d;
-            if (n < args.w_rows) load_row128(args.lora_b2 + n * args.lora_ld + j0, args.lora_r - j0, o);
-            else for (int j = 0; j < 32; ++j) o[j] = 0u;
+            if (n < args.w_rows) {
+              load_row128(args.lora_b2 + n * args.lora_ld + j0, args.lora_r - j0, o);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) o[j] = 0u;
+            }
           } else {      // bwd: B2 = lora A [r, K], row j0 + d/4, cols n0 + 64*(d%4) ..
             const int jr = j0 + (d >> 2);
             const int64_t kf = n0 + 64 * (d & 3);
-            if (jr < args.lora_r && kf < args.w_cols) load_row128(args.lora_b2 + (int64_t)jr * args.lora_ld + kf, 64, o);
-            else for (int j = 0; j < 32; ++j) o[j] = 0u;
+            if (jr < args.lora_r && kf < args.w_cols) {
+              load_row128(args.lora_b2 + (int64_t)jr * args.lora_ld + kf, 64, o);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) o[j] = 0u;
+            }
           }
         }
         if (!ptx::mbar_wait(&empty_b[sb], pb ^ 1, abort_flag)) { ok = false; break; }
         store_row128(sB + sb * C::B_STAGE + atom_off, row_in, o);
+        // Each thread orders its own writes before the tensor core's reads and
+        // arrives itself (one arrival per thread).
         ptx::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&full_b[sb]);
+        ptx::mbar_arrive(&full_b[sb]);
         if (++sb == C::SB) { sb = 0; pb ^= 1; }
       }
     }

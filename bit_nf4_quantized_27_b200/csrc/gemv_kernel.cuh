@@ -3,14 +3,16 @@
 //
 // HBM-bound: the packed codes (0.5 B/weight) dominate the traffic, so the kernel
 // streams them straight from HBM into registers with 8-byte vector loads and
-// decodes in registers.  Each byte (two codes) indexes a 256-entry table of bf16
+// decodes in registers.  Each byte (two codes) indexes a 256-entry table of fp16
 // level pairs (L[lo], L[hi]) kept in shared memory with one copy per lane (each
 // lane reads its own bank, so lookups never conflict); the pair is directly one
 // register of an m16n8k16 tensor-core A fragment (rows = 16 weight rows).  The
 // per-block scale S' = E4M3(q) * c2 multiplies the fp32 partial of each 64-weight
-// block after its four MMAs, so the sum equals X W'^T up to the bf16 rounding of
-// the products L * S' (the dequantised weight is bf16(L * S'); here L is exact in
-// the table and S' is applied in fp32).
+// block after its four MMAs.  X enters the MMA as fp16 after an exact per-token
+// power-of-two scaling (every bf16 value inside the scaled range is an fp16
+// value), undone on the partial sums.  The result equals X (L S')^T with L
+// rounded to fp16 (relative 2^-12); it differs from X W'^T only by the bf16
+// rounding of the dequantised weights W' = bf16(L S').
 //
 // Work split: 16 warps per CTA; warp w owns the w-th 256-wide slice of each
 // 4096-wide K chunk and keeps that slice of X as MMA B fragments in registers.  The
@@ -58,6 +60,24 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ void mma_16816_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// 2^e as a float (|e| <= 126).
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }
+
+// Two bf16 (packed) times 2^-e, converted to packed fp16.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_scaled(uint32_t v, float inv) {
+  const __half2 h = __floats2half2_rn(bf16lo_to_f32(v) * inv, bf16hi_to_f32(v) * inv);
+  return *reinterpret_cast<const uint32_t *>(&h);
+}
+
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -72,11 +92,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_lora_kernel(const Ge
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, q = lane & 3;
 
-  // Pair table: entry v = (bf16 L[v & 15]) | (bf16 L[v >> 4]) << 16, one copy per lane.
+  // Pair table: entry v = (fp16 L[v & 15]) | (fp16 L[v >> 4]) << 16, one copy per lane.
   for (int i = tid; i < 256 * 32; i += kGemvThreads) {
     const int v = i >> 5;
-    const float lo = __uint_as_float(kNf4LevelBits[v & 15]), hi = __uint_as_float(kNf4LevelBits[v >> 4]);
-    lut[i] = pack_bf16x2(lo, hi);
+    const __half2 h = __floats2half2_rn(__uint_as_float(kNf4LevelBits[v & 15]), __uint_as_float(kNf4LevelBits[v >> 4]));
+    lut[i] = *reinterpret_cast<const uint32_t *>(&h);
   }
   const int num_rg = static_cast<int>((a.N + 15) / 16);
   const int rg0 = blockIdx.x * a.rg_per_cta;
@@ -93,24 +113,52 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_lora_kernel(const Ge
     const int64_t kb0 = (int64_t)ch * 64 + warp * 4;  // first block of this warp's quad
     if (kb0 >= nbk) continue;
     const int nblk = static_cast<int>(nbk - kb0 < 4 ? nbk - kb0 : 4);
-    // X fragments: token (g + 8*ng), k = kb*64 + 16q + 4s + {0..3}
+    // X fragments: token (g + 8*ng), k = kb*64 + 16q + 4s + {0..3}, as fp16 after
+    // scaling token t's slice by 2^-e_t with max |x| * 2^-e_t in [2^14, 2^15).
     uint32_t xf[4][4][NG][2];
+    float unscale[NG][2];  // 2^e of tokens 2q, 2q+1 (+8 ng): the C fragment columns
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int ng = 0; ng < NG; ++ng) {
+      const int t = g + 8 * ng;
+      uint4 raw[4][2];
+      uint32_t mx = 0;
 #pragma unroll
-      for (int ng = 0; ng < NG; ++ng) {
-        const int t = g + 8 * ng;
+      for (int j = 0; j < 4; ++j) {
         uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
         if (j < nblk && t < a.M) {
           const uint4 *src = reinterpret_cast<const uint4 *>(a.X + (int64_t)t * a.K + (kb0 + j) * 64 + 16 * q);
           v0 = __ldg(src);
           v1 = __ldg(src + 1);
         }
-        xf[j][0][ng][0] = v0.x; xf[j][0][ng][1] = v0.y;
-        xf[j][1][ng][0] = v0.z; xf[j][1][ng][1] = v0.w;
-        xf[j][2][ng][0] = v1.x; xf[j][2][ng][1] = v1.y;
-        xf[j][3][ng][0] = v1.z; xf[j][3][ng][1] = v1.w;
+        raw[j][0] = v0;
+        raw[j][1] = v1;
+        mx = __vmaxu2(mx, __vmaxu2(__vmaxu2(v0.x & 0x7fff7fffu, v0.y & 0x7fff7fffu),
+                                   __vmaxu2(v0.z & 0x7fff7fffu, v0.w & 0x7fff7fffu)));
+        mx = __vmaxu2(mx, __vmaxu2(__vmaxu2(v1.x & 0x7fff7fffu, v1.y & 0x7fff7fffu),
+                                   __vmaxu2(v1.z & 0x7fff7fffu, v1.w & 0x7fff7fffu)));
       }
+      uint32_t m16 = max(mx & 0xffffu, mx >> 16);
+      m16 = max(m16, __shfl_xor_sync(0xffffffffu, m16, 1));
+      m16 = max(m16, __shfl_xor_sync(0xffffffffu, m16, 2));
+      // bf16 bits -> exponent E with max in [2^(E-1), 2^E); e = E - 15, clamped
+      const int E = m16 ? static_cast<int>((m16 >> 7) & 0xff) - 126 : 15;
+      const int e = max(-100, min(100, E - 15));
+      const float inv = pow2f(-e);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        xf[j][0][ng][0] = bf16x2_to_f16x2_scaled(raw[j][0].x, inv);
+        xf[j][0][ng][1] = bf16x2_to_f16x2_scaled(raw[j][0].y, inv);
+        xf[j][1][ng][0] = bf16x2_to_f16x2_scaled(raw[j][0].z, inv);
+        xf[j][1][ng][1] = bf16x2_to_f16x2_scaled(raw[j][0].w, inv);
+        xf[j][2][ng][0] = bf16x2_to_f16x2_scaled(raw[j][1].x, inv);
+        xf[j][2][ng][1] = bf16x2_to_f16x2_scaled(raw[j][1].y, inv);
+        xf[j][3][ng][0] = bf16x2_to_f16x2_scaled(raw[j][1].z, inv);
+        xf[j][3][ng][1] = bf16x2_to_f16x2_scaled(raw[j][1].w, inv);
+      }
+      // exponent of token (2q + i + 8 ng) lives in lane (2q + i) * 4
+      unscale[ng][0] = pow2f(__shfl_sync(0xffffffffu, e, (2 * q) * 4));
+      unscale[ng][1] = pow2f(__shfl_sync(0xffffffffu, e, (2 * q + 1) * 4));
+    }
 
     // Software pipeline over this CTA's row groups: codes of the next group are
     // loaded while the current one is decoded.
@@ -161,7 +209,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_lora_kernel(const Ge
           asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a2) : "r"(lut_lane + (b01 << 7)));
           asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a3) : "r"(lut_lane + (b11 << 7)));
 #pragma unroll
-          for (int ng = 0; ng < NG; ++ng) mma_16816(acc[ng], a0, a1, a2, a3, xf[j][s][ng][0], xf[j][s][ng][1]);
+          for (int ng = 0; ng < NG; ++ng) mma_16816_f16(acc[ng], a0, a1, a2, a3, xf[j][s][ng][0], xf[j][s][ng][1]);
         }
 #pragma unroll
         for (int ng = 0; ng < NG; ++ng) {
@@ -171,15 +219,15 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_lora_kernel(const Ge
           part[ng][3] = fmaf(S[1], acc[ng][3], part[ng][3]);
         }
       }
-      // red[i][warp][row][token] += partial (this warp is the only writer)
+      // red[i][warp][row][token] += partial * 2^e (this warp is the only writer)
       float *rb = red + ((size_t)i * kGemvWarps + warp) * 256;
 #pragma unroll
       for (int ng = 0; ng < NG; ++ng) {
         const int t = 2 * q + 8 * ng;
-        rb[g * 16 + t] += part[ng][0];
-        rb[g * 16 + t + 1] += part[ng][1];
-        rb[(g + 8) * 16 + t] += part[ng][2];
-        rb[(g + 8) * 16 + t + 1] += part[ng][3];
+        rb[g * 16 + t] += part[ng][0] * unscale[ng][0];
+        rb[g * 16 + t + 1] += part[ng][1] * unscale[ng][1];
+        rb[(g + 8) * 16 + t] += part[ng][2] * unscale[ng][0];
+        rb[(g + 8) * 16 + t + 1] += part[ng][3] * unscale[ng][1];
       }
 #pragma unroll
       for (int j = 0; j < 4; ++j) { cur[j][0] = nxt[j][0]; cur[j][1] = nxt[j][1]; }
@@ -201,8 +249,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_lora_kernel(const Ge
       for (int h = 0; h < 2; ++h) {
         const int64_t row = n0 + g + 8 * h;
         const uint32_t *src = reinterpret_cast<const uint32_t *>(a.B + row * a.r + j0 + 2 * q);
-        af[h] = row < a.N ? __ldg(src) : 0u;
-        af[2 + h] = row < a.N ? __ldg(src + 4) : 0u;
+        af[h] = (row < a.N && j0 + 2 * q < a.r) ? __ldg(src) : 0u;
+        af[2 + h] = (row < a.N && j0 + 8 + 2 * q < a.r) ? __ldg(src + 4) : 0u;
       }
 #pragma unroll
       for (int ng = 0; ng < NG; ++ng) {
@@ -210,8 +258,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_lora_kernel(const Ge
         uint32_t b0 = 0, b1 = 0;
         if (t < a.M) {
           const uint32_t *src = reinterpret_cast<const uint32_t *>(a.sT + (int64_t)t * a.r + j0 + 2 * q);
-          b0 = __ldg(src);
-          b1 = __ldg(src + 4);
+          if (j0 + 2 * q < a.r) b0 = __ldg(src);
+          if (j0 + 8 + 2 * q < a.r) b1 = __ldg(src + 4);
         }
         mma_16816(acc[ng], af[0], af[1], af[2], af[3], b0, b1);
       }
@@ -248,7 +296,8 @@ __global__ void __launch_bounds__(256) lora_down_small_kernel(const __nv_bfloat1
                                                               const __nv_bfloat16 *__restrict__ A, int M,
                                                               int64_t K, int r, float s,
                                                               __nv_bfloat16 *__restrict__ sT,
-                                                              __nv_bfloat16 *__restrict__ T_out) {
+                                                              __nv_bfloat16 *__restrict__ T_hi,
+                                                              __nv_bfloat16 *__restrict__ T_lo) {
   griddep_launch_dependents();
   __shared__ float red[8][kGemvMaxM];
   const int j = blockIdx.x;
@@ -288,7 +337,11 @@ __global__ void __launch_bounds__(256) lora_down_small_kernel(const __nv_bfloat1
 #pragma unroll
     for (int w = 0; w < 8; ++w) v += red[w][tid];
     sT[(int64_t)tid * r + j] = __float2bfloat16_rn(v * s);
-    if (T_out) T_out[(int64_t)tid * r + j] = __float2bfloat16_rn(v);
+    if (T_hi) {
+      const __nv_bfloat16 h = __float2bfloat16_rn(v);
+      T_hi[(int64_t)tid * r + j] = h;
+      T_lo[(int64_t)tid * r + j] = __float2bfloat16_rn(v - __bfloat162float(h));
+    }
   }
 }
 

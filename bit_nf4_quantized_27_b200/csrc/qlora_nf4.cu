@@ -70,7 +70,8 @@ qlora_status set_smem(F kernel, int bytes, int dev, std::once_flag *flags, qlora
 
 template <bool A_MN, bool B_MN, bool NF4, int BN, int MT>
 qlora_status launch_gemm(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmA2,
-                         const CUtensorMap &tmCodes, const GemmArgs &args, int dev, int sms, cudaStream_t st) {
+                         const CUtensorMap &tmB2, const CUtensorMap &tmCodes, const GemmArgs &args, int dev, int sms,
+                         cudaStream_t st) {
   using C = GemmCfg<A_MN, B_MN, NF4, BN, MT>;
   auto kernel = gemm_tc_kernel<A_MN, B_MN, NF4, BN, MT>;
   static std::once_flag flags[64];
@@ -81,7 +82,7 @@ qlora_status launch_gemm(const CUtensorMap &tmA, const CUtensorMap &tmB, const C
   const int num_n = (args.N_cols + BN - 1) / BN;
   const int tiles = num_m * num_n;
   const int grid = std::max(1, std::min(tiles, sms));
-  kernel<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tmA, tmB, tmA2, tmCodes, args);
+  kernel<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tmA, tmB, tmA2, tmB2, tmCodes, args);
   return launch_status();
 }
 
@@ -99,9 +100,10 @@ qlora_status check_lora(const qlora_lora *ad) {
 
 bool valid_dtype(qlora_dtype d) { return d == QLORA_F32 || d == QLORA_BF16; }
 
-// T = X A^T for the tokens: writes s*T (bf16) to sT and, if T_out, T (bf16).
+// T = X A^T for the tokens: writes s*T (bf16) to sT (if not null) and, if T_hi is
+// not null, T as the bf16 pair (T_hi, T_lo) with T_hi + T_lo = T to ~16 bits.
 qlora_status run_lora_down(const void *X, const qlora_lora *ad, int64_t M, int64_t K, float s, void *sT,
-                           void *T_out, uint32_t *status, int dev, int sms, cudaStream_t st) {
+                           void *T_hi, void *T_lo, uint32_t *status, int dev, int sms, cudaStream_t st) {
   CUtensorMap tmX, tmA;
   if (!tmap_bf16(&tmX, X, K, M, 64, 128) || !tmap_bf16(&tmA, ad->A, K, ad->r, 64, 64)) return QLORA_ERR_CUDA;
   GemmArgs g{};
@@ -112,11 +114,12 @@ qlora_status run_lora_down(const void *X, const qlora_lora *ad, int64_t M, int64
   g.ldo = ad->r;
   g.out_f32 = 0;
   g.out_scale = s;
-  g.out2 = T_out;
-  g.ldo2 = ad->r;
-  g.out2_scale = 1.0f;
+  g.out_hi = static_cast<__nv_bfloat16 *>(T_hi);
+  g.out_lo = static_cast<__nv_bfloat16 *>(T_lo);
+  g.ld_hl = ad->r;
+  g.hl_scale = 1.0f;
   g.status = status;
-  return launch_gemm<false, false, false, 64, 1>(tmX, tmA, tmX, tmX, g, dev, sms, st);
+  return launch_gemm<false, false, false, 64, 1>(tmX, tmA, tmX, tmX, tmX, g, dev, sms, st);
 }
 
 }  // namespace
@@ -151,7 +154,7 @@ size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r, int for
     bytes += mr;                                    // s*T
     if (M <= kGemvMaxM) bytes += gemv_workspace_bytes(M, N, K);
   } else {
-    bytes += 2 * mr;                                // s*U, recomputed T
+    bytes += 4 * mr;                                // s*U (hi, lo), recomputed T (hi, lo)
   }
   return bytes;
 }
@@ -225,10 +228,10 @@ qlora_status qlora_linear_fwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
   const size_t mr = align256(static_cast<size_t>(M) * ad->r * 2);
 
   if (M <= kGemvMaxM) {
+    __nv_bfloat16 *th = static_cast<__nv_bfloat16 *>(T_save);
     lora_down_small_kernel<<<ad->r, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(X),
                                                   static_cast<const __nv_bfloat16 *>(ad->A), (int)M, K, ad->r, sc,
-                                                  static_cast<__nv_bfloat16 *>(sT),
-                                                  static_cast<__nv_bfloat16 *>(T_save));
+                                                  static_cast<__nv_bfloat16 *>(sT), th, th ? th + M * ad->r : nullptr);
     if ((s = launch_status()) != QLORA_OK) return s;
     GemvArgs g{};
     g.codes = W->codes; g.scale_codes = W->scale_codes; g.c2 = W->c2;
@@ -243,7 +246,12 @@ qlora_status qlora_linear_fwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
     return launch_gemv(g, dev, sms, st);
   }
 
-  if ((s = run_lora_down(X, ad, M, K, sc, sT, T_save, status_ptr(ws), dev, sms, st)) != QLORA_OK) return s;
+  {
+    __nv_bfloat16 *th = static_cast<__nv_bfloat16 *>(T_save);
+    if ((s = run_lora_down(X, ad, M, K, sc, sT, th, th ? th + M * ad->r : nullptr, status_ptr(ws), dev, sms, st)) !=
+        QLORA_OK)
+      return s;
+  }
 
   CUtensorMap tmX, tmCodes, tmT;
   if (!tmap_bf16(&tmX, X, K, M, 64, 128) || !tmap_bf16(&tmT, sT, ad->r, M, 64, 128) ||
@@ -266,7 +274,7 @@ qlora_status qlora_linear_fwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
   g.lora_b2 = static_cast<const __nv_bfloat16 *>(ad->B);
   g.lora_ld = ad->r;
   g.status = status_ptr(ws);
-  return launch_gemm<false, false, true, 256, 1>(tmX, tmX, tmT, tmCodes, g, dev, sms, st);
+  return launch_gemm<false, false, true, 256, 1>(tmX, tmX, tmT, tmX, tmCodes, g, dev, sms, st);
 }
 
 qlora_status qlora_linear_bwd(const qlora_nf4_tensor *W, const qlora_lora *ad, const void *X, const void *dY,
@@ -290,17 +298,19 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
   const int r = ad->r;
   uint8_t *wsb = static_cast<uint8_t *>(ws);
   const size_t mr = align256(static_cast<size_t>(M) * r * 2);
-  void *sU = wsb + QLORA_STATUS_BYTES;
-  void *Tbuf = wsb + QLORA_STATUS_BYTES + mr;
+  void *sU_hi = wsb + QLORA_STATUS_BYTES;
+  void *sU_lo = wsb + QLORA_STATUS_BYTES + mr;
   uint32_t *status = status_ptr(ws);
 
-  const void *T = T_saved;
-  if (!T) {
-    // recompute T (unscaled) into the workspace; sU's slot serves as scratch for s*T
-    if ((s = run_lora_down(X, ad, M, K, sc, sU, Tbuf, status, dev, sms, st)) != QLORA_OK) return s;
-    T = Tbuf;
+  const void *T_hi = T_saved;
+  const void *T_lo = T_saved ? static_cast<const __nv_bfloat16 *>(T_saved) + M * r : nullptr;
+  if (!T_saved) {
+    void *th = wsb + QLORA_STATUS_BYTES + 2 * mr, *tl = wsb + QLORA_STATUS_BYTES + 3 * mr;
+    if ((s = run_lora_down(X, ad, M, K, sc, nullptr, th, tl, status, dev, sms, st)) != QLORA_OK) return s;
+    T_hi = th;
+    T_lo = tl;
   }
-  // U = dY B, stored as s*U (bf16)
+  // U = dY B, kept as the bf16 pair (hi, lo) of s*U
   {
     CUtensorMap tmDY, tmB;
     if (!tmap_bf16(&tmDY, dY, N, M, 64, 128) || !tmap_bf16(&tmB, ad->B, r, N, 64, 64)) return QLORA_ERR_CUDA;
@@ -308,16 +318,18 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
     g.M_rows = (int)M;
     g.N_cols = r;
     g.k_steps = (int)((N + 63) / 64);
-    g.out = sU;
-    g.ldo = r;
-    g.out_scale = sc;
+    g.out_hi = static_cast<__nv_bfloat16 *>(sU_hi);
+    g.out_lo = static_cast<__nv_bfloat16 *>(sU_lo);
+    g.ld_hl = r;
+    g.hl_scale = sc;
     g.status = status;
-    if ((s = launch_gemm<false, true, false, 64, 1>(tmDY, tmB, tmDY, tmDY, g, dev, sms, st)) != QLORA_OK) return s;
+    if ((s = launch_gemm<false, true, false, 64, 1>(tmDY, tmB, tmDY, tmDY, tmDY, g, dev, sms, st)) != QLORA_OK)
+      return s;
   }
   // dX = dY W' + (s U) A
   {
     CUtensorMap tmDY, tmU, tmCodes;
-    if (!tmap_bf16(&tmDY, dY, N, M, 64, 128) || !tmap_bf16(&tmU, sU, r, M, 64, 128) ||
+    if (!tmap_bf16(&tmDY, dY, N, M, 64, 128) || !tmap_bf16(&tmU, sU_hi, r, M, 64, 128) ||
         !make_tmap(&tmCodes, W->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, K / 2, 128, 64, false))
       return QLORA_ERR_CUDA;
     GemmArgs g{};
@@ -337,39 +349,47 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
     g.lora_b2 = static_cast<const __nv_bfloat16 *>(ad->A);
     g.lora_ld = K;
     g.status = status;
-    if ((s = launch_gemm<false, true, true, 256, 1>(tmDY, tmDY, tmU, tmCodes, g, dev, sms, st)) != QLORA_OK)
+    if ((s = launch_gemm<false, true, true, 256, 1>(tmDY, tmDY, tmU, tmDY, tmCodes, g, dev, sms, st)) != QLORA_OK)
       return s;
   }
-  // dA^T [K, r] = X^T (s U)  -> stored transposed into dA [r, K]
+  // dA^T [K, r] = X^T (s U_hi + s U_lo)  -> stored transposed into dA [r, K]
   {
-    CUtensorMap tmXt, tmU;
-    if (!tmap_bf16(&tmXt, X, K, M, 64, 64) || !tmap_bf16(&tmU, sU, r, M, 64, 64)) return QLORA_ERR_CUDA;
+    CUtensorMap tmXt, tmUh, tmUl;
+    if (!tmap_bf16(&tmXt, X, K, M, 64, 64) || !tmap_bf16(&tmUh, sU_hi, r, M, 64, 64) ||
+        !tmap_bf16(&tmUl, sU_lo, r, M, 64, 64))
+      return QLORA_ERR_CUDA;
     GemmArgs g{};
     g.M_rows = (int)K;
     g.N_cols = r;
     g.k_steps = (int)((M + 63) / 64);
+    g.hilo = 1;
     g.out = dA;
     g.ldo = K;
     g.out_f32 = grad_dtype == QLORA_F32;
     g.out_transpose = 1;
     g.out_scale = 1.0f;
     g.status = status;
-    if ((s = launch_gemm<true, true, false, 64, 1>(tmXt, tmU, tmXt, tmXt, g, dev, sms, st)) != QLORA_OK) return s;
+    if ((s = launch_gemm<true, true, false, 64, 1>(tmXt, tmUh, tmXt, tmUl, tmXt, g, dev, sms, st)) != QLORA_OK)
+      return s;
   }
-  // dB [N, r] = s dY^T T
+  // dB [N, r] = s dY^T (T_hi + T_lo)
   {
-    CUtensorMap tmDYt, tmT;
-    if (!tmap_bf16(&tmDYt, dY, N, M, 64, 64) || !tmap_bf16(&tmT, T, r, M, 64, 64)) return QLORA_ERR_CUDA;
+    CUtensorMap tmDYt, tmTh, tmTl;
+    if (!tmap_bf16(&tmDYt, dY, N, M, 64, 64) || !tmap_bf16(&tmTh, T_hi, r, M, 64, 64) ||
+        !tmap_bf16(&tmTl, T_lo, r, M, 64, 64))
+      return QLORA_ERR_CUDA;
     GemmArgs g{};
     g.M_rows = (int)N;
     g.N_cols = r;
     g.k_steps = (int)((M + 63) / 64);
+    g.hilo = 1;
     g.out = dB;
     g.ldo = r;
     g.out_f32 = grad_dtype == QLORA_F32;
     g.out_scale = sc;
     g.status = status;
-    if ((s = launch_gemm<true, true, false, 64, 1>(tmDYt, tmT, tmDYt, tmDYt, g, dev, sms, st)) != QLORA_OK) return s;
+    if ((s = launch_gemm<true, true, false, 64, 1>(tmDYt, tmTh, tmDYt, tmTl, tmDYt, g, dev, sms, st)) != QLORA_OK)
+      return s;
   }
   return QLORA_OK;
 }

@@ -49,19 +49,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(parity), "r"(20000u)  // suspend-time hint, ns
+      : "r"(smem_addr(bar)), "r"(parity), "r"(1000000u)  // suspend-time hint, ns
       : "memory");
   return ok != 0;
 }
 
-// Bounded wait: polls at most `limit` times (each poll may suspend up to the hint
-// above), so a wait that can never complete ends in well under a few seconds.
-constexpr uint32_t kWaitLimit = 1u << 17;
+// Bounded wait: gives up after about two seconds of %globaltimer (and after a
+// hard cap on polls), so a wait that can never complete ends the kernel with an
+// error status instead of hanging the GPU.
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr uint32_t kWaitPollCap = 1u << 26;
 
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const volatile int *abort_flag) {
-  for (uint32_t i = 0; i < kWaitLimit; ++i) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1; i < kWaitPollCap; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (abort_flag && *abort_flag) return false;
+    if ((i & 15) == 0) {
+      if (abort_flag && *abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitNs) return false;
+    }
   }
   return false;
 }

@@ -138,7 +138,9 @@ QLORA_API qlora_status qlora_nf4_dequantize(const qlora_nf4_tensor *w, void *W_o
  * works", forward rule):  Y [M, N] = X W'^T + s (X A^T) B^T.
  *   X      bf16 [M, K] device
  *   Y      [M, N] device, bf16 or float32 (y_dtype)
- *   T_save nullable bf16 [M, r] device: receives T = X A^T for the backward pass
+ *   T_save nullable bf16 [2, M, r] device: receives T = X A^T for the backward
+ *          pass as the pair T_hi = bf16(T) (first M*r elements) and
+ *          T_lo = bf16(T - T_hi) (next M*r), so T_hi + T_lo carries ~16 bits
  *   ws     device workspace of ws_bytes >= qlora_workspace_bytes(M, N, K, r, 0)
  * M >= 1.  M <= 16 takes the decode (GEMV) path; larger M the tensor-core path. */
 QLORA_API qlora_status qlora_linear_fwd(const qlora_nf4_tensor *W, const qlora_lora *adapter, const void *X,
@@ -150,7 +152,7 @@ QLORA_API qlora_status qlora_linear_fwd(const qlora_nf4_tensor *W, const qlora_l
  *   dX [M, K] = dY W' + s U A          (dx_dtype: bf16 or float32)
  *   dA [r, K] = s U^T X                (grad_dtype: bf16 or float32)
  *   dB [N, r] = s dY^T T,  T = X A^T   (grad_dtype)
- * T_saved: nullable bf16 [M, r] from qlora_linear_fwd; NULL recomputes it.
+ * T_saved: nullable bf16 [2, M, r] pair from qlora_linear_fwd; NULL recomputes it.
  * dY bf16 [M, N].  dX, dA, dB are overwritten (not accumulated).  W gets no
  * gradient. */
 QLORA_API qlora_status qlora_linear_bwd(const qlora_nf4_tensor *W, const qlora_lora *adapter, const void *X,
