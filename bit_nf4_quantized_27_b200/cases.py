@@ -1,0 +1,82 @@
+"""Single named cases of the hot path, for profiling one kernel at a time.
+
+Usage: python -m bit_nf4_quantized_27_b200.cases CASE [--reps R]
+
+CASE is one of:
+  fwd_8192      forward of one 8192x8192 layer, 4096 tokens, r=64 (65B-shaped q)
+  bwd_8192      backward of the same layer
+  fwd_11008     forward of 11008x4096 (gate/up of the Llama-7B block), 2048 tokens
+  gemv_m1 / gemv_m4 / gemv_m16   decode forward, W 11008x4096, r=64
+  quant_11008   quantise an 11008x4096 bf16 weight
+  dequant_11008 dequantise it
+Inputs are drawn on the device from fixed seeds; every run exits 0 on success.
+"""
+
+import argparse
+import sys
+
+import torch
+
+from . import binding as bd
+
+
+def _layer(n, k, m, r=64, seed=1):
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    w = (torch.randn(n, k, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    x = torch.randn(m, k, generator=g, device="cuda").to(torch.bfloat16)
+    a = (torch.randn(r, k, generator=g, device="cuda") / k ** 0.5).to(torch.bfloat16)
+    b = (torch.randn(n, r, generator=g, device="cuda") * 0.01).to(torch.bfloat16)
+    dy = torch.randn(m, n, generator=g, device="cuda").to(torch.bfloat16)
+    return w, x, a, b, dy
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("case")
+    ap.add_argument("--reps", type=int, default=3)
+    args = ap.parse_args(argv)
+    c = args.case
+    torch.cuda.set_device(0)
+    if c.startswith(("fwd", "bwd")):
+        n, k, m = {"8192": (8192, 8192, 4096), "11008": (11008, 4096, 2048)}[c.split("_")[1]]
+        w, x, a, b, dy = _layer(n, k, m)
+        q = bd.quantize(w)
+        y, t = bd.linear_fwd(q, a, b, 16.0, x)
+        ws_f = bd.new_workspace(bd.workspace_bytes(m, n, k, 64, False))
+        ws_b = bd.new_workspace(bd.workspace_bytes(m, n, k, 64, True))
+        for _ in range(args.reps):
+            if c.startswith("fwd"):
+                bd.linear_fwd(q, a, b, 16.0, x, ws=ws_f, out=y, t_out=t)
+            else:
+                bd.linear_bwd(q, a, b, 16.0, x, dy, t, ws=ws_b)
+        st = bd.read_status(ws_f) or bd.read_status(ws_b)
+    elif c.startswith("gemv"):
+        m = int(c.split("_m")[1])
+        w, x, a, b, _ = _layer(11008, 4096, m)
+        q = bd.quantize(w)
+        ws = bd.new_workspace(bd.workspace_bytes(m, 11008, 4096, 64, False))
+        for _ in range(args.reps):
+            bd.linear_fwd(q, a, b, 16.0, x, ws=ws)
+        st = bd.read_status(ws)
+    elif c in ("quant_11008", "dequant_11008"):
+        w, *_ = _layer(11008, 4096, 1)
+        ws = bd.new_workspace(bd.STATUS_BYTES)
+        q = bd.quantize(w, ws=ws)
+        out = torch.empty_like(w)
+        for _ in range(args.reps):
+            if c.startswith("quant"):
+                bd.quantize(w, out=q, ws=ws)
+            else:
+                bd.dequantize(q, out=out)
+        st = bd.read_status(ws)
+    else:
+        raise SystemExit(f"unknown case {c}")
+    torch.cuda.synchronize()
+    if st:
+        raise SystemExit(f"device status {bd.STATUS_NAMES[st]}")
+    print(f"{c}: ok")
+
+
+if __name__ == "__main__":
+    sys.exit(main())

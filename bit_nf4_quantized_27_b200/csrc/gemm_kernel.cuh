@@ -432,35 +432,65 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 #pragma unroll
     for (int j = 0; j < 16; ++j) lv[j] = __uint_as_float(kNf4LevelBits[j]);
     const int64_t kblocks = args.w_cols / 64;
+    // Which 128-byte row of which SW128 atom this thread fills (same for every step).
+    uint32_t atom_off, row_in;
+    if (!B_MN) {  // B[n, k]: thread = W row n0 + d, one 64-code block (K step ks)
+      atom_off = (d >> 3) * 1024;
+      row_in = d & 7;
+    } else {      // B[kf, n]: thread = (W row ks*64 + d/4, 64 in-features block d%4)
+      atom_off = (d & 3) * 8192 + ((d >> 2) >> 3) * 1024;
+      row_in = (d >> 2) & 7;
+    }
+    // Code bytes of this thread: 32 at d*32 in the stage.  The two 16-byte halves
+    // are read in an order that keeps each quarter-warp on distinct banks.
+    const uint32_t half_first = (d >> 2) & 1;
+    // Block scale of flat step (tile, ks), fetched two steps ahead of its use.
+    auto scale_src = [&](int tile, int ks, uint32_t &qv, float &cv) {
+      qv = 0x100u;  // marks "no block" (rows past N, LoRA steps)
+      cv = 0.0f;
+      if (tile >= num_tiles || ks >= main_steps) return;
+      const int n0 = (tile / num_m) * BN;
+      int64_t wrow, kblk;
+      if (!B_MN) { wrow = n0 + d; kblk = ks; }
+      else { wrow = (int64_t)ks * 64 + (d >> 2); kblk = n0 / 64 + (d & 3); }
+      if (wrow < args.w_rows && kblk < kblocks) {
+        const int64_t b = wrow * kblocks + kblk;
+        qv = __ldg(args.scale_codes + b);
+        cv = __ldg(args.c2 + (b >> 8));
+      }
+    };
+    auto next_pos = [&](int &tile, int &ks) {
+      if (++ks == steps) { ks = 0; tile += gridDim.x; }
+    };
+    int t1 = blockIdx.x, k1 = 0, t2 = blockIdx.x, k2 = 0;
+    next_pos(t2, k2);
+    uint32_t q_cur, q_nxt;
+    float c_cur, c_nxt;
+    scale_src(t1, k1, q_cur, c_cur);
+    scale_src(t2, k2, q_nxt, c_nxt);
+    int tp = t2, kp = k2;  // position of the most recent prefetch
     uint32_t sb = 0, pb = 0, sc = 0, pc = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
       const int n0 = (tile / num_m) * BN;
       for (int ks = 0; ks < steps && ok; ++ks) {
         const bool lora = ks >= main_steps;
+        // prefetch the scale two steps ahead
+        next_pos(tp, kp);
+        uint32_t q_pf;
+        float c_pf;
+        scale_src(tp, kp, q_pf, c_pf);
         uint32_t o[32];
-        // Which 128-byte row of which SW128 atom this thread fills.
-        uint32_t atom_off, row_in;
-        if (!B_MN) {  // B[n, k]: thread = W row n0 + d, one 64-code block (K step ks)
-          atom_off = (d >> 3) * 1024;
-          row_in = d & 7;
-        } else {      // B[kf, n]: thread = (W row ks*64 + d/4, 64 in-features block d%4)
-          const int nl = d >> 2, a = d & 3;
-          atom_off = a * 8192 + (nl >> 3) * 1024;
-          row_in = nl & 7;
-        }
         if (!lora) {
           if (!ptx::mbar_wait(&full_c[sc], pc, abort_flag)) { ok = false; break; }
           const uint8_t *cs = sC + sc * C::C_STAGE + d * 32;
-          const uint4 c0 = *reinterpret_cast<const uint4 *>(cs);
-          const uint4 c1 = *reinterpret_cast<const uint4 *>(cs + 16);
+          const uint4 ca = *reinterpret_cast<const uint4 *>(cs + 16 * half_first);
+          const uint4 cb = *reinterpret_cast<const uint4 *>(cs + 16 * (1 - half_first));
           ptx::mbar_arrive(&empty_c[sc]);
           if (++sc == C::SC) { sc = 0; pc ^= 1; }
-          int64_t wrow, kblk;
-          if (!B_MN) { wrow = n0 + d; kblk = ks; }
-          else { wrow = (int64_t)ks * 64 + (d >> 2); kblk = n0 / 64 + (d & 3); }
-          if (wrow < args.w_rows && kblk < kblocks) {
-            const float S = block_scale(args.scale_codes, args.c2, wrow * kblocks + kblk);
+          const uint4 c0 = half_first ? cb : ca, c1 = half_first ? ca : cb;
+          if (q_cur != 0x100u) {
+            const float S = __fmul_rn(e4m3_to_f32(static_cast<uint8_t>(q_cur)), c_cur);
             nf4_decode64(c0, c1, S, lv, o);
           } else {
 #pragma unroll
@@ -487,6 +517,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             }
           }
         }
+        q_cur = q_nxt; c_cur = c_nxt;
+        q_nxt = q_pf; c_nxt = c_pf;
         if (!ptx::mbar_wait(&empty_b[sb], pb ^ 1, abort_flag)) { ok = false; break; }
         store_row128(sB + sb * C::B_STAGE + atom_off, row_in, o);
         // Each thread orders its own writes before the tensor core's reads and

@@ -160,49 +160,78 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_lora_kernel(const Ge
       unscale[ng][1] = pow2f(__shfl_sync(0xffffffffu, e, (2 * q + 1) * 4));
     }
 
-    // Software pipeline over this CTA's row groups: codes of the next group are
-    // loaded while the current one is decoded.
-    uint2 cur[4][2], nxt[4][2];
-    auto load_codes = [&](int i, uint2 (&dst)[4][2]) {
-      const int64_t n0 = (int64_t)(rg0 + i) * 16;
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int64_t row = n0 + g + 8 * h;
-          if (j < nblk && row < a.N)
-            dst[j][h] = __ldg(reinterpret_cast<const uint2 *>(a.codes + row * row_bytes + (kb0 + j) * 32 + 8 * q));
-          else
-            dst[j][h] = make_uint2(0x77777777u, 0x77777777u);
-        }
+    // Software pipeline over this CTA's row groups: codes and scale bytes of the
+    // next PD groups are in flight while the current one is decoded.
+    constexpr int PD = 1;
+    struct Stage {
+      uint2 c[4][2];   // [block][row half] 8 code bytes
+      uint32_t q[2];   // 4 E4M3 scale bytes per row half (blocks kb0..kb0+3)
+      float c2[2][2];  // c2 of the quad's first group and, if it crosses one, the next
+      uint32_t split[2];  // blocks j >= split use c2[h][1]
     };
-    if (my_rg > 0) load_codes(0, cur);
-    for (int i = 0; i < my_rg; ++i) {
-      if (i + 1 < my_rg) load_codes(i + 1, nxt);
+    const bool quad_ok = (nbk & 3) == 0 && nblk == 4;  // 4-byte scale loads are aligned
+    auto load_stage = [&](int i, Stage &st) {
       const int64_t n0 = (int64_t)(rg0 + i) * 16;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int64_t row = n0 + g + 8 * h;
+        const bool rv = row < a.N;
+        const uint8_t *cp = a.codes + row * row_bytes + kb0 * 32 + 8 * q;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          st.c[j][h] = (rv && j < nblk) ? __ldg(reinterpret_cast<const uint2 *>(cp + 32 * j))
+                                        : make_uint2(0x77777777u, 0x77777777u);
+        const int64_t b0 = row * nbk + kb0;
+        if (rv && quad_ok) {
+          st.q[h] = __ldg(reinterpret_cast<const uint32_t *>(a.scale_codes + b0));
+        } else {
+          uint32_t w = 0;
+          for (int j = 0; j < 4; ++j)
+            if (rv && j < nblk) w |= static_cast<uint32_t>(__ldg(a.scale_codes + b0 + j)) << (8 * j);
+          st.q[h] = w;
+        }
+        // a quad crosses at most one boundary between groups of 256 blocks
+        const uint32_t left = 256u - static_cast<uint32_t>(b0 & 255);
+        st.split[h] = left < 4u ? left : 4u;
+        st.c2[h][0] = rv ? __ldg(a.c2 + (b0 >> 8)) : 0.0f;
+        st.c2[h][1] = (rv && left < 4u && left < static_cast<uint32_t>(nblk)) ? __ldg(a.c2 + (b0 >> 8) + 1) : st.c2[h][0];
+      }
+    };
+    Stage stg[PD + 1];
+#pragma unroll
+    for (int p = 0; p < PD; ++p)
+      if (p < my_rg) load_stage(p, stg[p]);
+    for (int i = 0; i < my_rg; ++i) {
+      Stage &cur = stg[0];
+      if (i + PD < my_rg) load_stage(i + PD, stg[PD]);
+      // block scales of rows g (h=0) and g+8 (h=1)
+      float S[2][4];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(cur.q[h] & 0xffffu), __NV_E4M3);
+        const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(cur.q[h] >> 16), __NV_E4M3);
+        const float2 f01 = __half22float2(__half2(lo)), f23 = __half22float2(__half2(hi));
+        S[h][0] = __fmul_rn(f01.x, cur.c2[h][0]);
+        S[h][1] = __fmul_rn(f01.y, cur.split[h] > 1 ? cur.c2[h][0] : cur.c2[h][1]);
+        S[h][2] = __fmul_rn(f23.x, cur.split[h] > 2 ? cur.c2[h][0] : cur.c2[h][1]);
+        S[h][3] = __fmul_rn(f23.y, cur.split[h] > 3 ? cur.c2[h][0] : cur.c2[h][1]);
+      }
       float part[NG][4];
 #pragma unroll
       for (int ng = 0; ng < NG; ++ng) part[ng][0] = part[ng][1] = part[ng][2] = part[ng][3] = 0.0f;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        if (j >= nblk) break;
-        float S[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int64_t row = n0 + g + 8 * h;
-          S[h] = row < a.N ? block_scale(a.scale_codes, a.c2, row * nbk + kb0 + j) : 0.0f;
-        }
         float acc[NG][4];
 #pragma unroll
         for (int ng = 0; ng < NG; ++ng) acc[ng][0] = acc[ng][1] = acc[ng][2] = acc[ng][3] = 0.0f;
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
           // bytes 2s, 2s+1 of the 8 code bytes of rows g (h=0) and g+8 (h=1)
-          const uint32_t w0 = (s < 2) ? cur[j][0].x : cur[j][0].y;
-          const uint32_t w1 = (s < 2) ? cur[j][1].x : cur[j][1].y;
-          const int sh = (s & 1) * 16;
-          const uint32_t b00 = (w0 >> sh) & 0xffu, b01 = (w0 >> (sh + 8)) & 0xffu;
-          const uint32_t b10 = (w1 >> sh) & 0xffu, b11 = (w1 >> (sh + 8)) & 0xffu;
+          const uint32_t w0 = (s < 2) ? cur.c[j][0].x : cur.c[j][0].y;
+          const uint32_t w1 = (s < 2) ? cur.c[j][1].x : cur.c[j][1].y;
+          const uint32_t p0 = (2 * s) & 3, p1 = (2 * s + 1) & 3;
+          const uint32_t b00 = __byte_perm(w0, 0u, 0x4440u | p0), b01 = __byte_perm(w0, 0u, 0x4440u | p1);
+          const uint32_t b10 = __byte_perm(w1, 0u, 0x4440u | p0), b11 = __byte_perm(w1, 0u, 0x4440u | p1);
           uint32_t a0, a1, a2, a3;
           asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a0) : "r"(lut_lane + (b00 << 7)));
           asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a1) : "r"(lut_lane + (b10 << 7)));
@@ -213,10 +242,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_lora_kernel(const Ge
         }
 #pragma unroll
         for (int ng = 0; ng < NG; ++ng) {
-          part[ng][0] = fmaf(S[0], acc[ng][0], part[ng][0]);
-          part[ng][1] = fmaf(S[0], acc[ng][1], part[ng][1]);
-          part[ng][2] = fmaf(S[1], acc[ng][2], part[ng][2]);
-          part[ng][3] = fmaf(S[1], acc[ng][3], part[ng][3]);
+          part[ng][0] = fmaf(S[0][j], acc[ng][0], part[ng][0]);
+          part[ng][1] = fmaf(S[0][j], acc[ng][1], part[ng][1]);
+          part[ng][2] = fmaf(S[1][j], acc[ng][2], part[ng][2]);
+          part[ng][3] = fmaf(S[1][j], acc[ng][3], part[ng][3]);
         }
       }
       // red[i][warp][row][token] += partial * 2^e (this warp is the only writer)
@@ -230,7 +259,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_lora_kernel(const Ge
         rb[(g + 8) * 16 + t + 1] += part[ng][3] * unscale[ng][1];
       }
 #pragma unroll
-      for (int j = 0; j < 4; ++j) { cur[j][0] = nxt[j][0]; cur[j][1] = nxt[j][1]; }
+      for (int p = 0; p < PD; ++p) stg[p] = stg[p + 1];
     }
   }
 

@@ -15,6 +15,13 @@
 
 using namespace qlora;
 
+// Token subtiles of 128 per fused-GEMM tile: each decoded 256x64 W' tile feeds
+// MT accumulators, so the decode work per tensor-core FLOP falls as 1/MT.
+#ifndef QLORA_FUSED_MT
+#define QLORA_FUSED_MT 2
+#endif
+constexpr int kFusedMT = QLORA_FUSED_MT;
+
 namespace {
 
 // ---------------------------------------------------------------------------
@@ -274,7 +281,7 @@ qlora_status qlora_linear_fwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
   g.lora_b2 = static_cast<const __nv_bfloat16 *>(ad->B);
   g.lora_ld = ad->r;
   g.status = status_ptr(ws);
-  return launch_gemm<false, false, true, 256, 1>(tmX, tmX, tmT, tmX, tmCodes, g, dev, sms, st);
+  return launch_gemm<false, false, true, 256, kFusedMT>(tmX, tmX, tmT, tmX, tmCodes, g, dev, sms, st);
 }
 
 qlora_status qlora_linear_bwd(const qlora_nf4_tensor *W, const qlora_lora *ad, const void *X, const void *dY,
@@ -349,7 +356,7 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
     g.lora_b2 = static_cast<const __nv_bfloat16 *>(ad->A);
     g.lora_ld = K;
     g.status = status;
-    if ((s = launch_gemm<false, true, true, 256, 1>(tmDY, tmDY, tmU, tmDY, tmCodes, g, dev, sms, st)) != QLORA_OK)
+    if ((s = launch_gemm<false, true, true, 256, kFusedMT>(tmDY, tmDY, tmU, tmDY, tmCodes, g, dev, sms, st)) != QLORA_OK)
       return s;
   }
   // dA^T [K, r] = X^T (s U_hi + s U_lo)  -> stored transposed into dA [r, K]
