@@ -432,101 +432,115 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 #pragma unroll
     for (int j = 0; j < 16; ++j) lv[j] = __uint_as_float(kNf4LevelBits[j]);
     const int64_t kblocks = args.w_cols / 64;
-    // Which 128-byte row of which SW128 atom this thread fills (same for every step).
-    uint32_t atom_off, row_in;
-    if (!B_MN) {  // B[n, k]: thread = W row n0 + d, one 64-code block (K step ks)
+    // Thread -> (B row it fills, code bytes it reads).  Chosen so that, within
+    // every quarter-warp, the eight 16-byte code reads and the eight swizzled
+    // 16-byte operand writes each fall on distinct banks.
+    int wr, fb;                // fwd: W row n0 + wr; dX: W row ks*64 + wr, in-feature block fb
+    uint32_t atom_off, row_in, code_off, half_first;
+    if (!B_MN) {
+      wr = d;
+      fb = 0;
       atom_off = (d >> 3) * 1024;
       row_in = d & 7;
-    } else {      // B[kf, n]: thread = (W row ks*64 + d/4, 64 in-features block d%4)
-      atom_off = (d & 3) * 8192 + ((d >> 2) >> 3) * 1024;
-      row_in = (d >> 2) & 7;
+      code_off = d * 32;
+      half_first = (d >> 2) & 1;
+    } else {
+      const int P = d >> 3, j = d & 7;
+      wr = 8 * (P & 7) + j;                  // 0..63: W row within the K step
+      fb = ((j >> 1) + (P >> 3)) & 3;        // 64-feature block within the tile
+      atom_off = fb * 8192 + (wr >> 3) * 1024;
+      row_in = wr & 7;
+      code_off = wr * 128 + fb * 32;
+      half_first = j & 1;
     }
-    // Code bytes of this thread: 32 at d*32 in the stage.  The two 16-byte halves
-    // are read in an order that keeps each quarter-warp on distinct banks.
-    const uint32_t half_first = (d >> 2) & 1;
-    // Block scale of flat step (tile, ks), fetched two steps ahead of its use.
+    // Block scale (E4M3 byte, c2) of flat step (tile, ks), loaded two steps
+    // before use into one of two register slots that are only ever refilled
+    // after being consumed.
     auto scale_src = [&](int tile, int ks, uint32_t &qv, float &cv) {
-      qv = 0x100u;  // marks "no block" (rows past N, LoRA steps)
+      qv = 0x100u;  // "no block": rows past N, LoRA steps, past the last tile
       cv = 0.0f;
       if (tile >= num_tiles || ks >= main_steps) return;
       const int n0 = (tile / num_m) * BN;
       int64_t wrow, kblk;
-      if (!B_MN) { wrow = n0 + d; kblk = ks; }
-      else { wrow = (int64_t)ks * 64 + (d >> 2); kblk = n0 / 64 + (d & 3); }
+      if (!B_MN) { wrow = n0 + wr; kblk = ks; }
+      else { wrow = (int64_t)ks * 64 + wr; kblk = n0 / 64 + fb; }
       if (wrow < args.w_rows && kblk < kblocks) {
         const int64_t b = wrow * kblocks + kblk;
         qv = __ldg(args.scale_codes + b);
         cv = __ldg(args.c2 + (b >> 8));
       }
     };
-    auto next_pos = [&](int &tile, int &ks) {
-      if (++ks == steps) { ks = 0; tile += gridDim.x; }
-    };
-    int t1 = blockIdx.x, k1 = 0, t2 = blockIdx.x, k2 = 0;
-    next_pos(t2, k2);
-    uint32_t q_cur, q_nxt;
-    float c_cur, c_nxt;
-    scale_src(t1, k1, q_cur, c_cur);
-    scale_src(t2, k2, q_nxt, c_nxt);
-    int tp = t2, kp = k2;  // position of the most recent prefetch
     uint32_t sb = 0, pb = 0, sc = 0, pc = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+    int tile = blockIdx.x, ks = 0;        // step being produced
+    int ptile = blockIdx.x, pks = 0;      // step whose scale is fetched next
+    auto advance = [&](int &t, int &k) {
+      if (++k == steps) { k = 0; t += gridDim.x; }
+    };
+    uint32_t qa, qb;
+    float ca, cb;
+    scale_src(ptile, pks, qa, ca);
+    advance(ptile, pks);
+    scale_src(ptile, pks, qb, cb);
+    advance(ptile, pks);
+
+    auto produce = [&](uint32_t &qs, float &cs) -> bool {
+      const bool lora = ks >= main_steps;
       const int n0 = (tile / num_m) * BN;
-      for (int ks = 0; ks < steps && ok; ++ks) {
-        const bool lora = ks >= main_steps;
-        // prefetch the scale two steps ahead
-        next_pos(tp, kp);
-        uint32_t q_pf;
-        float c_pf;
-        scale_src(tp, kp, q_pf, c_pf);
-        uint32_t o[32];
-        if (!lora) {
-          if (!ptx::mbar_wait(&full_c[sc], pc, abort_flag)) { ok = false; break; }
-          const uint8_t *cs = sC + sc * C::C_STAGE + d * 32;
-          const uint4 ca = *reinterpret_cast<const uint4 *>(cs + 16 * half_first);
-          const uint4 cb = *reinterpret_cast<const uint4 *>(cs + 16 * (1 - half_first));
-          ptx::mbar_arrive(&empty_c[sc]);
-          if (++sc == C::SC) { sc = 0; pc ^= 1; }
-          const uint4 c0 = half_first ? cb : ca, c1 = half_first ? ca : cb;
-          if (q_cur != 0x100u) {
-            const float S = __fmul_rn(e4m3_to_f32(static_cast<uint8_t>(q_cur)), c_cur);
-            nf4_decode64(c0, c1, S, lv, o);
+      uint32_t o[32];
+      if (!lora) {
+        if (!ptx::mbar_wait(&full_c[sc], pc, abort_flag)) return false;
+        const uint8_t *csrc = sC + sc * C::C_STAGE + code_off;
+        const uint4 x0 = *reinterpret_cast<const uint4 *>(csrc + 16 * half_first);
+        const uint4 x1 = *reinterpret_cast<const uint4 *>(csrc + 16 * (1 - half_first));
+        ptx::mbar_arrive(&empty_c[sc]);
+        if (++sc == C::SC) { sc = 0; pc ^= 1; }
+        const uint4 c0 = half_first ? x1 : x0, c1 = half_first ? x0 : x1;
+        if (qs != 0x100u) {
+          const float S = __fmul_rn(e4m3_to_f32(static_cast<uint8_t>(qs)), cs);
+          nf4_decode64(c0, c1, S, lv, o);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[j] = 0u;
+        }
+      } else {
+        const int j0 = (ks - main_steps) * 64;
+        if (!B_MN) {  // fwd: B2 = lora B [N, r], row n0 + wr, cols j0..j0+63
+          const int64_t n = n0 + wr;
+          if (n < args.w_rows) {
+            load_row128(args.lora_b2 + n * args.lora_ld + j0, args.lora_r - j0, o);
           } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j) o[j] = 0u;
           }
-        } else {
-          const int j0 = (ks - main_steps) * 64;
-          if (!B_MN) {  // fwd: B2 = lora B [N, r], row n0 + d, cols j0..j0+63
-            const int64_t n = n0 + d;
-            if (n < args.w_rows) {
-              load_row128(args.lora_b2 + n * args.lora_ld + j0, args.lora_r - j0, o);
-            } else {
+        } else {      // dX: B2 = lora A [r, K], row j0 + wr, cols n0 + 64*fb ..
+          const int jr = j0 + wr;
+          const int64_t kf = n0 + 64 * fb;
+          if (jr < args.lora_r && kf < args.w_cols) {
+            load_row128(args.lora_b2 + (int64_t)jr * args.lora_ld + kf, 64, o);
+          } else {
 #pragma unroll
-              for (int j = 0; j < 32; ++j) o[j] = 0u;
-            }
-          } else {      // bwd: B2 = lora A [r, K], row j0 + d/4, cols n0 + 64*(d%4) ..
-            const int jr = j0 + (d >> 2);
-            const int64_t kf = n0 + 64 * (d & 3);
-            if (jr < args.lora_r && kf < args.w_cols) {
-              load_row128(args.lora_b2 + (int64_t)jr * args.lora_ld + kf, 64, o);
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) o[j] = 0u;
-            }
+            for (int j = 0; j < 32; ++j) o[j] = 0u;
           }
         }
-        q_cur = q_nxt; c_cur = c_nxt;
-        q_nxt = q_pf; c_nxt = c_pf;
-        if (!ptx::mbar_wait(&empty_b[sb], pb ^ 1, abort_flag)) { ok = false; break; }
-        store_row128(sB + sb * C::B_STAGE + atom_off, row_in, o);
-        // Each thread orders its own writes before the tensor core's reads and
-        // arrives itself (one arrival per thread).
-        ptx::fence_proxy_async_smem();
-        ptx::mbar_arrive(&full_b[sb]);
-        if (++sb == C::SB) { sb = 0; pb ^= 1; }
       }
+      // refill this slot with the scale of the step two ahead
+      scale_src(ptile, pks, qs, cs);
+      advance(ptile, pks);
+      if (!ptx::mbar_wait(&empty_b[sb], pb ^ 1, abort_flag)) return false;
+      store_row128(sB + sb * C::B_STAGE + atom_off, row_in, o);
+      // Each thread orders its own writes before the tensor core's reads and
+      // arrives itself (one arrival per thread).
+      ptx::fence_proxy_async_smem();
+      ptx::mbar_arrive(&full_b[sb]);
+      if (++sb == C::SB) { sb = 0; pb ^= 1; }
+      advance(tile, ks);
+      return true;
+    };
+    while (ok && tile < num_tiles) {
+      ok = produce(qa, ca);
+      if (!ok || tile >= num_tiles) break;
+      ok = produce(qb, cb);
     }
     if (!ok && lane == 0) fail();
   }

@@ -162,7 +162,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_lora_kernel(const Ge
 
     // Software pipeline over this CTA's row groups: codes and scale bytes of the
     // next PD groups are in flight while the current one is decoded.
-    constexpr int PD = 1;
     struct Stage {
       uint2 c[4][2];   // [block][row half] 8 code bytes
       uint32_t q[2];   // 4 E4M3 scale bytes per row half (blocks kb0..kb0+3)
@@ -197,13 +196,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_lora_kernel(const Ge
         st.c2[h][1] = (rv && left < 4u && left < static_cast<uint32_t>(nblk)) ? __ldg(a.c2 + (b0 >> 8) + 1) : st.c2[h][0];
       }
     };
-    Stage stg[PD + 1];
-#pragma unroll
-    for (int p = 0; p < PD; ++p)
-      if (p < my_rg) load_stage(p, stg[p]);
-    for (int i = 0; i < my_rg; ++i) {
-      Stage &cur = stg[0];
-      if (i + PD < my_rg) load_stage(i + PD, stg[PD]);
+    // Two stages filled alternately: a stage is refilled only after it has been
+    // consumed, so no register holding an in-flight load is ever copied.
+    auto process = [&](int i, const Stage &cur) {
       // block scales of rows g (h=0) and g+8 (h=1)
       float S[2][4];
 #pragma unroll
@@ -258,8 +253,15 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_lora_kernel(const Ge
         rb[(g + 8) * 16 + t] += part[ng][2] * unscale[ng][0];
         rb[(g + 8) * 16 + t + 1] += part[ng][3] * unscale[ng][1];
       }
-#pragma unroll
-      for (int p = 0; p < PD; ++p) stg[p] = stg[p + 1];
+    };
+    Stage sa, sb;
+    if (my_rg > 0) load_stage(0, sa);
+    for (int i = 0; i < my_rg; i += 2) {
+      if (i + 1 < my_rg) load_stage(i + 1, sb);
+      process(i, sa);
+      if (i + 1 >= my_rg) break;
+      if (i + 2 < my_rg) load_stage(i + 2, sa);
+      process(i + 1, sb);
     }
   }
 
@@ -319,52 +321,61 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_lora_kernel(const Ge
   }
 }
 
-// T = X A^T for M <= 16 tokens: one CTA per LoRA rank row j; the CTA's threads
-// stride over K, then reduce.  Writes s*T (bf16) and optionally T (bf16).
-__global__ void __launch_bounds__(256) lora_down_small_kernel(const __nv_bfloat16 *__restrict__ X,
-                                                              const __nv_bfloat16 *__restrict__ A, int M,
-                                                              int64_t K, int r, float s,
-                                                              __nv_bfloat16 *__restrict__ sT,
-                                                              __nv_bfloat16 *__restrict__ T_hi,
-                                                              __nv_bfloat16 *__restrict__ T_lo) {
+// T = X A^T for M <= 16 tokens: one CTA of 128 threads per LoRA rank row j.
+// Thread i covers k in {8i + 1024 u}; loads of two iterations are in flight
+// together; partial sums are reduced over the M live tokens only.  Writes s*T
+// (bf16) and, if T_hi is given, the bf16 pair (T_hi, T_lo).
+constexpr int kLoraDownThreads = 128;
+__global__ void __launch_bounds__(kLoraDownThreads) lora_down_small_kernel(
+    const __nv_bfloat16 *__restrict__ X, const __nv_bfloat16 *__restrict__ A, int M, int64_t K, int r, float s,
+    __nv_bfloat16 *__restrict__ sT, __nv_bfloat16 *__restrict__ T_hi, __nv_bfloat16 *__restrict__ T_lo) {
   griddep_launch_dependents();
-  __shared__ float red[8][kGemvMaxM];
+  __shared__ float red[kLoraDownThreads / 32][kGemvMaxM];
   const int j = blockIdx.x;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   float acc[kGemvMaxM];
 #pragma unroll
   for (int t = 0; t < kGemvMaxM; ++t) acc[t] = 0.0f;
-  for (int64_t k = (int64_t)tid * 8; k < K; k += 256 * 8) {
-    const uint4 av = __ldg(reinterpret_cast<const uint4 *>(A + (int64_t)j * K + k));
-    const float af[8] = {bf16lo_to_f32(av.x), bf16hi_to_f32(av.x), bf16lo_to_f32(av.y), bf16hi_to_f32(av.y),
-                         bf16lo_to_f32(av.z), bf16hi_to_f32(av.z), bf16lo_to_f32(av.w), bf16hi_to_f32(av.w)};
+  const __nv_bfloat16 *Aj = A + (int64_t)j * K;
+  auto fma8 = [&](const uint4 &av, const uint4 &xv, float &a) {
+    a = fmaf(bf16lo_to_f32(av.x), bf16lo_to_f32(xv.x), a);
+    a = fmaf(bf16hi_to_f32(av.x), bf16hi_to_f32(xv.x), a);
+    a = fmaf(bf16lo_to_f32(av.y), bf16lo_to_f32(xv.y), a);
+    a = fmaf(bf16hi_to_f32(av.y), bf16hi_to_f32(xv.y), a);
+    a = fmaf(bf16lo_to_f32(av.z), bf16lo_to_f32(xv.z), a);
+    a = fmaf(bf16hi_to_f32(av.z), bf16hi_to_f32(xv.z), a);
+    a = fmaf(bf16lo_to_f32(av.w), bf16lo_to_f32(xv.w), a);
+    a = fmaf(bf16hi_to_f32(av.w), bf16hi_to_f32(xv.w), a);
+  };
+  for (int64_t k = (int64_t)tid * 8; k < K; k += 2 * kLoraDownThreads * 8) {
+    const int64_t k2 = k + kLoraDownThreads * 8;
+    const bool two = k2 < K;
+    const uint4 a0 = __ldg(reinterpret_cast<const uint4 *>(Aj + k));
+    const uint4 a1 = two ? __ldg(reinterpret_cast<const uint4 *>(Aj + k2)) : make_uint4(0, 0, 0, 0);
 #pragma unroll
     for (int t = 0; t < kGemvMaxM; ++t) {
       if (t < M) {
-        const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(X + (int64_t)t * K + k));
-        acc[t] = fmaf(af[0], bf16lo_to_f32(xv.x), acc[t]);
-        acc[t] = fmaf(af[1], bf16hi_to_f32(xv.x), acc[t]);
-        acc[t] = fmaf(af[2], bf16lo_to_f32(xv.y), acc[t]);
-        acc[t] = fmaf(af[3], bf16hi_to_f32(xv.y), acc[t]);
-        acc[t] = fmaf(af[4], bf16lo_to_f32(xv.z), acc[t]);
-        acc[t] = fmaf(af[5], bf16hi_to_f32(xv.z), acc[t]);
-        acc[t] = fmaf(af[6], bf16lo_to_f32(xv.w), acc[t]);
-        acc[t] = fmaf(af[7], bf16hi_to_f32(xv.w), acc[t]);
+        const uint4 x0 = __ldg(reinterpret_cast<const uint4 *>(X + (int64_t)t * K + k));
+        const uint4 x1 = two ? __ldg(reinterpret_cast<const uint4 *>(X + (int64_t)t * K + k2)) : make_uint4(0, 0, 0, 0);
+        fma8(a0, x0, acc[t]);
+        fma8(a1, x1, acc[t]);
       }
     }
   }
 #pragma unroll
   for (int t = 0; t < kGemvMaxM; ++t) {
-    float v = acc[t];
+    if (t < M) {
+      float v = acc[t];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if ((tid & 31) == 0) red[tid >> 5][t] = v;
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0) red[warp][t] = v;
+    }
   }
   __syncthreads();
   if (tid < M) {
     float v = 0.0f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) v += red[w][tid];
+    for (int w = 0; w < kLoraDownThreads / 32; ++w) v += red[w][tid];
     sT[(int64_t)tid * r + j] = __float2bfloat16_rn(v * s);
     if (T_hi) {
       const __nv_bfloat16 h = __float2bfloat16_rn(v);
