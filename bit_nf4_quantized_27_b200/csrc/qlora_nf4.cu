@@ -401,6 +401,50 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
   return QLORA_OK;
 }
 
+}  // extern "C"
+
+// Scratch of qlora_linear_fwd_noalloc: one static device array per GPU that
+// loads the library.  Host code must not pass `g_noalloc_scratch` itself to a
+// kernel (on the host it only names the symbol); its device address is looked up
+// once per device with cudaGetSymbolAddress.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[QLORA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+qlora_status noalloc_scratch(int dev, void **out) {
+  static std::once_flag flags[64];
+  static void *addr[64];
+  static cudaError_t err[64];
+  std::call_once(flags[dev], [&] {
+    void *p = nullptr;
+    err[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    addr[dev] = p;
+    cudaGetLastError();
+  });
+  if (err[dev] != cudaSuccess || !addr[dev]) return QLORA_ERR_CUDA;
+  *out = addr[dev];
+  return QLORA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+qlora_status qlora_linear_fwd_noalloc(const qlora_nf4_tensor *W, const qlora_lora *adapter, const void *X,
+                                      int64_t M, void *Y, qlora_dtype y_dtype, void *T_save,
+                                      qlora_stream_t stream) {
+  qlora_status s = check_nf4(W);
+  if (s != QLORA_OK) return s;
+  if ((s = check_lora(adapter)) != QLORA_OK) return s;
+  if (M < 1) return QLORA_ERR_INVALID_ARGUMENT;
+  const size_t need = qlora_workspace_bytes(M, W->rows, W->cols, adapter->r, 0);
+  if (need == 0) return QLORA_ERR_INVALID_ARGUMENT;
+  if (need > QLORA_NOALLOC_SCRATCH_BYTES) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  int dev, sms;
+  if ((s = check_device(&dev, &sms)) != QLORA_OK) return s;
+  void *scratch = nullptr;
+  if ((s = noalloc_scratch(dev, &scratch)) != QLORA_OK) return s;
+  return qlora_linear_fwd(W, adapter, X, M, Y, y_dtype, T_save, scratch, QLORA_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 qlora_status qlora_clear_status(void *ws, qlora_stream_t stream) {
   if (!ws) return QLORA_ERR_INVALID_ARGUMENT;
   return cudaMemsetAsync(ws, 0, sizeof(uint32_t), reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess

@@ -160,6 +160,28 @@ QLORA_API qlora_status qlora_linear_bwd(const qlora_nf4_tensor *W, const qlora_l
                               qlora_dtype dx_dtype, void *dA, void *dB, qlora_dtype grad_dtype,
                               void *ws, size_t ws_bytes, qlora_stream_t stream);
 
+/* Forward of the frozen linear layer with LoRA for callers that cannot allocate
+ * device memory when they call in: same inputs, outputs and results as
+ * qlora_linear_fwd, but with no workspace argument.  Examples are a plugin run
+ * from another runtime's launch callback, where cudaMalloc is not allowed
+ * because it synchronises the device and breaks the host's memory plan, or a
+ * serving loop whose device memory budget is fixed up front.
+ * This entry point has no counterpart on the QLoRA pages; it is a deployment
+ * convenience.  Its scratch (status word and the s*T buffer) is one static
+ * device array of QLORA_NOALLOC_SCRATCH_BYTES that the library holds on every
+ * GPU that loads it until the process exits.  Sizes whose workspace
+ * (qlora_workspace_bytes(M, N, K, r, 0)) exceeds it return
+ * QLORA_ERR_UNSUPPORTED_SHAPE and launch nothing.
+ * The first call on a device looks up the array's device address (with that
+ * device current); make that first call before any stream capture.  Every call
+ * on a device shares the one array and the contents left by the last call: calls
+ * that overlap on the GPU (different streams, or other threads) race on it, so
+ * serialise them.  Device-side status of these calls is not readable. */
+#define QLORA_NOALLOC_SCRATCH_BYTES (256u + 2u * 1024u * 1024u)
+QLORA_API qlora_status qlora_linear_fwd_noalloc(const qlora_nf4_tensor *W, const qlora_lora *adapter,
+                                                const void *X, int64_t M, void *Y, qlora_dtype y_dtype,
+                                                void *T_save, qlora_stream_t stream);
+
 /* Zero the status word at the start of ws (enqueued on stream). */
 QLORA_API qlora_status qlora_clear_status(void *ws, qlora_stream_t stream);
 
