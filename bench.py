@@ -256,9 +256,41 @@ def launches_per_step(nlayers):
     return nlayers * 7
 
 
+def graph_time_us(calls, reps=5):
+    """Captures `calls()` (a sequence of enqueues) into a CUDA graph and returns
+    the device time of one replay in microseconds (CUDA events, median of reps).
+    Graph replay removes the host enqueue cost, which exceeds the kernel time of
+    a microsecond-scale call."""
+    import torch
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        calls()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        calls()
+    g.replay()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        s, e = cuda_timer()
+        s.record()
+        g.replay()
+        e.record()
+        torch.cuda.synchronize()
+        times.append(s.elapsed_time(e) * 1e3)
+    del g
+    return statistics.median(times)
+
+
 def sub_gemv(device, peaks):
     """Decode-shaped forward (W 11008x4096, M in {1,4,16}, r=64): GB/s over the
-    NF4 codes + scales + activations, weights rotated over copies larger than L2."""
+    NF4 codes + scales + activations.  64 calls per CUDA graph, rotating over 8
+    weight copies (186 MB, larger than L2), so every call reads its weights from
+    HBM."""
     import torch
 
     from bit_nf4_quantized_27_b200 import binding as bd
@@ -282,32 +314,25 @@ def sub_gemv(device, peaks):
         y = torch.empty(m, n, dtype=torch.bfloat16, device=device)
         t = torch.empty(2, m, r, dtype=torch.bfloat16, device=device)
         ws = bd.new_workspace(bd.workspace_bytes(m, n, k, r, False), device)
-        reps = 16 * copies
+        reps = 8 * copies
 
-        def run():
+        def calls():
             for i in range(reps):
                 bd.linear_fwd(qs[i % copies], a, b, wl.alpha, x, ws=ws, out=y, t_out=t)
 
-        for _ in range(3):
-            run()
-        torch.cuda.synchronize()
-        s, e = cuda_timer()
-        s.record()
-        run()
-        e.record()
-        torch.cuda.synchronize()
-        us = s.elapsed_time(e) * 1e3 / reps
+        us = graph_time_us(calls) / reps
         nf4 = n * k // 2 + n * k // 64 + 4 * ((n * k // 64 + 255) // 256)
         act = m * k * 2 + m * n * 2
         gbs = (nf4 + act) / (us * 1e-6) / 1e9
         out[f"m{m}"] = {"us_per_call": us, "GB/s": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
                         "GB/s_incl_adapters": (nf4 + act + (r * k + n * r) * 2) / (us * 1e-6) / 1e9,
-                        "launches_per_call": 2}
+                        "launches_per_call": 2, "timing": "CUDA graph of 64 calls, 8 weight copies"}
     return out
 
 
 def sub_quant(device, peaks):
-    """Quantise / dequantise sweep (4096x4096 and 11008x4096 bf16): GB/s."""
+    """Quantise / dequantise sweep (4096x4096 and 11008x4096 bf16): GB/s, timed as
+    CUDA-graph replays over weight copies larger than L2 in total."""
     import torch
 
     from bit_nf4_quantized_27_b200 import binding as bd
@@ -319,20 +344,14 @@ def sub_quant(device, peaks):
         qs = [bd.NF4Weight(n, k, device) for _ in range(copies)]
         outs = [torch.empty(n, k, dtype=torch.bfloat16, device=device) for _ in range(copies)]
         st = bd.new_workspace(256, device)
-        reps = 8 * copies
+        reps = 4 * copies
         nbytes = n * k * 2 + n * k // 2 + n * k // 64 + 4 * ((n * k // 64 + 255) // 256)
         for name, fn in (("quantize", lambda i: bd.quantize(ws_[i % copies], out=qs[i % copies], ws=st)),
                          ("dequantize", lambda i: bd.dequantize(qs[i % copies], out=outs[i % copies]))):
             for i in range(copies):
                 fn(i)
             torch.cuda.synchronize()
-            s, e = cuda_timer()
-            s.record()
-            for i in range(reps):
-                fn(i)
-            e.record()
-            torch.cuda.synchronize()
-            us = s.elapsed_time(e) * 1e3 / reps
+            us = graph_time_us(lambda: [fn(i) for i in range(reps)]) / reps
             gbs = nbytes / (us * 1e-6) / 1e9
             res[f"{name}_{n}x{k}"] = {"us": us, "GB/s": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"]}
         del ws_, qs, outs

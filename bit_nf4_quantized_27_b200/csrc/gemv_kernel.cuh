@@ -24,6 +24,7 @@
 #pragma once
 
 #include "nf4_device.cuh"
+#include "sm100_ptx.cuh"
 
 namespace qlora {
 
@@ -321,89 +322,387 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_lora_kernel(const Ge
   }
 }
 
-// T = X A^T for M <= 16 tokens: one CTA of 128 threads per LoRA rank row j.
-// Thread i covers k in {8i + 1024 u}; loads of two iterations are in flight
-// together; partial sums are reduced over the M live tokens only.  Writes s*T
-// (bf16) and, if T_hi is given, the bf16 pair (T_hi, T_lo).
-constexpr int kLoraDownThreads = 128;
+// ---------------------------------------------------------------------------
+// Bulk-staged variant: each 16-row group's codes (16 x CH/2 contiguous bytes)
+// and block scales (16 x CH/64 bytes) arrive in shared memory through
+// cp.async.bulk into a 3-stage ring, so DRAM sees long contiguous reads and
+// about 100 KB stays in flight per SM without holding registers.  Requirements:
+// N % 16 == 0, K % 256 == 0 and (K <= 4096 or K % 4096 == 0); CH = min(K, 4096).
+// ---------------------------------------------------------------------------
+constexpr int kBulkStages = 3;
+constexpr int kBulkMaxRG = 5;
+
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+      "l"(src), "r"(bytes), "r"(static_cast<uint32_t>(__cvta_generic_to_shared(bar)))
+      : "memory");
+}
+
+inline bool gemv_bulk_ok(int64_t N, int64_t K) {
+  return N % 16 == 0 && K % 256 == 0 && (K <= 4096 || K % 4096 == 0);
+}
+
+template <int NG>
+__global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_bulk_kernel(const GemvArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  const int64_t CH = a.K < 4096 ? a.K : 4096;
+  const uint32_t stage_bytes = static_cast<uint32_t>(16 * CH / 2 + 16 * CH / 64);
+  uint32_t *lut = reinterpret_cast<uint32_t *>(smem_raw);
+  float *red = reinterpret_cast<float *>(smem_raw + 256 * 32 * 4);
+  uint8_t *ring = smem_raw + 256 * 32 * 4 + kBulkMaxRG * kGemvWarps * 256 * 4;
+  uint64_t *full = reinterpret_cast<uint64_t *>(ring + kBulkStages * stage_bytes);
+  uint64_t *empty = full + kBulkStages;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, q = lane & 3;
+
+  const int num_rg = static_cast<int>(a.N / 16);
+  const int rg0 = blockIdx.x * a.rg_per_cta;
+  const int my_rg = max(0, min(a.rg_per_cta, num_rg - rg0));
+  const int64_t nbk = a.K / 64;
+  const int nch = static_cast<int>(a.K / CH);
+  const int total = my_rg * nch;
+
+  // producer (thread 0): stage u = (chunk u / my_rg, row group u % my_rg)
+  auto issue = [&](int u) {
+    const int ch = u / my_rg, i = u % my_rg;
+    const int slot = u % kBulkStages;
+    uint8_t *st = ring + slot * stage_bytes;
+    const int64_t n0 = (int64_t)(rg0 + i) * 16;
+    ptx::mbar_arrive_expect_tx(&full[slot], stage_bytes);
+    if (CH == a.K) {
+      bulk_g2s(st, a.codes + n0 * (a.K / 2), static_cast<uint32_t>(16 * a.K / 2), &full[slot]);
+      bulk_g2s(st + 16 * CH / 2, a.scale_codes + n0 * nbk, static_cast<uint32_t>(16 * nbk), &full[slot]);
+    } else {
+      for (int rw = 0; rw < 16; ++rw) {
+        bulk_g2s(st + rw * (CH / 2), a.codes + (n0 + rw) * (a.K / 2) + ch * (CH / 2), static_cast<uint32_t>(CH / 2),
+                 &full[slot]);
+        bulk_g2s(st + 16 * CH / 2 + rw * (CH / 64), a.scale_codes + (n0 + rw) * nbk + ch * (CH / 64),
+                 static_cast<uint32_t>(CH / 64), &full[slot]);
+      }
+    }
+  };
+  if (tid == 0) {
+    for (int i = 0; i < kBulkStages; ++i) {
+      ptx::mbar_init(&full[i], 1);
+      ptx::mbar_init(&empty[i], kGemvThreads);
+    }
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0)
+    for (int u = 0; u < kBulkStages && u < total; ++u) issue(u);
+
+  for (int i = tid; i < 256 * 32; i += kGemvThreads) {
+    const int v = i >> 5;
+    const __half2 h = __floats2half2_rn(__uint_as_float(kNf4LevelBits[v & 15]), __uint_as_float(kNf4LevelBits[v >> 4]));
+    lut[i] = *reinterpret_cast<const uint32_t *>(&h);
+  }
+  for (int i = tid; i < my_rg * kGemvWarps * 256; i += kGemvThreads) red[i] = 0.0f;
+  __syncthreads();
+  const uint32_t lut_lane = static_cast<uint32_t>(__cvta_generic_to_shared(lut)) + lane * 4;
+  bool ok = true;
+
+  // warps whose 256-wide slice lies past K (K < 4096) only keep the ring's
+  // barrier counts: they wait for each stage and release it.
+  const bool active = warp * 4 < CH / 64;
+  for (int ch = 0; ch < nch && ok; ++ch) {
+    const int64_t kb0 = (int64_t)ch * 64 + warp * 4;  // first block of this warp's quad (global)
+    uint32_t xf[4][4][NG][2];
+    float unscale[NG][2];
+#pragma unroll
+    for (int ng = 0; ng < NG; ++ng) {
+      const int t = g + 8 * ng;
+      uint4 raw[4][2];
+      uint32_t mx = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+        if (active && t < a.M) {
+          const uint4 *src = reinterpret_cast<const uint4 *>(a.X + (int64_t)t * a.K + (kb0 + j) * 64 + 16 * q);
+          v0 = __ldg(src);
+          v1 = __ldg(src + 1);
+        }
+        raw[j][0] = v0;
+        raw[j][1] = v1;
+        mx = __vmaxu2(mx, __vmaxu2(__vmaxu2(v0.x & 0x7fff7fffu, v0.y & 0x7fff7fffu),
+                                   __vmaxu2(v0.z & 0x7fff7fffu, v0.w & 0x7fff7fffu)));
+        mx = __vmaxu2(mx, __vmaxu2(__vmaxu2(v1.x & 0x7fff7fffu, v1.y & 0x7fff7fffu),
+                                   __vmaxu2(v1.z & 0x7fff7fffu, v1.w & 0x7fff7fffu)));
+      }
+      uint32_t m16 = max(mx & 0xffffu, mx >> 16);
+      m16 = max(m16, __shfl_xor_sync(0xffffffffu, m16, 1));
+      m16 = max(m16, __shfl_xor_sync(0xffffffffu, m16, 2));
+      const int E = m16 ? static_cast<int>((m16 >> 7) & 0xff) - 126 : 15;
+      const int e = max(-100, min(100, E - 15));
+      const float inv = pow2f(-e);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        xf[j][0][ng][0] = bf16x2_to_f16x2_scaled(raw[j][0].x, inv);
+        xf[j][0][ng][1] = bf16x2_to_f16x2_scaled(raw[j][0].y, inv);
+        xf[j][1][ng][0] = bf16x2_to_f16x2_scaled(raw[j][0].z, inv);
+        xf[j][1][ng][1] = bf16x2_to_f16x2_scaled(raw[j][0].w, inv);
+        xf[j][2][ng][0] = bf16x2_to_f16x2_scaled(raw[j][1].x, inv);
+        xf[j][2][ng][1] = bf16x2_to_f16x2_scaled(raw[j][1].y, inv);
+        xf[j][3][ng][0] = bf16x2_to_f16x2_scaled(raw[j][1].z, inv);
+        xf[j][3][ng][1] = bf16x2_to_f16x2_scaled(raw[j][1].w, inv);
+      }
+      unscale[ng][0] = pow2f(__shfl_sync(0xffffffffu, e, (2 * q) * 4));
+      unscale[ng][1] = pow2f(__shfl_sync(0xffffffffu, e, (2 * q + 1) * 4));
+    }
+
+    // c2 of this thread's two rows for row group i: one value per (row, quad)
+    auto c2_of = [&](int i, float (&c)[2]) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int64_t row = (int64_t)(rg0 + i) * 16 + g + 8 * h;
+        c[h] = active ? __ldg(a.c2 + ((row * nbk + kb0) >> 8)) : 0.0f;
+      }
+    };
+    auto process = [&](int i, const float (&c2v)[2]) -> bool {
+      const int u = ch * my_rg + i;
+      const int slot = u % kBulkStages;
+      if (!ptx::mbar_wait(&full[slot], (u / kBulkStages) & 1, nullptr)) return false;
+      const uint8_t *st = ring + slot * stage_bytes;
+      const int kl = warp * 4;  // quad's first block within the chunk
+      if (!active) {
+        ptx::mbar_arrive(&empty[slot]);
+        if (tid == 0 && u + kBulkStages < total) {
+          if (!ptx::mbar_wait(&empty[slot], (u / kBulkStages) & 1, nullptr)) return false;
+          issue(u + kBulkStages);
+        }
+        return true;
+      }
+      uint2 cw[4][2];
+      uint32_t qw[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int rw = g + 8 * h;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          cw[j][h] = *reinterpret_cast<const uint2 *>(st + rw * (CH / 2) + (kl + j) * 32 + 8 * q);
+        qw[h] = *reinterpret_cast<const uint32_t *>(st + 16 * CH / 2 + rw * (CH / 64) + kl);
+      }
+      // this thread has read everything it needs from the stage
+      ptx::mbar_arrive(&empty[slot]);
+      float S[2][4];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(qw[h] & 0xffffu), __NV_E4M3);
+        const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(qw[h] >> 16), __NV_E4M3);
+        const float2 f01 = __half22float2(__half2(lo)), f23 = __half22float2(__half2(hi));
+        S[h][0] = __fmul_rn(f01.x, c2v[h]);
+        S[h][1] = __fmul_rn(f01.y, c2v[h]);
+        S[h][2] = __fmul_rn(f23.x, c2v[h]);
+        S[h][3] = __fmul_rn(f23.y, c2v[h]);
+      }
+      float part[NG][4];
+#pragma unroll
+      for (int ng = 0; ng < NG; ++ng) part[ng][0] = part[ng][1] = part[ng][2] = part[ng][3] = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float acc[NG][4];
+#pragma unroll
+        for (int ng = 0; ng < NG; ++ng) acc[ng][0] = acc[ng][1] = acc[ng][2] = acc[ng][3] = 0.0f;
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          const uint32_t w0 = (s < 2) ? cw[j][0].x : cw[j][0].y;
+          const uint32_t w1 = (s < 2) ? cw[j][1].x : cw[j][1].y;
+          const uint32_t p0 = (2 * s) & 3, p1 = (2 * s + 1) & 3;
+          const uint32_t b00 = __byte_perm(w0, 0u, 0x4440u | p0), b01 = __byte_perm(w0, 0u, 0x4440u | p1);
+          const uint32_t b10 = __byte_perm(w1, 0u, 0x4440u | p0), b11 = __byte_perm(w1, 0u, 0x4440u | p1);
+          uint32_t a0, a1, a2, a3;
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a0) : "r"(lut_lane + (b00 << 7)));
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a1) : "r"(lut_lane + (b10 << 7)));
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a2) : "r"(lut_lane + (b01 << 7)));
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a3) : "r"(lut_lane + (b11 << 7)));
+#pragma unroll
+          for (int ng = 0; ng < NG; ++ng) mma_16816_f16(acc[ng], a0, a1, a2, a3, xf[j][s][ng][0], xf[j][s][ng][1]);
+        }
+#pragma unroll
+        for (int ng = 0; ng < NG; ++ng) {
+          part[ng][0] = fmaf(S[0][j], acc[ng][0], part[ng][0]);
+          part[ng][1] = fmaf(S[0][j], acc[ng][1], part[ng][1]);
+          part[ng][2] = fmaf(S[1][j], acc[ng][2], part[ng][2]);
+          part[ng][3] = fmaf(S[1][j], acc[ng][3], part[ng][3]);
+        }
+      }
+      float *rb = red + ((size_t)i * kGemvWarps + warp) * 256;
+#pragma unroll
+      for (int ng = 0; ng < NG; ++ng) {
+        const int t = 2 * q + 8 * ng;
+        rb[g * 16 + t] += part[ng][0] * unscale[ng][0];
+        rb[g * 16 + t + 1] += part[ng][1] * unscale[ng][1];
+        rb[(g + 8) * 16 + t] += part[ng][2] * unscale[ng][0];
+        rb[(g + 8) * 16 + t + 1] += part[ng][3] * unscale[ng][1];
+      }
+      // refill the slot once every thread has released it
+      if (tid == 0 && u + kBulkStages < total) {
+        if (!ptx::mbar_wait(&empty[slot], (u / kBulkStages) & 1, nullptr)) return false;
+        issue(u + kBulkStages);
+      }
+      return true;
+    };
+    float ca[2], cb[2];
+    if (my_rg > 0) c2_of(0, ca);
+    for (int i = 0; i < my_rg && ok; i += 2) {
+      if (i + 1 < my_rg) c2_of(i + 1, cb);
+      ok = process(i, ca);
+      if (!ok || i + 1 >= my_rg) break;
+      if (i + 2 < my_rg) c2_of(i + 2, ca);
+      ok = process(i + 1, cb);
+    }
+  }
+  if (!ok && lane == 0) raise_status(a.status, QLORA_ERR_TIMEOUT);
+
+  // LoRA up-projection (needs s T from the preceding kernel), then reduction.
+  griddep_wait();
+  for (int i = warp; i < my_rg; i += kGemvWarps) {
+    const int64_t n0 = (int64_t)(rg0 + i) * 16;
+    float acc[NG][4];
+#pragma unroll
+    for (int ng = 0; ng < NG; ++ng) acc[ng][0] = acc[ng][1] = acc[ng][2] = acc[ng][3] = 0.0f;
+    for (int j0 = 0; j0 < a.r; j0 += 16) {
+      uint32_t af[4];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int64_t row = n0 + g + 8 * h;
+        const uint32_t *src = reinterpret_cast<const uint32_t *>(a.B + row * a.r + j0 + 2 * q);
+        af[h] = (j0 + 2 * q < a.r) ? __ldg(src) : 0u;
+        af[2 + h] = (j0 + 8 + 2 * q < a.r) ? __ldg(src + 4) : 0u;
+      }
+#pragma unroll
+      for (int ng = 0; ng < NG; ++ng) {
+        const int t = g + 8 * ng;
+        uint32_t b0 = 0, b1 = 0;
+        if (t < a.M) {
+          const uint32_t *src = reinterpret_cast<const uint32_t *>(a.sT + (int64_t)t * a.r + j0 + 2 * q);
+          if (j0 + 2 * q < a.r) b0 = __ldg(src);
+          if (j0 + 8 + 2 * q < a.r) b1 = __ldg(src + 4);
+        }
+        mma_16816(acc[ng], af[0], af[1], af[2], af[3], b0, b1);
+      }
+    }
+    float *rb = red + ((size_t)i * kGemvWarps + warp) * 256;
+#pragma unroll
+    for (int ng = 0; ng < NG; ++ng) {
+      const int t = 2 * q + 8 * ng;
+      rb[g * 16 + t] += acc[ng][0];
+      rb[g * 16 + t + 1] += acc[ng][1];
+      rb[(g + 8) * 16 + t] += acc[ng][2];
+      rb[(g + 8) * 16 + t + 1] += acc[ng][3];
+    }
+  }
+  __syncthreads();
+  for (int idx = tid; idx < my_rg * 256; idx += kGemvThreads) {
+    const int i = idx >> 8, e = idx & 255, row = e >> 4, t = e & 15;
+    const int64_t n = (int64_t)(rg0 + i) * 16 + row;
+    if (t >= a.M) continue;
+    const float *rb = red + (size_t)i * kGemvWarps * 256 + e;
+    float sum = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kGemvWarps; ++w) sum += rb[w * 256];
+    if (a.y_f32) reinterpret_cast<float *>(a.Y)[(int64_t)t * a.N + n] = sum;
+    else reinterpret_cast<__nv_bfloat16 *>(a.Y)[(int64_t)t * a.N + n] = __float2bfloat16_rn(sum);
+  }
+}
+
+// T = X A^T for M <= 16 tokens on tensor cores, in few CTAs so that it runs on
+// SMs the decode GEMV leaves free.  CTA c computes rank rows [16c, 16c + 16):
+// 8 warps split K, each runs m16n8k16 MMAs with A = 16 rows of the LoRA A matrix
+// and B = X^T (tokens), both bf16; the partials are summed over the warps in a
+// fixed order.  Writes s*T (bf16) and, if T_hi is given, (T_hi, T_lo).
+constexpr int kLoraDownThreads = 256;
 __global__ void __launch_bounds__(kLoraDownThreads) lora_down_small_kernel(
     const __nv_bfloat16 *__restrict__ X, const __nv_bfloat16 *__restrict__ A, int M, int64_t K, int r, float s,
     __nv_bfloat16 *__restrict__ sT, __nv_bfloat16 *__restrict__ T_hi, __nv_bfloat16 *__restrict__ T_lo) {
   griddep_launch_dependents();
-  __shared__ float red[kLoraDownThreads / 32][kGemvMaxM];
-  const int j = blockIdx.x;
+  __shared__ float red[kLoraDownThreads / 32][16][kGemvMaxM];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  float acc[kGemvMaxM];
+  const int g = lane >> 2, q = lane & 3;
+  const int j0 = blockIdx.x * 16;
+  const int64_t nk16 = K / 16;
+  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  const int rows[2] = {j0 + g, j0 + g + 8};
+  for (int64_t kk = warp; kk < nk16; kk += kLoraDownThreads / 32) {
+    const int64_t k = kk * 16 + 2 * q;
+    uint32_t af[4];
 #pragma unroll
-  for (int t = 0; t < kGemvMaxM; ++t) acc[t] = 0.0f;
-  const __nv_bfloat16 *Aj = A + (int64_t)j * K;
-  auto fma8 = [&](const uint4 &av, const uint4 &xv, float &a) {
-    a = fmaf(bf16lo_to_f32(av.x), bf16lo_to_f32(xv.x), a);
-    a = fmaf(bf16hi_to_f32(av.x), bf16hi_to_f32(xv.x), a);
-    a = fmaf(bf16lo_to_f32(av.y), bf16lo_to_f32(xv.y), a);
-    a = fmaf(bf16hi_to_f32(av.y), bf16hi_to_f32(xv.y), a);
-    a = fmaf(bf16lo_to_f32(av.z), bf16lo_to_f32(xv.z), a);
-    a = fmaf(bf16hi_to_f32(av.z), bf16hi_to_f32(xv.z), a);
-    a = fmaf(bf16lo_to_f32(av.w), bf16lo_to_f32(xv.w), a);
-    a = fmaf(bf16hi_to_f32(av.w), bf16hi_to_f32(xv.w), a);
-  };
-  for (int64_t k = (int64_t)tid * 8; k < K; k += 2 * kLoraDownThreads * 8) {
-    const int64_t k2 = k + kLoraDownThreads * 8;
-    const bool two = k2 < K;
-    const uint4 a0 = __ldg(reinterpret_cast<const uint4 *>(Aj + k));
-    const uint4 a1 = two ? __ldg(reinterpret_cast<const uint4 *>(Aj + k2)) : make_uint4(0, 0, 0, 0);
+    for (int h = 0; h < 2; ++h) {
+      const bool rv = rows[h] < r;
+      const uint32_t *src = reinterpret_cast<const uint32_t *>(A + (int64_t)rows[h] * K + k);
+      af[h] = rv ? __ldg(src) : 0u;
+      af[2 + h] = rv ? __ldg(src + 4) : 0u;
+    }
 #pragma unroll
-    for (int t = 0; t < kGemvMaxM; ++t) {
+    for (int ng = 0; ng < 2; ++ng) {
+      const int t = g + 8 * ng;
+      if (ng * 8 >= M) break;
+      uint32_t b0 = 0, b1 = 0;
       if (t < M) {
-        const uint4 x0 = __ldg(reinterpret_cast<const uint4 *>(X + (int64_t)t * K + k));
-        const uint4 x1 = two ? __ldg(reinterpret_cast<const uint4 *>(X + (int64_t)t * K + k2)) : make_uint4(0, 0, 0, 0);
-        fma8(a0, x0, acc[t]);
-        fma8(a1, x1, acc[t]);
+        const uint32_t *src = reinterpret_cast<const uint32_t *>(X + (int64_t)t * K + k);
+        b0 = __ldg(src);
+        b1 = __ldg(src + 4);
       }
+      mma_16816(acc[ng], af[0], af[1], af[2], af[3], b0, b1);
     }
   }
+  // C fragment: rows g / g+8 (rank), columns 2q, 2q+1 (+8 ng) (tokens)
 #pragma unroll
-  for (int t = 0; t < kGemvMaxM; ++t) {
-    if (t < M) {
-      float v = acc[t];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0) red[warp][t] = v;
-    }
+  for (int ng = 0; ng < 2; ++ng) {
+    const int t = 2 * q + 8 * ng;
+    red[warp][g][t] = acc[ng][0];
+    red[warp][g][t + 1] = acc[ng][1];
+    red[warp][g + 8][t] = acc[ng][2];
+    red[warp][g + 8][t + 1] = acc[ng][3];
   }
   __syncthreads();
-  if (tid < M) {
+  // one output per thread: rank row tid / 16, token tid % 16
+  const int jr = tid >> 4, t = tid & 15;
+  if (t < M && j0 + jr < r) {
     float v = 0.0f;
 #pragma unroll
-    for (int w = 0; w < kLoraDownThreads / 32; ++w) v += red[w][tid];
-    sT[(int64_t)tid * r + j] = __float2bfloat16_rn(v * s);
+    for (int w = 0; w < kLoraDownThreads / 32; ++w) v += red[w][jr][t];
+    const int64_t o = (int64_t)t * r + j0 + jr;
+    sT[o] = __float2bfloat16_rn(v * s);
     if (T_hi) {
       const __nv_bfloat16 h = __float2bfloat16_rn(v);
-      T_hi[(int64_t)tid * r + j] = h;
-      T_lo[(int64_t)tid * r + j] = __float2bfloat16_rn(v - __bfloat162float(h));
+      T_hi[o] = h;
+      T_lo[o] = __float2bfloat16_rn(v - __bfloat162float(h));
     }
   }
 }
 
 inline qlora_status launch_gemv(GemvArgs g, int dev, int sms, cudaStream_t st) {
   const int num_rg = static_cast<int>((g.N + 15) / 16);
+  const bool bulk = gemv_bulk_ok(g.N, g.K);
+  const int cap = bulk ? kBulkMaxRG : kGemvMaxRG;
   int per = (num_rg + sms - 1) / sms;
-  if (per > kGemvMaxRG) per = kGemvMaxRG;
+  if (per > cap) per = cap;
   g.rg_per_cta = per;
   const int grid = (num_rg + per - 1) / per;
-  const int smem = 256 * 32 * 4 + per * kGemvWarps * 256 * 4;
-  static std::once_flag flags[2][64];
-  static qlora_status results[2][64];
+  const int64_t CH = g.K < 4096 ? g.K : 4096;
+  const int bulk_smem = 256 * 32 * 4 + kBulkMaxRG * kGemvWarps * 256 * 4 +
+                        kBulkStages * static_cast<int>(16 * CH / 2 + 16 * CH / 64) + 2 * kBulkStages * 8;
+  const int smem = bulk ? bulk_smem : 256 * 32 * 4 + per * kGemvWarps * 256 * 4;
+  static std::once_flag flags[4][64];
+  static qlora_status results[4][64];
   const bool two = g.M > 8;
-  auto kernel = two ? nf4_gemv_lora_kernel<2> : nf4_gemv_lora_kernel<1>;
-  std::call_once(flags[two][dev], [&] {
-    results[two][dev] = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             256 * 32 * 4 + kGemvMaxRG * kGemvWarps * 256 * 4) == cudaSuccess
-                            ? QLORA_OK
-                            : QLORA_ERR_CUDA;
+  const int which = (bulk ? 2 : 0) + (two ? 1 : 0);
+  auto kernel = bulk ? (two ? nf4_gemv_bulk_kernel<2> : nf4_gemv_bulk_kernel<1>)
+                     : (two ? nf4_gemv_lora_kernel<2> : nf4_gemv_lora_kernel<1>);
+  std::call_once(flags[which][dev], [&] {
+    const int max_smem = bulk ? 256 * 32 * 4 + kBulkMaxRG * kGemvWarps * 256 * 4 +
+                                    kBulkStages * (16 * 4096 / 2 + 16 * 4096 / 64) + 2 * kBulkStages * 8
+                              : 256 * 32 * 4 + kGemvMaxRG * kGemvWarps * 256 * 4;
+    results[which][dev] = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) ==
+                                  cudaSuccess
+                              ? QLORA_OK
+                              : QLORA_ERR_CUDA;
     cudaGetLastError();
   });
-  if (results[two][dev] != QLORA_OK) return results[two][dev];
+  if (results[which][dev] != QLORA_OK) return results[which][dev];
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kGemvThreads);

@@ -236,7 +236,7 @@ qlora_status qlora_linear_fwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
 
   if (M <= kGemvMaxM) {
     __nv_bfloat16 *th = static_cast<__nv_bfloat16 *>(T_save);
-    lora_down_small_kernel<<<ad->r, kLoraDownThreads, 0, st>>>(static_cast<const __nv_bfloat16 *>(X),
+    lora_down_small_kernel<<<(ad->r + 15) / 16, kLoraDownThreads, 0, st>>>(static_cast<const __nv_bfloat16 *>(X),
                                                   static_cast<const __nv_bfloat16 *>(ad->A), (int)M, K, ad->r, sc,
                                                   static_cast<__nv_bfloat16 *>(sT), th, th ? th + M * ad->r : nullptr);
     if ((s = launch_status()) != QLORA_OK) return s;
