@@ -183,6 +183,7 @@ def build_block(wl, device, rank, gen_seed_offset=0):
     import torch
 
     from bit_nf4_quantized_27_b200 import binding as bd
+    from bit_nf4_quantized_27_b200 import dp
     from bit_nf4_quantized_27_b200 import inputs as I
 
     def dnormal(shape, std, seed):
@@ -207,14 +208,10 @@ def build_block(wl, device, rank, gen_seed_offset=0):
         d["ws_b"] = bd.new_workspace(bd.workspace_bytes(m, ly.n, ly.k, r, True), device)
         layers.append(d)
     # one flat fp32 buffer holds every layer's dA and dB (one all-reduce per step)
-    total = sum(r * d["k"] + d["n"] * r for d in layers)
-    flat = torch.zeros(total, dtype=torch.float32, device=device)
-    off = 0
-    for d in layers:
-        d["da"] = flat[off:off + r * d["k"]].view(r, d["k"])
-        off += r * d["k"]
-        d["db"] = flat[off:off + d["n"] * r].view(d["n"], r)
-        off += d["n"] * r
+    shapes = [(d["n"], d["k"]) for d in layers]
+    flat = torch.zeros(dp.flat_size(shapes, r), dtype=torch.float32, device=device)
+    for d, (da, db) in zip(layers, dp.grad_views(flat, shapes, r)):
+        d["da"], d["db"] = da, db
     return layers, flat
 
 
@@ -246,9 +243,9 @@ def run_step(layers, wl, flat, world, timing=None):
             e1.record()
             timing["bwd"].append((e0, e1))
     if world > 1:
-        import torch.distributed as dist
+        from bit_nf4_quantized_27_b200 import dp
 
-        dist.all_reduce(flat)
+        dp.allreduce_grads(flat)
 
 
 def launches_per_step(nlayers):
