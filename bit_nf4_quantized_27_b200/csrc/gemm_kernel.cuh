@@ -62,7 +62,7 @@ struct GemmCfg {
   static constexpr int B_STAGE = BN * BK * 2;
   static constexpr int C_STAGE = NF4 ? BN * 32 : 0;  // codes: 64 weights (32 B) per B row
   static constexpr int SA = NF4 ? (MT == 1 ? 4 : 3) : 6;
-  static constexpr int SB = NF4 ? (MT == 1 ? 3 : 2) : SA;
+  static constexpr int SB = NF4 ? 3 : SA;
   static constexpr int SC = NF4 ? 4 : 1;
   static constexpr int NUM_ACC = (2 * MT * BN <= 512) ? 2 : 1;
   static constexpr int ACC_COLS = MT * BN;
@@ -85,11 +85,10 @@ __device__ __forceinline__ uint32_t sw128_row_chunk(uint32_t row, uint32_t c) {
 // Decode 64 NF4 codes (two uint4 of packed nibbles) with block scale S into 32
 // packed bf16x2 words, via a per-block table of the 16 products split into byte
 // planes and looked up with byte permutes.
-__device__ __forceinline__ void nf4_decode64(const uint4 &c0, const uint4 &c1, float S, const float (&lv)[16],
-                                             uint32_t (&o)[32]) {
+__device__ __forceinline__ void nf4_decode64(const uint4 &c0, const uint4 &c1, float S, uint32_t (&o)[32]) {
   uint32_t p[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) p[j] = pack_bf16x2(__fmul_rn(lv[2 * j], S), __fmul_rn(lv[2 * j + 1], S));
+  for (int j = 0; j < 8; ++j) p[j] = pack_bf16x2(__fmul_rn(nf4_level(2 * j), S), __fmul_rn(nf4_level(2 * j + 1), S));
   // lo/hi byte planes of entries 0-3, 4-7, 8-11, 12-15
   uint32_t lo[4], hi[4];
 #pragma unroll
@@ -285,6 +284,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const int num_m = (args.M_rows + C::BM * MT - 1) / (C::BM * MT);
   const int num_n = (args.N_cols + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
+  auto tile_of = [&](int w, int &m0, int &n0) {
+    m0 = (w % num_m) * C::BM * MT;
+    n0 = (w / num_m) * BN;
+  };
   const int main_steps = args.k_steps * (args.hilo ? 2 : 1);
   const int steps = main_steps + args.lora_steps;
 
@@ -300,8 +303,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       int issued_a = 0, issued_c = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int m0 = (tile % num_m) * C::BM * MT;
-        const int n0 = (tile / num_m) * BN;
+        int m0, n0;
+        tile_of(tile, m0, n0);
         for (int ks = 0; ks < steps && ok; ++ks) {
           const bool lora = ks >= main_steps;
           const bool second = !lora && ks >= args.k_steps;  // hi/lo second pass
@@ -409,8 +412,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         break;
       }
       ptx::tc_fence_after();
-      const int m0 = (tile % num_m) * C::BM * MT;
-      const int n0 = (tile / num_m) * BN;
+      int m0, n0;
+      tile_of(tile, m0, n0);
       for (int t = 0; t < MT; ++t) {
         const int row = m0 + t * 128 + q * 32 + lane;
         for (int cb = 0; cb < BN; cb += 32) {
@@ -428,9 +431,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   } else if (NF4 && warp >= 8) {
     // ------------------------------------------------------------ dequant producer
     const int d = threadIdx.x - 256;  // 0..255
-    float lv[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) lv[j] = __uint_as_float(kNf4LevelBits[j]);
     const int64_t kblocks = args.w_cols / 64;
     // Thread -> (B row it fills, code bytes it reads).  Chosen so that, within
     // every quarter-warp, the eight 16-byte code reads and the eight swizzled
@@ -460,7 +460,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       qv = 0x100u;  // "no block": rows past N, LoRA steps, past the last tile
       cv = 0.0f;
       if (tile >= num_tiles || ks >= main_steps) return;
-      const int n0 = (tile / num_m) * BN;
+      int m0_, n0;
+      tile_of(tile, m0_, n0);
       int64_t wrow, kblk;
       if (!B_MN) { wrow = n0 + wr; kblk = ks; }
       else { wrow = (int64_t)ks * 64 + wr; kblk = n0 / 64 + fb; }
@@ -486,7 +487,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
     auto produce = [&](uint32_t &qs, float &cs) -> bool {
       const bool lora = ks >= main_steps;
-      const int n0 = (tile / num_m) * BN;
+      int m0_, n0;
+      tile_of(tile, m0_, n0);
       uint32_t o[32];
       if (!lora) {
         if (!ptx::mbar_wait(&full_c[sc], pc, abort_flag)) return false;
@@ -498,7 +500,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const uint4 c0 = half_first ? x1 : x0, c1 = half_first ? x0 : x1;
         if (qs != 0x100u) {
           const float S = __fmul_rn(e4m3_to_f32(static_cast<uint8_t>(qs)), cs);
-          nf4_decode64(c0, c1, S, lv, o);
+          nf4_decode64(c0, c1, S, o);
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j) o[j] = 0u;

@@ -22,6 +22,19 @@ __constant__ uint32_t kNf4LevelBits[16] = {
     0xbdba786bu, 0x00000000u, 0x3da2fb03u, 0x3e24cae1u, 0x3e7c04dcu, 0x3ead0338u,
     0x3ee1a4b7u, 0x3f1007aau, 0x3f3913b1u, 0x3f800000u};
 
+// The same 16 levels as compile-time float constants (identical bit patterns;
+// a CPU test checks the two lists against each other), so that kernels can use
+// them as instruction immediates instead of registers.  j must be a constant
+// after unrolling.
+__host__ __device__ constexpr float nf4_level(int j) {
+  return j == 0 ? -0x1.000000p+0f : j == 1 ? -0x1.647366p-1f : j == 2 ? -0x1.0cd660p-1f
+       : j == 3 ? -0x1.946540p-2f : j == 4 ? -0x1.234498p-2f : j == 5 ? -0x1.7a6a7ep-3f
+       : j == 6 ? -0x1.74f0d6p-4f : j == 7 ? 0x0.0p+0f : j == 8 ? 0x1.45f606p-4f
+       : j == 9 ? 0x1.4995c2p-3f : j == 10 ? 0x1.f809b8p-3f : j == 11 ? 0x1.5a0670p-2f
+       : j == 12 ? 0x1.c3496ep-2f : j == 13 ? 0x1.200f54p-1f : j == 14 ? 0x1.722762p-1f
+       : 0x1.000000p+0f;
+}
+
 // Device status word flags (bit k set <=> status code k was raised).
 __device__ __forceinline__ void raise_status(uint32_t *status, qlora_status code) {
   if (status) atomicOr(status, 1u << static_cast<uint32_t>(code));

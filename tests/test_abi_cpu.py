@@ -89,3 +89,22 @@ def test_status_strings(L):
     for code in range(9):
         assert L.qlora_status_string(code)
     assert L.qlora_status_string(0) == b"ok"
+
+
+def test_device_level_literals_match_bit_patterns():
+    # the kernels use the 16 levels both as float32 bit patterns and as hex-float
+    # immediates; both lists, and the oracle's table, must be identical
+    import os
+    import re
+    import struct
+
+    src = open(os.path.join(os.path.dirname(bd.LIB_PATH), "csrc", "nf4_device.cuh")).read()
+    bits_block = src[src.index("kNf4LevelBits[16] = {"):]
+    bits = [int(b, 16) for b in re.findall(r"0x([0-9a-f]{8})u", bits_block[:bits_block.index("};")])]
+    fn = src[src.index("constexpr float nf4_level(int j)"):]
+    fn = fn[:fn.index("}")]
+    lits = re.findall(r"(-?0x[0-9a-f.]+p[+-]\d+)f", fn)
+    vals = [struct.unpack("<I", struct.pack("<f", float.fromhex(v)))[0] for v in lits]
+    assert len(bits) == 16 and len(vals) == 16
+    assert bits == vals
+    assert bits == [int(x) for x in O.nf4_levels().view(np.uint32)]
