@@ -329,7 +329,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_lora_kernel(const Ge
 // about 100 KB stays in flight per SM without holding registers.  Requirements:
 // N % 16 == 0, K % 256 == 0 and (K <= 4096 or K % 4096 == 0); CH = min(K, 4096).
 // ---------------------------------------------------------------------------
-constexpr int kBulkStages = 3;
 constexpr int kBulkMaxRG = 5;
 
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
@@ -344,18 +343,88 @@ inline bool gemv_bulk_ok(int64_t N, int64_t K) {
   return N % 16 == 0 && K % 256 == 0 && (K <= 4096 || K % 4096 == 0);
 }
 
+// Shared memory of the bulk kernel.  The pair table sits at a 64 KB-aligned
+// shared address with a 256-byte row per byte value (a lane's entry at
+// row * 256 + lane * 4), so one byte permute builds the whole lookup address:
+// [lane * 4 | code byte | table base bits 16..31].  Row-group partial sums
+// (16 KB each), the stage ring and the barriers are placed before the table
+// where they fit and after it otherwise.
+constexpr uint32_t kBulkLutBytes = 256 * 256;
+constexpr uint32_t kBulkRedBytes = kGemvWarps * 256 * 4;
+constexpr int kBulkStagesV4 = 2;
+
+// Staged code rows are CH/2 + 32 bytes apart, so the 8 rows one warp reads in a
+// single instruction fall on 8 different 32-byte bank groups.
+__host__ __device__ inline uint32_t gemv_bulk_row_stride(int64_t K) {
+  const int64_t CH = K < 4096 ? K : 4096;
+  return static_cast<uint32_t>(CH / 2 + 32);
+}
+__host__ __device__ inline uint32_t gemv_bulk_stage_bytes(int64_t K) {
+  const int64_t CH = K < 4096 ? K : 4096;
+  return static_cast<uint32_t>((16 * gemv_bulk_row_stride(K) + 16 * CH / 64 + 127) & ~int64_t(127));
+}
+
+// Placement of the bulk kernel's buffers around the 64 KB-aligned table, for a
+// dynamic window starting at shared address `base`; returns the end address.
+struct BulkLayout {
+  uint32_t lut, red[kBulkMaxRG], stage[kBulkStagesV4], bar, end;
+};
+__host__ __device__ inline BulkLayout gemv_bulk_layout(uint32_t base, uint32_t stage_bytes) {
+  BulkLayout L;
+  L.lut = (base + 0xffffu) & ~0xffffu;
+  uint32_t lo_next = base, hi_next = L.lut + kBulkLutBytes;
+  auto place = [&](uint32_t bytes, uint32_t align) -> uint32_t {
+    const uint32_t lo = (lo_next + align - 1) & ~(align - 1);
+    if (lo + bytes <= L.lut) {
+      lo_next = lo + bytes;
+      return lo;
+    }
+    const uint32_t hi = (hi_next + align - 1) & ~(align - 1);
+    hi_next = hi + bytes;
+    return hi;
+  };
+  for (int i = 0; i < kBulkMaxRG; ++i) L.red[i] = place(kBulkRedBytes, 16);
+  for (int i = 0; i < kBulkStagesV4; ++i) L.stage[i] = place(stage_bytes, 128);
+  L.bar = place(64, 16);
+  L.end = hi_next > lo_next ? hi_next : lo_next;
+  return L;
+}
+
+// Dynamic shared memory that covers the layout for any window start (16-byte
+// steps within a 64 KB period).
+inline int gemv_bulk_smem_bytes(int64_t K) {
+  const uint32_t sb = gemv_bulk_stage_bytes(K);
+  uint32_t worst = 0;
+  for (uint32_t base = 0; base < 65536; base += 16) {
+    const BulkLayout L = gemv_bulk_layout(base, sb);
+    if (L.end - base > worst) worst = L.end - base;
+  }
+  return static_cast<int>(worst);
+}
+
 template <int NG>
-__global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_bulk_kernel(const GemvArgs a) {
-  extern __shared__ uint8_t smem_raw[];
+__global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_bulk_kernel(const GemvArgs a, int dyn_bytes) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
   const int64_t CH = a.K < 4096 ? a.K : 4096;
-  const uint32_t stage_bytes = static_cast<uint32_t>(16 * CH / 2 + 16 * CH / 64);
-  uint32_t *lut = reinterpret_cast<uint32_t *>(smem_raw);
-  float *red = reinterpret_cast<float *>(smem_raw + 256 * 32 * 4);
-  uint8_t *ring = smem_raw + 256 * 32 * 4 + kBulkMaxRG * kGemvWarps * 256 * 4;
-  uint64_t *full = reinterpret_cast<uint64_t *>(ring + kBulkStages * stage_bytes);
-  uint64_t *empty = full + kBulkStages;
+  const uint32_t stage_bytes = gemv_bulk_stage_bytes(a.K);
+  const uint32_t RS = gemv_bulk_row_stride(a.K);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, q = lane & 3;
+
+  // ---- layout around the 64 KB-aligned table
+  const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw));
+  const BulkLayout Lay = gemv_bulk_layout(base, stage_bytes);
+  const uint32_t lut_addr = Lay.lut;
+  const uint32_t *red_addr = Lay.red;
+  const uint32_t *stage_addr = Lay.stage;
+  const uint32_t bar_addr = Lay.bar;
+  if (Lay.end > base + static_cast<uint32_t>(dyn_bytes)) {  // cannot happen with the host's size
+    if (tid == 0) raise_status(a.status, QLORA_ERR_CUDA);
+    return;
+  }
+  auto at = [&](uint32_t addr) { return smem_raw + (addr - base); };
+  uint64_t *full = reinterpret_cast<uint64_t *>(at(bar_addr));
+  uint64_t *empty = full + kBulkStagesV4;
 
   const int num_rg = static_cast<int>(a.N / 16);
   const int rg0 = blockIdx.x * a.rg_per_cta;
@@ -367,24 +436,23 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_bulk_kernel(const Ge
   // producer (thread 0): stage u = (chunk u / my_rg, row group u % my_rg)
   auto issue = [&](int u) {
     const int ch = u / my_rg, i = u % my_rg;
-    const int slot = u % kBulkStages;
-    uint8_t *st = ring + slot * stage_bytes;
+    const int slot = u % kBulkStagesV4;
+    uint8_t *st = at(stage_addr[slot]);
     const int64_t n0 = (int64_t)(rg0 + i) * 16;
-    ptx::mbar_arrive_expect_tx(&full[slot], stage_bytes);
+    ptx::mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(16 * CH / 2 + 16 * CH / 64));
+    for (int rw = 0; rw < 16; ++rw)
+      bulk_g2s(st + rw * RS, a.codes + (n0 + rw) * (a.K / 2) + ch * (CH / 2), static_cast<uint32_t>(CH / 2),
+               &full[slot]);
     if (CH == a.K) {
-      bulk_g2s(st, a.codes + n0 * (a.K / 2), static_cast<uint32_t>(16 * a.K / 2), &full[slot]);
-      bulk_g2s(st + 16 * CH / 2, a.scale_codes + n0 * nbk, static_cast<uint32_t>(16 * nbk), &full[slot]);
+      bulk_g2s(st + 16 * RS, a.scale_codes + n0 * nbk, static_cast<uint32_t>(16 * nbk), &full[slot]);
     } else {
-      for (int rw = 0; rw < 16; ++rw) {
-        bulk_g2s(st + rw * (CH / 2), a.codes + (n0 + rw) * (a.K / 2) + ch * (CH / 2), static_cast<uint32_t>(CH / 2),
-                 &full[slot]);
-        bulk_g2s(st + 16 * CH / 2 + rw * (CH / 64), a.scale_codes + (n0 + rw) * nbk + ch * (CH / 64),
+      for (int rw = 0; rw < 16; ++rw)
+        bulk_g2s(st + 16 * RS + rw * (CH / 64), a.scale_codes + (n0 + rw) * nbk + ch * (CH / 64),
                  static_cast<uint32_t>(CH / 64), &full[slot]);
-      }
     }
   };
   if (tid == 0) {
-    for (int i = 0; i < kBulkStages; ++i) {
+    for (int i = 0; i < kBulkStagesV4; ++i) {
       ptx::mbar_init(&full[i], 1);
       ptx::mbar_init(&empty[i], kGemvThreads);
     }
@@ -392,21 +460,22 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_bulk_kernel(const Ge
   }
   __syncthreads();
   if (tid == 0)
-    for (int u = 0; u < kBulkStages && u < total; ++u) issue(u);
+    for (int u = 0; u < kBulkStagesV4 && u < total; ++u) issue(u);
 
+  // pair table: row v, lane l holds fp16 (L[v & 15], L[v >> 4]) at v*256 + l*4
   for (int i = tid; i < 256 * 32; i += kGemvThreads) {
-    const int v = i >> 5;
+    const int v = i >> 5, l = i & 31;
     const __half2 h = __floats2half2_rn(__uint_as_float(kNf4LevelBits[v & 15]), __uint_as_float(kNf4LevelBits[v >> 4]));
-    lut[i] = *reinterpret_cast<const uint32_t *>(&h);
+    *reinterpret_cast<uint32_t *>(at(lut_addr + v * 256 + l * 4)) = *reinterpret_cast<const uint32_t *>(&h);
   }
-  for (int i = tid; i < my_rg * kGemvWarps * 256; i += kGemvThreads) red[i] = 0.0f;
+  for (int i = 0; i < my_rg; ++i)
+    for (int e = tid; e < kGemvWarps * 256; e += kGemvThreads) reinterpret_cast<float *>(at(red_addr[i]))[e] = 0.0f;
   __syncthreads();
-  const uint32_t lut_lane = static_cast<uint32_t>(__cvta_generic_to_shared(lut)) + lane * 4;
+  // [lane * 4, -, table base bits 16..23, 24..31]: the byte permute inserts the code byte
+  const uint32_t laneword = (lut_addr & 0xffff0000u) | static_cast<uint32_t>(lane * 4);
   bool ok = true;
-
-  // warps whose 256-wide slice lies past K (K < 4096) only keep the ring's
-  // barrier counts: they wait for each stage and release it.
   const bool active = warp * 4 < CH / 64;
+
   for (int ch = 0; ch < nch && ok; ++ch) {
     const int64_t kb0 = (int64_t)ch * 64 + warp * 4;  // first block of this warp's quad (global)
     uint32_t xf[4][4][NG][2];
@@ -452,7 +521,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_bulk_kernel(const Ge
       unscale[ng][1] = pow2f(__shfl_sync(0xffffffffu, e, (2 * q + 1) * 4));
     }
 
-    // c2 of this thread's two rows for row group i: one value per (row, quad)
     auto c2_of = [&](int i, float (&c)[2]) {
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -460,20 +528,21 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_bulk_kernel(const Ge
         c[h] = active ? __ldg(a.c2 + ((row * nbk + kb0) >> 8)) : 0.0f;
       }
     };
+    auto release = [&](int u, int slot) -> bool {
+      ptx::mbar_arrive(&empty[slot]);
+      if (tid == 0 && u + kBulkStagesV4 < total) {
+        if (!ptx::mbar_wait(&empty[slot], (u / kBulkStagesV4) & 1, nullptr)) return false;
+        issue(u + kBulkStagesV4);
+      }
+      return true;
+    };
     auto process = [&](int i, const float (&c2v)[2]) -> bool {
       const int u = ch * my_rg + i;
-      const int slot = u % kBulkStages;
-      if (!ptx::mbar_wait(&full[slot], (u / kBulkStages) & 1, nullptr)) return false;
-      const uint8_t *st = ring + slot * stage_bytes;
+      const int slot = u % kBulkStagesV4;
+      if (!ptx::mbar_wait(&full[slot], (u / kBulkStagesV4) & 1, nullptr)) return false;
+      if (!active) return release(u, slot);
+      const uint8_t *st = at(stage_addr[slot]);
       const int kl = warp * 4;  // quad's first block within the chunk
-      if (!active) {
-        ptx::mbar_arrive(&empty[slot]);
-        if (tid == 0 && u + kBulkStages < total) {
-          if (!ptx::mbar_wait(&empty[slot], (u / kBulkStages) & 1, nullptr)) return false;
-          issue(u + kBulkStages);
-        }
-        return true;
-      }
       uint2 cw[4][2];
       uint32_t qw[2];
 #pragma unroll
@@ -481,11 +550,10 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_bulk_kernel(const Ge
         const int rw = g + 8 * h;
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          cw[j][h] = *reinterpret_cast<const uint2 *>(st + rw * (CH / 2) + (kl + j) * 32 + 8 * q);
-        qw[h] = *reinterpret_cast<const uint32_t *>(st + 16 * CH / 2 + rw * (CH / 64) + kl);
+          cw[j][h] = *reinterpret_cast<const uint2 *>(st + rw * RS + (kl + j) * 32 + 8 * q);
+        qw[h] = *reinterpret_cast<const uint32_t *>(st + 16 * RS + rw * (CH / 64) + kl);
       }
-      // this thread has read everything it needs from the stage
-      ptx::mbar_arrive(&empty[slot]);
+      if (!release(u, slot)) return false;
       float S[2][4];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -510,13 +578,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_bulk_kernel(const Ge
           const uint32_t w0 = (s < 2) ? cw[j][0].x : cw[j][0].y;
           const uint32_t w1 = (s < 2) ? cw[j][1].x : cw[j][1].y;
           const uint32_t p0 = (2 * s) & 3, p1 = (2 * s + 1) & 3;
-          const uint32_t b00 = __byte_perm(w0, 0u, 0x4440u | p0), b01 = __byte_perm(w0, 0u, 0x4440u | p1);
-          const uint32_t b10 = __byte_perm(w1, 0u, 0x4440u | p0), b11 = __byte_perm(w1, 0u, 0x4440u | p1);
           uint32_t a0, a1, a2, a3;
-          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a0) : "r"(lut_lane + (b00 << 7)));
-          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a1) : "r"(lut_lane + (b10 << 7)));
-          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a2) : "r"(lut_lane + (b01 << 7)));
-          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a3) : "r"(lut_lane + (b11 << 7)));
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a0) : "r"(__byte_perm(w0, laneword, 0x7604u | (p0 << 4))));
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a1) : "r"(__byte_perm(w1, laneword, 0x7604u | (p0 << 4))));
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a2) : "r"(__byte_perm(w0, laneword, 0x7604u | (p1 << 4))));
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a3) : "r"(__byte_perm(w1, laneword, 0x7604u | (p1 << 4))));
 #pragma unroll
           for (int ng = 0; ng < NG; ++ng) mma_16816_f16(acc[ng], a0, a1, a2, a3, xf[j][s][ng][0], xf[j][s][ng][1]);
         }
@@ -528,7 +594,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_bulk_kernel(const Ge
           part[ng][3] = fmaf(S[1][j], acc[ng][3], part[ng][3]);
         }
       }
-      float *rb = red + ((size_t)i * kGemvWarps + warp) * 256;
+      float *rb = reinterpret_cast<float *>(at(red_addr[i])) + warp * 256;
 #pragma unroll
       for (int ng = 0; ng < NG; ++ng) {
         const int t = 2 * q + 8 * ng;
@@ -536,11 +602,6 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_bulk_kernel(const Ge
         rb[g * 16 + t + 1] += part[ng][1] * unscale[ng][1];
         rb[(g + 8) * 16 + t] += part[ng][2] * unscale[ng][0];
         rb[(g + 8) * 16 + t + 1] += part[ng][3] * unscale[ng][1];
-      }
-      // refill the slot once every thread has released it
-      if (tid == 0 && u + kBulkStages < total) {
-        if (!ptx::mbar_wait(&empty[slot], (u / kBulkStages) & 1, nullptr)) return false;
-        issue(u + kBulkStages);
       }
       return true;
     };
@@ -556,8 +617,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_bulk_kernel(const Ge
   }
   if (!ok && lane == 0) raise_status(a.status, QLORA_ERR_TIMEOUT);
 
-  // LoRA up-projection (needs s T from the preceding kernel), then reduction.
-  griddep_wait();
+  // LoRA up-projection: B rows are loaded before waiting for s T.
   for (int i = warp; i < my_rg; i += kGemvWarps) {
     const int64_t n0 = (int64_t)(rg0 + i) * 16;
     float acc[NG][4];
@@ -572,6 +632,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_bulk_kernel(const Ge
         af[h] = (j0 + 2 * q < a.r) ? __ldg(src) : 0u;
         af[2 + h] = (j0 + 8 + 2 * q < a.r) ? __ldg(src + 4) : 0u;
       }
+      if (j0 == 0) griddep_wait();
 #pragma unroll
       for (int ng = 0; ng < NG; ++ng) {
         const int t = g + 8 * ng;
@@ -584,7 +645,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_bulk_kernel(const Ge
         mma_16816(acc[ng], af[0], af[1], af[2], af[3], b0, b1);
       }
     }
-    float *rb = red + ((size_t)i * kGemvWarps + warp) * 256;
+    float *rb = reinterpret_cast<float *>(at(red_addr[i])) + warp * 256;
 #pragma unroll
     for (int ng = 0; ng < NG; ++ng) {
       const int t = 2 * q + 8 * ng;
@@ -594,12 +655,13 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_bulk_kernel(const Ge
       rb[(g + 8) * 16 + t + 1] += acc[ng][3];
     }
   }
+  if (warp >= my_rg) griddep_wait();
   __syncthreads();
   for (int idx = tid; idx < my_rg * 256; idx += kGemvThreads) {
     const int i = idx >> 8, e = idx & 255, row = e >> 4, t = e & 15;
     const int64_t n = (int64_t)(rg0 + i) * 16 + row;
     if (t >= a.M) continue;
-    const float *rb = red + (size_t)i * kGemvWarps * 256 + e;
+    const float *rb = reinterpret_cast<const float *>(at(red_addr[i])) + e;
     float sum = 0.0f;
 #pragma unroll
     for (int w = 0; w < kGemvWarps; ++w) sum += rb[w * 256];
@@ -682,27 +744,13 @@ inline qlora_status launch_gemv(GemvArgs g, int dev, int sms, cudaStream_t st) {
   if (per > cap) per = cap;
   g.rg_per_cta = per;
   const int grid = (num_rg + per - 1) / per;
-  const int64_t CH = g.K < 4096 ? g.K : 4096;
-  const int bulk_smem = 256 * 32 * 4 + kBulkMaxRG * kGemvWarps * 256 * 4 +
-                        kBulkStages * static_cast<int>(16 * CH / 2 + 16 * CH / 64) + 2 * kBulkStages * 8;
+  const int bulk_smem = gemv_bulk_smem_bytes(g.K);
   const int smem = bulk ? bulk_smem : 256 * 32 * 4 + per * kGemvWarps * 256 * 4;
   static std::once_flag flags[4][64];
   static qlora_status results[4][64];
   const bool two = g.M > 8;
   const int which = (bulk ? 2 : 0) + (two ? 1 : 0);
-  auto kernel = bulk ? (two ? nf4_gemv_bulk_kernel<2> : nf4_gemv_bulk_kernel<1>)
-                     : (two ? nf4_gemv_lora_kernel<2> : nf4_gemv_lora_kernel<1>);
-  std::call_once(flags[which][dev], [&] {
-    const int max_smem = bulk ? 256 * 32 * 4 + kBulkMaxRG * kGemvWarps * 256 * 4 +
-                                    kBulkStages * (16 * 4096 / 2 + 16 * 4096 / 64) + 2 * kBulkStages * 8
-                              : 256 * 32 * 4 + kGemvMaxRG * kGemvWarps * 256 * 4;
-    results[which][dev] = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) ==
-                                  cudaSuccess
-                              ? QLORA_OK
-                              : QLORA_ERR_CUDA;
-    cudaGetLastError();
-  });
-  if (results[which][dev] != QLORA_OK) return results[which][dev];
+  const int max_smem = bulk ? gemv_bulk_smem_bytes(4096) : 256 * 32 * 4 + kGemvMaxRG * kGemvWarps * 256 * 4;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kGemvThreads);
@@ -713,7 +761,26 @@ inline qlora_status launch_gemv(GemvArgs g, int dev, int sms, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, g);
+  cudaError_t e;
+  if (bulk) {
+    auto kernel = two ? nf4_gemv_bulk_kernel<2> : nf4_gemv_bulk_kernel<1>;
+    std::call_once(flags[which][dev], [&] {
+      results[which][dev] = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) ==
+                                    cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+      cudaGetLastError();
+    });
+    if (results[which][dev] != QLORA_OK) return results[which][dev];
+    e = cudaLaunchKernelEx(&cfg, kernel, g, smem);
+  } else {
+    auto kernel = two ? nf4_gemv_lora_kernel<2> : nf4_gemv_lora_kernel<1>;
+    std::call_once(flags[which][dev], [&] {
+      results[which][dev] = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) ==
+                                    cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+      cudaGetLastError();
+    });
+    if (results[which][dev] != QLORA_OK) return results[which][dev];
+    e = cudaLaunchKernelEx(&cfg, kernel, g);
+  }
   if (e != cudaSuccess) {
     cudaGetLastError();
     return QLORA_ERR_CUDA;
