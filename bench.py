@@ -43,6 +43,27 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+# DRAM bytes (read + write) of one fused forward GEMM launch, mean over the block's
+# seven layers (4 of 8192x8192, 2 of 22016x8192, 1 of 8192x22016), from ncu
+# captures of the `cases` module's fwd_8192 / fwd_65b_up / fwd_65b_down.  The
+# figure belongs to the kernel sources it was measured on: it is reported only
+# while their digest still matches, else the traffic is null.
+FUSED_FWD_TRAFFIC_BYTES = 570.06e6
+FUSED_FWD_TRAFFIC_SOURCES = ("gemm_kernel.cuh", "sm100_ptx.cuh", "nf4_device.cuh", "qlora_nf4.cu")
+FUSED_FWD_TRAFFIC_DIGEST = "13f814ae0971338c"
+
+
+def fused_fwd_traffic():
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in FUSED_FWD_TRAFFIC_SOURCES:
+        with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "bit_nf4_quantized_27_b200", "csrc", f),
+                  "rb") as fh:
+            h.update(fh.read())
+    return FUSED_FWD_TRAFFIC_BYTES if h.hexdigest()[:16] == FUSED_FWD_TRAFFIC_DIGEST else None
+
+
 def layer_flops(m, n, k, r):
     fwd = 2 * m * n * k + 2 * m * r * (k + n)
     bwd = 2 * m * n * k + 4 * m * r * (n + k)
@@ -106,10 +127,11 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # CPU oracle baseline (bounded sample of the same step)
 # ---------------------------------------------------------------------------
-def oracle_sample(seconds_budget=20.0):
+def oracle_sample(seconds_budget=20.0, rows=2048, toks=1024):
     """Runs the oracle on row/token slices of the 65B-shaped block's layers:
-    quantise a 512-row slice of each weight, then forward+backward of 512 tokens
-    through it.  Returns (TFLOP/s, threads, description, seconds)."""
+    quantise a `rows`-row slice of each weight, then forward+backward of `toks`
+    tokens through it, layer after layer until `seconds_budget` is spent.
+    Returns (TFLOP/s, threads, description, seconds)."""
     import numpy as np
     from threadpoolctl import threadpool_info
 
@@ -117,7 +139,6 @@ def oracle_sample(seconds_budget=20.0):
     from bit_nf4_quantized_27_b200 import inputs as I
 
     wl = I.L65B_BLOCK
-    rows, toks = 512, 512
     flops, t_total, done = 0.0, 0.0, []
     for li, ly in enumerate(wl.layers):
         w = I.normal((rows, ly.k), 0.02, I.seed_for(wl.wid, I.W_ID, li)).float().numpy()
@@ -148,7 +169,7 @@ def run_reference(args, rank):
         return
     vals = []
     for i in range(args.warmup + args.steps):
-        v, threads, desc, secs = oracle_sample(seconds_budget=args.ref_seconds)
+        v, threads, desc, secs = oracle_sample(seconds_budget=args.ref_seconds, rows=512, toks=512)
         if i >= args.warmup:
             vals.append(v)
     value = statistics.median(vals)
@@ -480,7 +501,8 @@ def main():
         "roofline": {"bound": "tensor", "kernel": "NF4 fused tensor-core GEMM, forward call (T = X A^T + fused "
                                                   "dequant GEMM with the LoRA K steps), all 7 layers",
                      "achieved": fwd_tf, "peak": peak_tc, "unit": "TFLOP/s", "frac": fwd_tf / peak_tc,
-                     "traffic": None, "peak_kind": f"{peaks_kind} bf16 dense, sustained",
+                     "traffic": fused_fwd_traffic(), "traffic_unit": "bytes per fused forward launch",
+                     "peak_kind": f"{peaks_kind} bf16 dense, sustained",
                      "step_frac": value / world / peak_tc},
         "breakdown_ms_per_step": {"quantize": t_q, "forward": t_fwd, "backward": t_bwd,
                                   "forward_TFLOP/s": fwd_tf, "backward_TFLOP/s": bwd_tf},

@@ -6,6 +6,8 @@ CASE is one of:
   fwd_8192      forward of one 8192x8192 layer, 4096 tokens, r=64 (65B-shaped q)
   bwd_8192      backward of the same layer
   fwd_11008     forward of 11008x4096 (gate/up of the Llama-7B block), 2048 tokens
+  fwd_65b_up / bwd_65b_up       22016x8192 (gate/up of the 65B-shaped block), 4096 tokens
+  fwd_65b_down / bwd_65b_down   8192x22016 (down of the 65B-shaped block), 4096 tokens
   gemv_m1 / gemv_m4 / gemv_m16   decode forward, W 11008x4096, r=64
   quant_11008   quantise an 11008x4096 bf16 weight
   dequant_11008 dequantise it
@@ -39,7 +41,8 @@ def main(argv=None):
     c = args.case
     torch.cuda.set_device(0)
     if c.startswith(("fwd", "bwd")):
-        n, k, m = {"8192": (8192, 8192, 4096), "11008": (11008, 4096, 2048)}[c.split("_")[1]]
+        n, k, m = {"8192": (8192, 8192, 4096), "11008": (11008, 4096, 2048), "65b_up": (22016, 8192, 4096),
+                   "65b_down": (8192, 22016, 4096)}[c.split("_", 1)[1]]
         w, x, a, b, dy = _layer(n, k, m)
         q = bd.quantize(w)
         y, t = bd.linear_fwd(q, a, b, 16.0, x)

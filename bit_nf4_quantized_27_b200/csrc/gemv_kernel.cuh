@@ -325,8 +325,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_lora_kernel(const Ge
 // ---------------------------------------------------------------------------
 // Bulk-staged variant: each 16-row group's codes (16 x CH/2 contiguous bytes)
 // and block scales (16 x CH/64 bytes) arrive in shared memory through
-// cp.async.bulk into a 3-stage ring, so DRAM sees long contiguous reads and
-// about 100 KB stays in flight per SM without holding registers.  Requirements:
+// cp.async.bulk into a 2-stage ring, so DRAM sees long contiguous reads and
+// up to 68 KB stays in flight per SM without holding registers.  Requirements:
 // N % 16 == 0, K % 256 == 0 and (K <= 4096 or K % 4096 == 0); CH = min(K, 4096).
 // ---------------------------------------------------------------------------
 constexpr int kBulkMaxRG = 5;
