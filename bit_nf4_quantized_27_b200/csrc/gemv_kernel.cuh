@@ -48,6 +48,7 @@ struct GemvArgs {
   float *partial;           // unused scratch slot (reserved)
   uint32_t *status;
   int rg_per_cta;
+  int stages;               // bulk kernel: depth of the shared-memory ring
 };
 
 inline size_t gemv_workspace_bytes(int64_t, int64_t, int64_t) { return 0; }
@@ -56,6 +57,21 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
                                           uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Read-only shared-memory load and an MMA without `volatile`, so the compiler
+// may reorder them for latency (both have no side effects beyond their outputs).
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t v;
+  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void mma_16816_f16_nv(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                                 uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
       "{%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -346,30 +362,37 @@ inline bool gemv_bulk_ok(int64_t N, int64_t K) {
 // Shared memory of the bulk kernel.  The pair table sits at a 64 KB-aligned
 // shared address with a 256-byte row per byte value (a lane's entry at
 // row * 256 + lane * 4), so one byte permute builds the whole lookup address:
-// [lane * 4 | code byte | table base bits 16..31].  Row-group partial sums
-// (16 KB each), the stage ring and the barriers are placed before the table
-// where they fit and after it otherwise.
+// [lane * 4 | code byte | table base bits 16..31].  The stage ring, the
+// row-group partial sums and the barriers are placed before the table where
+// they fit and after it otherwise.
 constexpr uint32_t kBulkLutBytes = 256 * 256;
-constexpr uint32_t kBulkRedBytes = kGemvWarps * 256 * 4;
-constexpr int kBulkStagesV4 = 2;
+constexpr int kBulkMaxStages = 6;
+constexpr uint32_t kBulkSmemLimit = 232448;  // opt-in dynamic shared memory per CTA
 
-// Staged code rows are CH/2 + 32 bytes apart, so the 8 rows one warp reads in a
-// single instruction fall on 8 different 32-byte bank groups.
-__host__ __device__ inline uint32_t gemv_bulk_row_stride(int64_t K) {
-  const int64_t CH = K < 4096 ? K : 4096;
-  return static_cast<uint32_t>(CH / 2 + 32);
-}
+// A stage holds one 16-row group's codes for a chunk of CH = min(K, 4096)
+// columns, brought in by one 3-D TMA copy (128 bytes x 16 rows x CH/256
+// column chunks) with the 128-byte swizzle: shared layout [chunk][row][128 B]
+// with each 16-byte unit's index XORed with (row & 7), so the eight rows one
+// warp reads in an instruction land in different banks.  The stage's block
+// scales (16 rows x CH/64 bytes, row-major) follow the codes.
 __host__ __device__ inline uint32_t gemv_bulk_stage_bytes(int64_t K) {
   const int64_t CH = K < 4096 ? K : 4096;
-  return static_cast<uint32_t>((16 * gemv_bulk_row_stride(K) + 16 * CH / 64 + 127) & ~int64_t(127));
+  return static_cast<uint32_t>((16 * CH / 2 + 16 * CH / 64 + 1023) & ~int64_t(1023));
+}
+// Partial sums of one row group: [16 warps][16 rows][TR tokens] floats, TR = M
+// for M <= 8 (one n8 tile), else 16.
+__host__ __device__ inline int gemv_bulk_red_tokens(int M) { return M <= 8 ? M : 16; }
+__host__ __device__ inline uint32_t gemv_bulk_red_bytes(int M) {
+  return static_cast<uint32_t>(kGemvWarps * 16 * gemv_bulk_red_tokens(M) * 4);
 }
 
 // Placement of the bulk kernel's buffers around the 64 KB-aligned table, for a
-// dynamic window starting at shared address `base`; returns the end address.
+// dynamic window starting at shared address `base`.
 struct BulkLayout {
-  uint32_t lut, red[kBulkMaxRG], stage[kBulkStagesV4], bar, end;
+  uint32_t lut, red[kBulkMaxRG], stage[kBulkMaxStages], bar, end;
 };
-__host__ __device__ inline BulkLayout gemv_bulk_layout(uint32_t base, uint32_t stage_bytes) {
+__host__ __device__ inline BulkLayout gemv_bulk_layout(uint32_t base, uint32_t stage_bytes, int stages,
+                                                       uint32_t red_bytes) {
   BulkLayout L;
   L.lut = (base + 0xffffu) & ~0xffffu;
   uint32_t lo_next = base, hi_next = L.lut + kBulkLutBytes;
@@ -383,48 +406,61 @@ __host__ __device__ inline BulkLayout gemv_bulk_layout(uint32_t base, uint32_t s
     hi_next = hi + bytes;
     return hi;
   };
-  for (int i = 0; i < kBulkMaxRG; ++i) L.red[i] = place(kBulkRedBytes, 16);
-  for (int i = 0; i < kBulkStagesV4; ++i) L.stage[i] = place(stage_bytes, 128);
-  L.bar = place(64, 16);
+  for (int i = 0; i < kBulkMaxStages; ++i) L.stage[i] = i < stages ? place(stage_bytes, 1024) : 0u;
+  for (int i = 0; i < kBulkMaxRG; ++i) L.red[i] = place(red_bytes, 16);
+  L.bar = place(2 * kBulkMaxStages * 8, 16);
   L.end = hi_next > lo_next ? hi_next : lo_next;
   return L;
 }
 
-// Dynamic shared memory that covers the layout for any window start (16-byte
-// steps within a 64 KB period).
-inline int gemv_bulk_smem_bytes(int64_t K) {
-  const uint32_t sb = gemv_bulk_stage_bytes(K);
-  uint32_t worst = 0;
-  for (uint32_t base = 0; base < 65536; base += 16) {
-    const BulkLayout L = gemv_bulk_layout(base, sb);
-    if (L.end - base > worst) worst = L.end - base;
-  }
-  return static_cast<int>(worst);
+inline int gemv_bulk_smem_bytes(int64_t K, int stages, int M, uint32_t base) {
+  const BulkLayout L = gemv_bulk_layout(base, gemv_bulk_stage_bytes(K), stages, gemv_bulk_red_bytes(M));
+  return static_cast<int>(L.end - base);
+}
+
+// Largest stage count (at most `uses`, the stages one CTA consumes, but at least
+// two) whose layout fits a dynamic window starting at `base`; 0 if two do not fit.
+inline int gemv_bulk_stages(int64_t K, int M, uint32_t base, int uses) {
+  const int top = uses < 2 ? 2 : (uses > kBulkMaxStages ? kBulkMaxStages : uses);
+  for (int s = top; s >= 2; --s)
+    if (gemv_bulk_smem_bytes(K, s, M, base) <= static_cast<int>(kBulkSmemLimit)) return s;
+  return 0;
 }
 
 template <int NG>
-__global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_bulk_kernel(const GemvArgs a, int dyn_bytes) {
+__global__ void __launch_bounds__(kGemvThreads, 1)
+    nf4_gemv_bulk_kernel(const __grid_constant__ CUtensorMap tm_codes, const GemvArgs a, int dyn_bytes) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const int64_t CH = a.K < 4096 ? a.K : 4096;
-  const uint32_t stage_bytes = gemv_bulk_stage_bytes(a.K);
-  const uint32_t RS = gemv_bulk_row_stride(a.K);
+  const int S = a.stages;
+  const int TR = gemv_bulk_red_tokens(a.M);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, q = lane & 3;
 
   // ---- layout around the 64 KB-aligned table
   const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw));
-  const BulkLayout Lay = gemv_bulk_layout(base, stage_bytes);
-  const uint32_t lut_addr = Lay.lut;
-  const uint32_t *red_addr = Lay.red;
-  const uint32_t *stage_addr = Lay.stage;
-  const uint32_t bar_addr = Lay.bar;
-  if (Lay.end > base + static_cast<uint32_t>(dyn_bytes)) {  // cannot happen with the host's size
-    if (tid == 0) raise_status(a.status, QLORA_ERR_CUDA);
+  const BulkLayout Lay = gemv_bulk_layout(base, gemv_bulk_stage_bytes(a.K), S, gemv_bulk_red_bytes(a.M));
+  if (S < 2 || S > kBulkMaxStages || Lay.end > base + static_cast<uint32_t>(dyn_bytes)) {
+    if (tid == 0) raise_status(a.status, QLORA_ERR_CUDA);  // the host sized the window for another start
     return;
   }
+  const uint32_t lut_addr = Lay.lut;
   auto at = [&](uint32_t addr) { return smem_raw + (addr - base); };
-  uint64_t *full = reinterpret_cast<uint64_t *>(at(bar_addr));
-  uint64_t *empty = full + kBulkStagesV4;
+  // run-time indices pick addresses by selects, keeping the layout in registers
+  auto stage_at = [&](int slot) {
+    uint32_t v = Lay.stage[0];
+#pragma unroll
+    for (int k = 1; k < kBulkMaxStages; ++k) v = slot == k ? Lay.stage[k] : v;
+    return at(v);
+  };
+  auto red_at = [&](int i) {
+    uint32_t v = Lay.red[0];
+#pragma unroll
+    for (int k = 1; k < kBulkMaxRG; ++k) v = i == k ? Lay.red[k] : v;
+    return reinterpret_cast<float *>(at(v));
+  };
+  uint64_t *full = reinterpret_cast<uint64_t *>(at(Lay.bar));
+  uint64_t *empty = full + kBulkMaxStages;
 
   const int num_rg = static_cast<int>(a.N / 16);
   const int rg0 = blockIdx.x * a.rg_per_cta;
@@ -432,27 +468,27 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_bulk_kernel(const Ge
   const int64_t nbk = a.K / 64;
   const int nch = static_cast<int>(a.K / CH);
   const int total = my_rg * nch;
+  const int nw = static_cast<int>(CH / 256);  // warps with columns in a chunk
+  const bool active = warp < nw;
 
   // producer (thread 0): stage u = (chunk u / my_rg, row group u % my_rg)
   auto issue = [&](int u) {
     const int ch = u / my_rg, i = u % my_rg;
-    const int slot = u % kBulkStagesV4;
-    uint8_t *st = at(stage_addr[slot]);
+    const int slot = u % S;
+    uint8_t *st = stage_at(slot);
     const int64_t n0 = (int64_t)(rg0 + i) * 16;
     ptx::mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(16 * CH / 2 + 16 * CH / 64));
-    for (int rw = 0; rw < 16; ++rw)
-      bulk_g2s(st + rw * RS, a.codes + (n0 + rw) * (a.K / 2) + ch * (CH / 2), static_cast<uint32_t>(CH / 2),
-               &full[slot]);
+    ptx::tma_load_3d(st, &tm_codes, &full[slot], 0, static_cast<int32_t>(n0), ch * static_cast<int32_t>(CH / 256));
     if (CH == a.K) {
-      bulk_g2s(st + 16 * RS, a.scale_codes + n0 * nbk, static_cast<uint32_t>(16 * nbk), &full[slot]);
+      bulk_g2s(st + 16 * CH / 2, a.scale_codes + n0 * nbk, static_cast<uint32_t>(16 * nbk), &full[slot]);
     } else {
       for (int rw = 0; rw < 16; ++rw)
-        bulk_g2s(st + 16 * RS + rw * (CH / 64), a.scale_codes + (n0 + rw) * nbk + ch * (CH / 64),
+        bulk_g2s(st + 16 * CH / 2 + rw * (CH / 64), a.scale_codes + (n0 + rw) * nbk + ch * (CH / 64),
                  static_cast<uint32_t>(CH / 64), &full[slot]);
     }
   };
   if (tid == 0) {
-    for (int i = 0; i < kBulkStagesV4; ++i) {
+    for (int i = 0; i < S; ++i) {
       ptx::mbar_init(&full[i], 1);
       ptx::mbar_init(&empty[i], kGemvThreads);
     }
@@ -460,31 +496,15 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_bulk_kernel(const Ge
   }
   __syncthreads();
   if (tid == 0)
-    for (int u = 0; u < kBulkStagesV4 && u < total; ++u) issue(u);
+    for (int u = 0; u < S && u < total; ++u) issue(u);
 
-  // pair table: row v, lane l holds fp16 (L[v & 15], L[v >> 4]) at v*256 + l*4
-  for (int i = tid; i < 256 * 32; i += kGemvThreads) {
-    const int v = i >> 5, l = i & 31;
-    const __half2 h = __floats2half2_rn(__uint_as_float(kNf4LevelBits[v & 15]), __uint_as_float(kNf4LevelBits[v >> 4]));
-    *reinterpret_cast<uint32_t *>(at(lut_addr + v * 256 + l * 4)) = *reinterpret_cast<const uint32_t *>(&h);
-  }
-  for (int i = 0; i < my_rg; ++i)
-    for (int e = tid; e < kGemvWarps * 256; e += kGemvThreads) reinterpret_cast<float *>(at(red_addr[i]))[e] = 0.0f;
-  __syncthreads();
-  // [lane * 4, -, table base bits 16..23, 24..31]: the byte permute inserts the code byte
-  const uint32_t laneword = (lut_addr & 0xffff0000u) | static_cast<uint32_t>(lane * 4);
-  bool ok = true;
-  const bool active = warp * 4 < CH / 64;
-
-  for (int ch = 0; ch < nch && ok; ++ch) {
-    const int64_t kb0 = (int64_t)ch * 64 + warp * 4;  // first block of this warp's quad (global)
-    uint32_t xf[4][4][NG][2];
-    float unscale[NG][2];
+  // this warp's slice of X for a chunk (raw bf16)
+  uint4 xraw[NG][4][2];
+  auto load_x = [&](int ch) {
+    const int64_t kb0 = (int64_t)ch * 64 + warp * 4;
 #pragma unroll
     for (int ng = 0; ng < NG; ++ng) {
       const int t = g + 8 * ng;
-      uint4 raw[4][2];
-      uint32_t mx = 0;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
@@ -493,8 +513,42 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_bulk_kernel(const Ge
           v0 = __ldg(src);
           v1 = __ldg(src + 1);
         }
-        raw[j][0] = v0;
-        raw[j][1] = v1;
+        xraw[ng][j][0] = v0;
+        xraw[ng][j][1] = v1;
+      }
+    }
+  };
+  // pair table: row v, lane l holds fp16 (L[v & 15], L[v >> 4]) at v*256 + l*4;
+  // four lanes' identical entries per 16-byte store
+  for (int i = tid; i < 256 * 8; i += kGemvThreads) {
+    const int v = i >> 3;
+    const __half2 h = __floats2half2_rn(__uint_as_float(kNf4LevelBits[v & 15]), __uint_as_float(kNf4LevelBits[v >> 4]));
+    const uint32_t e = *reinterpret_cast<const uint32_t *>(&h);
+    *reinterpret_cast<uint4 *>(at(lut_addr + v * 256 + (i & 7) * 16)) = make_uint4(e, e, e, e);
+  }
+  __syncthreads();
+  // [lane * 4, -, table base bits 16..23, 24..31]: the byte permute inserts the code byte
+  const uint32_t laneword = (lut_addr & 0xffff0000u) | static_cast<uint32_t>(lane * 4);
+  // this thread's 8 code bytes of block 4*warp + j, row g (+8 for h = 1): chunk
+  // `warp`, line offset 32j + 8q, 16-byte unit (2j + q/2) XOR g
+  const uint32_t code_off = warp * 2048 + g * 128 + 8 * (q & 1);
+  uint32_t code_xo[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) code_xo[j] = static_cast<uint32_t>(((2 * j + (q >> 1)) ^ g) << 4);
+  bool ok = true;
+
+  for (int ch = 0; ch < nch && ok; ++ch) {
+    const int64_t kb0 = (int64_t)ch * 64 + warp * 4;  // first block of this warp's quad (global)
+    load_x(ch);
+    uint32_t xf[4][4][NG][2];
+    float unscale[NG][2];
+#pragma unroll
+    for (int ng = 0; ng < NG; ++ng) {
+      const uint4(&raw)[4][2] = xraw[ng];
+      uint32_t mx = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 v0 = raw[j][0], v1 = raw[j][1];
         mx = __vmaxu2(mx, __vmaxu2(__vmaxu2(v0.x & 0x7fff7fffu, v0.y & 0x7fff7fffu),
                                    __vmaxu2(v0.z & 0x7fff7fffu, v0.w & 0x7fff7fffu)));
         mx = __vmaxu2(mx, __vmaxu2(__vmaxu2(v1.x & 0x7fff7fffu, v1.y & 0x7fff7fffu),
@@ -530,18 +584,18 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_bulk_kernel(const Ge
     };
     auto release = [&](int u, int slot) -> bool {
       ptx::mbar_arrive(&empty[slot]);
-      if (tid == 0 && u + kBulkStagesV4 < total) {
-        if (!ptx::mbar_wait(&empty[slot], (u / kBulkStagesV4) & 1, nullptr)) return false;
-        issue(u + kBulkStagesV4);
+      if (tid == 0 && u + S < total) {
+        if (!ptx::mbar_wait(&empty[slot], (u / S) & 1, nullptr)) return false;
+        issue(u + S);
       }
       return true;
     };
     auto process = [&](int i, const float (&c2v)[2]) -> bool {
       const int u = ch * my_rg + i;
-      const int slot = u % kBulkStagesV4;
-      if (!ptx::mbar_wait(&full[slot], (u / kBulkStagesV4) & 1, nullptr)) return false;
+      const int slot = u % S;
+      if (!ptx::mbar_wait(&full[slot], (u / S) & 1, nullptr)) return false;
       if (!active) return release(u, slot);
-      const uint8_t *st = at(stage_addr[slot]);
+      const uint8_t *st = stage_at(slot);
       const int kl = warp * 4;  // quad's first block within the chunk
       uint2 cw[4][2];
       uint32_t qw[2];
@@ -550,20 +604,20 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_bulk_kernel(const Ge
         const int rw = g + 8 * h;
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          cw[j][h] = *reinterpret_cast<const uint2 *>(st + rw * RS + (kl + j) * 32 + 8 * q);
-        qw[h] = *reinterpret_cast<const uint32_t *>(st + 16 * RS + rw * (CH / 64) + kl);
+          cw[j][h] = *reinterpret_cast<const uint2 *>(st + code_off + h * 1024 + code_xo[j]);
+        qw[h] = *reinterpret_cast<const uint32_t *>(st + 16 * CH / 2 + rw * (CH / 64) + kl);
       }
       if (!release(u, slot)) return false;
-      float S[2][4];
+      float S4[2][4];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(qw[h] & 0xffffu), __NV_E4M3);
         const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(qw[h] >> 16), __NV_E4M3);
         const float2 f01 = __half22float2(__half2(lo)), f23 = __half22float2(__half2(hi));
-        S[h][0] = __fmul_rn(f01.x, c2v[h]);
-        S[h][1] = __fmul_rn(f01.y, c2v[h]);
-        S[h][2] = __fmul_rn(f23.x, c2v[h]);
-        S[h][3] = __fmul_rn(f23.y, c2v[h]);
+        S4[h][0] = __fmul_rn(f01.x, c2v[h]);
+        S4[h][1] = __fmul_rn(f01.y, c2v[h]);
+        S4[h][2] = __fmul_rn(f23.x, c2v[h]);
+        S4[h][3] = __fmul_rn(f23.y, c2v[h]);
       }
       float part[NG][4];
 #pragma unroll
@@ -573,35 +627,47 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_bulk_kernel(const Ge
         float acc[NG][4];
 #pragma unroll
         for (int ng = 0; ng < NG; ++ng) acc[ng][0] = acc[ng][1] = acc[ng][2] = acc[ng][3] = 0.0f;
+        // all 16 table lookups of the block first, then its 4 MMAs (the table
+        // is read-only here, so these loads may be scheduled freely)
+        uint32_t af[4][4];
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
           const uint32_t w0 = (s < 2) ? cw[j][0].x : cw[j][0].y;
           const uint32_t w1 = (s < 2) ? cw[j][1].x : cw[j][1].y;
           const uint32_t p0 = (2 * s) & 3, p1 = (2 * s + 1) & 3;
-          uint32_t a0, a1, a2, a3;
-          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a0) : "r"(__byte_perm(w0, laneword, 0x7604u | (p0 << 4))));
-          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a1) : "r"(__byte_perm(w1, laneword, 0x7604u | (p0 << 4))));
-          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a2) : "r"(__byte_perm(w0, laneword, 0x7604u | (p1 << 4))));
-          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a3) : "r"(__byte_perm(w1, laneword, 0x7604u | (p1 << 4))));
+          af[s][0] = lds_u32(__byte_perm(w0, laneword, 0x7604u | (p0 << 4)));
+          af[s][1] = lds_u32(__byte_perm(w1, laneword, 0x7604u | (p0 << 4)));
+          af[s][2] = lds_u32(__byte_perm(w0, laneword, 0x7604u | (p1 << 4)));
+          af[s][3] = lds_u32(__byte_perm(w1, laneword, 0x7604u | (p1 << 4)));
+        }
 #pragma unroll
-          for (int ng = 0; ng < NG; ++ng) mma_16816_f16(acc[ng], a0, a1, a2, a3, xf[j][s][ng][0], xf[j][s][ng][1]);
+        for (int s = 0; s < 4; ++s) {
+#pragma unroll
+          for (int ng = 0; ng < NG; ++ng)
+            mma_16816_f16_nv(acc[ng], af[s][0], af[s][1], af[s][2], af[s][3], xf[j][s][ng][0], xf[j][s][ng][1]);
         }
 #pragma unroll
         for (int ng = 0; ng < NG; ++ng) {
-          part[ng][0] = fmaf(S[0][j], acc[ng][0], part[ng][0]);
-          part[ng][1] = fmaf(S[0][j], acc[ng][1], part[ng][1]);
-          part[ng][2] = fmaf(S[1][j], acc[ng][2], part[ng][2]);
-          part[ng][3] = fmaf(S[1][j], acc[ng][3], part[ng][3]);
+          part[ng][0] = fmaf(S4[0][j], acc[ng][0], part[ng][0]);
+          part[ng][1] = fmaf(S4[0][j], acc[ng][1], part[ng][1]);
+          part[ng][2] = fmaf(S4[1][j], acc[ng][2], part[ng][2]);
+          part[ng][3] = fmaf(S4[1][j], acc[ng][3], part[ng][3]);
         }
       }
-      float *rb = reinterpret_cast<float *>(at(red_addr[i])) + warp * 256;
+      // this warp's slot of row group i: written by the first chunk, accumulated by later ones
+      float *rb = red_at(i) + warp * 16 * TR;
 #pragma unroll
       for (int ng = 0; ng < NG; ++ng) {
         const int t = 2 * q + 8 * ng;
-        rb[g * 16 + t] += part[ng][0] * unscale[ng][0];
-        rb[g * 16 + t + 1] += part[ng][1] * unscale[ng][1];
-        rb[(g + 8) * 16 + t] += part[ng][2] * unscale[ng][0];
-        rb[(g + 8) * 16 + t + 1] += part[ng][3] * unscale[ng][1];
+        const float v00 = part[ng][0] * unscale[ng][0], v01 = part[ng][1] * unscale[ng][1];
+        const float v10 = part[ng][2] * unscale[ng][0], v11 = part[ng][3] * unscale[ng][1];
+        if (ch == 0) {
+          if (t < TR) rb[g * TR + t] = v00, rb[(g + 8) * TR + t] = v10;
+          if (t + 1 < TR) rb[g * TR + t + 1] = v01, rb[(g + 8) * TR + t + 1] = v11;
+        } else {
+          if (t < TR) rb[g * TR + t] += v00, rb[(g + 8) * TR + t] += v10;
+          if (t + 1 < TR) rb[g * TR + t + 1] += v01, rb[(g + 8) * TR + t + 1] += v11;
+        }
       }
       return true;
     };
@@ -617,22 +683,59 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_bulk_kernel(const Ge
   }
   if (!ok && lane == 0) raise_status(a.status, QLORA_ERR_TIMEOUT);
 
-  // LoRA up-projection: B rows are loaded before waiting for s T.
-  for (int i = warp; i < my_rg; i += kGemvWarps) {
-    const int64_t n0 = (int64_t)(rg0 + i) * 16;
+  // LoRA up-projection, added to warp 0's slot of each row group once every
+  // warp has written its own.  B rows are loaded before the barrier, s T after
+  // waiting for the kernel that computes it.
+  const int lora_rg = warp < my_rg ? warp : -1;
+  uint32_t bfr[4][4];
+  if (lora_rg >= 0) {
+    const int64_t n0 = (int64_t)(rg0 + lora_rg) * 16;
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const int j0 = 16 * jj;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t *src = reinterpret_cast<const uint32_t *>(a.B + (n0 + g + 8 * h) * a.r + j0 + 2 * q);
+        bfr[jj][h] = (j0 + 2 * q < a.r) ? __ldg(src) : 0u;
+        bfr[jj][2 + h] = (j0 + 8 + 2 * q < a.r) ? __ldg(src + 4) : 0u;
+      }
+    }
+  }
+  __syncthreads();
+  griddep_wait();
+  if (lora_rg >= 0) {
+    const int64_t n0 = (int64_t)(rg0 + lora_rg) * 16;
     float acc[NG][4];
 #pragma unroll
     for (int ng = 0; ng < NG; ++ng) acc[ng][0] = acc[ng][1] = acc[ng][2] = acc[ng][3] = 0.0f;
-    for (int j0 = 0; j0 < a.r; j0 += 16) {
-      uint32_t af[4];
+    // the first 64 ranks: every s T fragment loaded at once, then the MMAs
+    uint32_t bt[4][NG][2];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int64_t row = n0 + g + 8 * h;
-        const uint32_t *src = reinterpret_cast<const uint32_t *>(a.B + row * a.r + j0 + 2 * q);
-        af[h] = (j0 + 2 * q < a.r) ? __ldg(src) : 0u;
-        af[2 + h] = (j0 + 8 + 2 * q < a.r) ? __ldg(src + 4) : 0u;
+    for (int jj = 0; jj < 4; ++jj) {
+      const int j0 = 16 * jj;
+#pragma unroll
+      for (int ng = 0; ng < NG; ++ng) {
+        const int t = g + 8 * ng;
+        const uint32_t *src = reinterpret_cast<const uint32_t *>(a.sT + (int64_t)t * a.r + j0 + 2 * q);
+        bt[jj][ng][0] = (t < a.M && j0 + 2 * q < a.r) ? __ldg(src) : 0u;
+        bt[jj][ng][1] = (t < a.M && j0 + 8 + 2 * q < a.r) ? __ldg(src + 4) : 0u;
       }
-      if (j0 == 0) griddep_wait();
+    }
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+      for (int ng = 0; ng < NG; ++ng)
+        mma_16816(acc[ng], bfr[jj][0], bfr[jj][1], bfr[jj][2], bfr[jj][3], bt[jj][ng][0], bt[jj][ng][1]);
+    for (int j0 = 64; j0 < a.r; j0 += 16) {
+      uint32_t af[4];
+      {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t *src = reinterpret_cast<const uint32_t *>(a.B + (n0 + g + 8 * h) * a.r + j0 + 2 * q);
+          af[h] = (j0 + 2 * q < a.r) ? __ldg(src) : 0u;
+          af[2 + h] = (j0 + 8 + 2 * q < a.r) ? __ldg(src + 4) : 0u;
+        }
+      }
 #pragma unroll
       for (int ng = 0; ng < NG; ++ng) {
         const int t = g + 8 * ng;
@@ -645,26 +748,23 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_bulk_kernel(const Ge
         mma_16816(acc[ng], af[0], af[1], af[2], af[3], b0, b1);
       }
     }
-    float *rb = reinterpret_cast<float *>(at(red_addr[i])) + warp * 256;
+    float *rb = red_at(lora_rg);  // warp 0's slot
 #pragma unroll
     for (int ng = 0; ng < NG; ++ng) {
       const int t = 2 * q + 8 * ng;
-      rb[g * 16 + t] += acc[ng][0];
-      rb[g * 16 + t + 1] += acc[ng][1];
-      rb[(g + 8) * 16 + t] += acc[ng][2];
-      rb[(g + 8) * 16 + t + 1] += acc[ng][3];
+      if (t < TR) rb[g * TR + t] += acc[ng][0], rb[(g + 8) * TR + t] += acc[ng][2];
+      if (t + 1 < TR) rb[g * TR + t + 1] += acc[ng][1], rb[(g + 8) * TR + t + 1] += acc[ng][3];
     }
   }
-  if (warp >= my_rg) griddep_wait();
   __syncthreads();
-  for (int idx = tid; idx < my_rg * 256; idx += kGemvThreads) {
-    const int i = idx >> 8, e = idx & 255, row = e >> 4, t = e & 15;
+  // deterministic sum over the warps that hold columns, in warp order
+  const int per_rg = 16 * a.M;
+  for (int idx = tid; idx < my_rg * per_rg; idx += kGemvThreads) {
+    const int i = idx / per_rg, e = idx - i * per_rg, row = e / a.M, t = e - row * a.M;
     const int64_t n = (int64_t)(rg0 + i) * 16 + row;
-    if (t >= a.M) continue;
-    const float *rb = reinterpret_cast<const float *>(at(red_addr[i])) + e;
+    const float *rb = red_at(i) + row * TR + t;
     float sum = 0.0f;
-#pragma unroll
-    for (int w = 0; w < kGemvWarps; ++w) sum += rb[w * 256];
+    for (int w = 0; w < nw; ++w) sum += rb[w * 16 * TR];
     if (a.y_f32) reinterpret_cast<float *>(a.Y)[(int64_t)t * a.N + n] = sum;
     else reinterpret_cast<__nv_bfloat16 *>(a.Y)[(int64_t)t * a.N + n] = __float2bfloat16_rn(sum);
   }
@@ -672,11 +772,17 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_bulk_kernel(const Ge
 
 // T = X A^T for M <= 16 tokens on tensor cores, in few CTAs so that it runs on
 // SMs the decode GEMV leaves free.  CTA c computes rank rows [16c, 16c + 16):
-// 8 warps split K, each runs m16n8k16 MMAs with A = 16 rows of the LoRA A matrix
-// and B = X^T (tokens), both bf16; the partials are summed over the warps in a
-// fixed order.  Writes s*T (bf16) and, if T_hi is given, (T_hi, T_lo).
+// 8 warps split K in 64-column blocks (warp w takes blocks w, w + 8, ...), each
+// runs m16n8k16 MMAs with A = 16 rows of the LoRA A matrix and B = X^T (tokens),
+// both bf16.  Inside a block, k is permuted identically for A and X (thread quad
+// q owns k in [16q, 16q + 16)), so each thread reads two 16-byte vectors per row
+// and block, and a warp has kLoraDownBlocks blocks of loads in flight before its
+// first MMA.  The partials are summed over the warps in a fixed order.  Writes
+// s*T (bf16) and, if T_hi is given, (T_hi, T_lo).
 constexpr int kLoraDownThreads = 256;
-__global__ void __launch_bounds__(kLoraDownThreads) lora_down_small_kernel(
+constexpr int kLoraDownBlocks = 4;
+template <int NG>
+__global__ void __launch_bounds__(kLoraDownThreads, 1) lora_down_small_kernel(
     const __nv_bfloat16 *__restrict__ X, const __nv_bfloat16 *__restrict__ A, int M, int64_t K, int r, float s,
     __nv_bfloat16 *__restrict__ sT, __nv_bfloat16 *__restrict__ T_hi, __nv_bfloat16 *__restrict__ T_lo) {
   griddep_launch_dependents();
@@ -684,40 +790,57 @@ __global__ void __launch_bounds__(kLoraDownThreads) lora_down_small_kernel(
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, q = lane & 3;
   const int j0 = blockIdx.x * 16;
-  const int64_t nk16 = K / 16;
-  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-  const int rows[2] = {j0 + g, j0 + g + 8};
-  for (int64_t kk = warp; kk < nk16; kk += kLoraDownThreads / 32) {
-    const int64_t k = kk * 16 + 2 * q;
-    uint32_t af[4];
+  const int64_t nb = K / 64;
+  float acc[NG][4];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const bool rv = rows[h] < r;
-      const uint32_t *src = reinterpret_cast<const uint32_t *>(A + (int64_t)rows[h] * K + k);
-      af[h] = rv ? __ldg(src) : 0u;
-      af[2 + h] = rv ? __ldg(src + 4) : 0u;
+  for (int ng = 0; ng < NG; ++ng) acc[ng][0] = acc[ng][1] = acc[ng][2] = acc[ng][3] = 0.0f;
+  const bool rv[2] = {j0 + g < r, j0 + g + 8 < r};
+  for (int64_t kb0 = warp; kb0 < nb; kb0 += (kLoraDownThreads / 32) * kLoraDownBlocks) {
+    uint4 av[kLoraDownBlocks][2][2], xv[kLoraDownBlocks][NG][2];
+#pragma unroll
+    for (int u = 0; u < kLoraDownBlocks; ++u) {
+      const int64_t kb = kb0 + (kLoraDownThreads / 32) * u;
+      const bool kin = kb < nb;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(A + (int64_t)(j0 + g + 8 * h) * K + kb * 64 + 16 * q);
+        av[u][h][0] = (kin && rv[h]) ? __ldg(src) : make_uint4(0, 0, 0, 0);
+        av[u][h][1] = (kin && rv[h]) ? __ldg(src + 1) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int ng = 0; ng < NG; ++ng) {
+        const int t = g + 8 * ng;
+        const uint4 *src = reinterpret_cast<const uint4 *>(X + (int64_t)t * K + kb * 64 + 16 * q);
+        xv[u][ng][0] = (kin && t < M) ? __ldg(src) : make_uint4(0, 0, 0, 0);
+        xv[u][ng][1] = (kin && t < M) ? __ldg(src + 1) : make_uint4(0, 0, 0, 0);
+      }
     }
 #pragma unroll
-    for (int ng = 0; ng < 2; ++ng) {
-      const int t = g + 8 * ng;
-      if (ng * 8 >= M) break;
-      uint32_t b0 = 0, b1 = 0;
-      if (t < M) {
-        const uint32_t *src = reinterpret_cast<const uint32_t *>(X + (int64_t)t * K + k);
-        b0 = __ldg(src);
-        b1 = __ldg(src + 4);
+    for (int u = 0; u < kLoraDownBlocks; ++u) {
+#pragma unroll
+      for (int st = 0; st < 4; ++st) {
+        // step st uses k = 16q + 4st + {0, 1} (fragment slots 2q, 2q+1) and + {2, 3} (slots 2q+8, 2q+9)
+        const int hv = st >> 1;
+        const bool zw = st & 1;
+        const uint32_t a0 = zw ? av[u][0][hv].z : av[u][0][hv].x, a2 = zw ? av[u][0][hv].w : av[u][0][hv].y;
+        const uint32_t a1 = zw ? av[u][1][hv].z : av[u][1][hv].x, a3 = zw ? av[u][1][hv].w : av[u][1][hv].y;
+#pragma unroll
+        for (int ng = 0; ng < NG; ++ng) {
+          const uint32_t b0 = zw ? xv[u][ng][hv].z : xv[u][ng][hv].x, b1 = zw ? xv[u][ng][hv].w : xv[u][ng][hv].y;
+          mma_16816(acc[ng], a0, a1, a2, a3, b0, b1);
+        }
       }
-      mma_16816(acc[ng], af[0], af[1], af[2], af[3], b0, b1);
     }
   }
   // C fragment: rows g / g+8 (rank), columns 2q, 2q+1 (+8 ng) (tokens)
 #pragma unroll
   for (int ng = 0; ng < 2; ++ng) {
     const int t = 2 * q + 8 * ng;
-    red[warp][g][t] = acc[ng][0];
-    red[warp][g][t + 1] = acc[ng][1];
-    red[warp][g + 8][t] = acc[ng][2];
-    red[warp][g + 8][t + 1] = acc[ng][3];
+    const bool have = ng < NG;
+    red[warp][g][t] = have ? acc[ng < NG ? ng : 0][0] : 0.0f;
+    red[warp][g][t + 1] = have ? acc[ng < NG ? ng : 0][1] : 0.0f;
+    red[warp][g + 8][t] = have ? acc[ng < NG ? ng : 0][2] : 0.0f;
+    red[warp][g + 8][t + 1] = have ? acc[ng < NG ? ng : 0][3] : 0.0f;
   }
   __syncthreads();
   // one output per thread: rank row tid / 16, token tid % 16
@@ -736,21 +859,51 @@ __global__ void __launch_bounds__(kLoraDownThreads) lora_down_small_kernel(
   }
 }
 
-inline qlora_status launch_gemv(GemvArgs g, int dev, int sms, cudaStream_t st) {
+// Start of the dynamic shared-memory window of a kernel without static shared
+// memory: after the block's system reservation.  The bulk kernel recomputes its
+// layout from its real window start and reports an error if it does not fit.
+inline uint32_t dyn_smem_base(int dev) {
+  static std::once_flag flags[64];
+  static uint32_t base[64];
+  std::call_once(flags[dev], [&] {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess) {
+      v = 0;
+      cudaGetLastError();
+    }
+    base[dev] = static_cast<uint32_t>(v);
+  });
+  return base[dev];
+}
+
+inline qlora_status launch_gemv(GemvArgs g, const CUtensorMap *tm_codes, int dev, int sms, cudaStream_t st) {
   const int num_rg = static_cast<int>((g.N + 15) / 16);
-  const bool bulk = gemv_bulk_ok(g.N, g.K);
+  bool bulk = tm_codes != nullptr && gemv_bulk_ok(g.N, g.K);
   const int cap = bulk ? kBulkMaxRG : kGemvMaxRG;
   int per = (num_rg + sms - 1) / sms;
   if (per > cap) per = cap;
   g.rg_per_cta = per;
+  g.stages = 0;
+  int smem = 0;
+  if (bulk) {
+    const int64_t CH = g.K < 4096 ? g.K : 4096;
+    const uint32_t base = dyn_smem_base(dev);
+    g.stages = gemv_bulk_stages(g.K, g.M, base, per * static_cast<int>(g.K / CH));
+    if (g.stages == 0) bulk = false;
+    else smem = gemv_bulk_smem_bytes(g.K, g.stages, g.M, base);
+  }
+  if (!bulk) {
+    per = (num_rg + sms - 1) / sms;
+    if (per > kGemvMaxRG) per = kGemvMaxRG;
+    g.rg_per_cta = per;
+    smem = 256 * 32 * 4 + per * kGemvWarps * 256 * 4;
+  }
   const int grid = (num_rg + per - 1) / per;
-  const int bulk_smem = gemv_bulk_smem_bytes(g.K);
-  const int smem = bulk ? bulk_smem : 256 * 32 * 4 + per * kGemvWarps * 256 * 4;
   static std::once_flag flags[4][64];
   static qlora_status results[4][64];
   const bool two = g.M > 8;
   const int which = (bulk ? 2 : 0) + (two ? 1 : 0);
-  const int max_smem = bulk ? gemv_bulk_smem_bytes(4096) : 256 * 32 * 4 + kGemvMaxRG * kGemvWarps * 256 * 4;
+  const int max_smem = bulk ? static_cast<int>(kBulkSmemLimit) : 256 * 32 * 4 + kGemvMaxRG * kGemvWarps * 256 * 4;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kGemvThreads);
@@ -770,7 +923,7 @@ inline qlora_status launch_gemv(GemvArgs g, int dev, int sms, cudaStream_t st) {
       cudaGetLastError();
     });
     if (results[which][dev] != QLORA_OK) return results[which][dev];
-    e = cudaLaunchKernelEx(&cfg, kernel, g, smem);
+    e = cudaLaunchKernelEx(&cfg, kernel, *tm_codes, g, smem);
   } else {
     auto kernel = two ? nf4_gemv_lora_kernel<2> : nf4_gemv_lora_kernel<1>;
     std::call_once(flags[which][dev], [&] {

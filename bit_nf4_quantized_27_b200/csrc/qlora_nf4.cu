@@ -58,6 +58,22 @@ bool make_tmap(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, uint32_t
   return r == CUDA_SUCCESS;
 }
 
+// NF4 codes [N][K/2 bytes] as a 3-D map (128 bytes, N rows, K/256 chunks of 128
+// bytes), box 128 x 16 rows x `chunks`, 128-byte swizzle: the decode GEMV's
+// stage layout [chunk][row][128 B].
+bool tmap_codes_gemv(CUtensorMap *m, const void *codes, int64_t N, int64_t K, uint32_t chunks) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(K / 256)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K / 2), 128};
+  const cuuint32_t box[3] = {128, 16, chunks};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(codes), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool tmap_bf16(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
                uint32_t box_outer) {
   return make_tmap(m, ptr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, inner, outer, inner, box_inner, box_outer, true);
@@ -236,9 +252,11 @@ qlora_status qlora_linear_fwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
 
   if (M <= kGemvMaxM) {
     __nv_bfloat16 *th = static_cast<__nv_bfloat16 *>(T_save);
-    lora_down_small_kernel<<<(ad->r + 15) / 16, kLoraDownThreads, 0, st>>>(static_cast<const __nv_bfloat16 *>(X),
-                                                  static_cast<const __nv_bfloat16 *>(ad->A), (int)M, K, ad->r, sc,
-                                                  static_cast<__nv_bfloat16 *>(sT), th, th ? th + M * ad->r : nullptr);
+    auto down = M > 8 ? lora_down_small_kernel<2> : lora_down_small_kernel<1>;
+    down<<<(ad->r + 15) / 16, kLoraDownThreads, 0, st>>>(static_cast<const __nv_bfloat16 *>(X),
+                                                        static_cast<const __nv_bfloat16 *>(ad->A), (int)M, K, ad->r, sc,
+                                                        static_cast<__nv_bfloat16 *>(sT), th,
+                                                        th ? th + M * ad->r : nullptr);
     if ((s = launch_status()) != QLORA_OK) return s;
     GemvArgs g{};
     g.codes = W->codes; g.scale_codes = W->scale_codes; g.c2 = W->c2;
@@ -250,7 +268,10 @@ qlora_status qlora_linear_fwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
     g.Y = Y; g.y_f32 = y_dtype == QLORA_F32;
     g.partial = reinterpret_cast<float *>(wsb + QLORA_STATUS_BYTES + mr);
     g.status = status_ptr(ws);
-    return launch_gemv(g, dev, sms, st);
+    CUtensorMap tmc;
+    const bool staged = gemv_bulk_ok(N, K) &&
+                        tmap_codes_gemv(&tmc, W->codes, N, K, static_cast<uint32_t>((K < 4096 ? K : 4096) / 256));
+    return launch_gemv(g, staged ? &tmc : nullptr, dev, sms, st);
   }
 
   {

@@ -103,6 +103,21 @@ def test_gemv_path_small_shapes(m):
         check(f"T m={m}", t[0].float() + t[1].float(), tr)
 
 
+@pytest.mark.parametrize("n,k,m,r", [(1024, 256, 1, 8), (2048, 1024, 3, 16), (4096, 8192, 5, 64),
+                                     (1040, 4096, 8, 128), (2064, 12288, 12, 64), (3072, 4096, 16, 64),
+                                     (4816, 1024, 2, 64), (1536, 4096, 9, 48)])
+def test_gemv_staged_shapes(n, k, m, r):
+    # staged decode kernel: fewer active warps (K < 4096), 4096-column chunks
+    # (K > 4096), ranks beyond 64, both partial-sum widths (M <= 8 and M > 8), and
+    # a last CTA with fewer row groups than the others
+    c = _custom(n, k, m, r, 31 * n + k + m)
+    qg, a, b, x, _ = c.gpu()
+    y, t = bd.linear_fwd(qg, a, b, c.alpha, x, y_dtype=torch.float32)
+    yr, tr = c.ref_fwd()
+    check(f"y {n}x{k} m={m} r={r}", y, yr)
+    check(f"T {n}x{k} m={m} r={r}", t[0].float() + t[1].float(), tr)
+
+
 @pytest.mark.parametrize("m", [1, 4, 16])
 def test_gemv_workload_11008x4096(m):
     wl = I.GEMV
