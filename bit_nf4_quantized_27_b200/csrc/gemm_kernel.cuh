@@ -526,15 +526,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           }
         }
       }
-      // refill this slot with the scale of the step two ahead
-      scale_src(ptile, pks, qs, cs);
-      advance(ptile, pks);
       if (!ptx::mbar_wait(&empty_b[sb], pb ^ 1, abort_flag)) return false;
       store_row128(sB + sb * C::B_STAGE + atom_off, row_in, o);
       // Each thread orders its own writes before the tensor core's reads and
       // arrives itself (one arrival per thread).
       ptx::fence_proxy_async_smem();
       ptx::mbar_arrive(&full_b[sb]);
+      // refill this slot with the scale of the step two ahead; issued after the
+      // arrive, whose release would otherwise wait for these loads
+      scale_src(ptile, pks, qs, cs);
+      advance(ptile, pks);
       if (++sb == C::SB) { sb = 0; pb ^= 1; }
       advance(tile, ks);
       return true;

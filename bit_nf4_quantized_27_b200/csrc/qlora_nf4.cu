@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "gemm_kernel.cuh"
+#include "gemm_pair_kernel.cuh"
 #include "gemv_kernel.cuh"
 #include "host_common.h"
 #include "qlora_nf4.h"
@@ -90,6 +91,53 @@ qlora_status set_smem(F kernel, int bytes, int dev, std::once_flag *flags, qlora
   });
   return results[dev];
 }
+
+// The fused NF4 GEMM on CTA pairs, persistent over as many pairs as fit at
+// once.  Returns QLORA_ERR_UNSUPPORTED_SHAPE when no pair cluster can be
+// resident (the caller then uses the single-CTA kernel).
+template <bool B_MN, int MT>
+qlora_status launch_gemm_pair(const CUtensorMap &tmA, const CUtensorMap &tmA2, const CUtensorMap &tmCodes,
+                              const GemmArgs &args, int dev, cudaStream_t st) {
+  using C = GemmPairCfg<B_MN, MT>;
+  auto kernel = gemm_nf4_pair_kernel<B_MN, MT>;
+  static std::once_flag flags[64], occ_flags[64];
+  static qlora_status results[64];
+  static int max_clusters[64];
+  qlora_status s = set_smem(kernel, C::SMEM_BYTES, dev, flags, results);
+  if (s != QLORA_OK) return s;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  std::call_once(occ_flags[dev], [&] {
+    cudaLaunchConfig_t q = cfg;
+    q.gridDim = dim3(2);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &q) != cudaSuccess) n = 0;
+    cudaGetLastError();
+    max_clusters[dev] = n;
+  });
+  if (max_clusters[dev] <= 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  const int num_m = (args.M_rows + 2 * C::BM * MT - 1) / (2 * C::BM * MT);
+  const int num_n = (args.N_cols + C::BN - 1) / C::BN;
+  const int clusters = std::max(1, std::min(num_m * num_n, max_clusters[dev]));
+  cfg.gridDim = dim3(2 * clusters);
+  if (cudaLaunchKernelEx(&cfg, kernel, tmA, tmA2, tmCodes, args) != cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  return QLORA_OK;
+}
+
+// Token counts from which the fused GEMMs run on CTA pairs (512-token tiles).
+constexpr int64_t kPairMinRows = 257;
 
 template <bool A_MN, bool B_MN, bool NF4, int BN, int MT>
 qlora_status launch_gemm(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmA2,
@@ -281,9 +329,10 @@ qlora_status qlora_linear_fwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
       return s;
   }
 
-  CUtensorMap tmX, tmCodes, tmT;
+  CUtensorMap tmX, tmCodes, tmT, tmCodesPair;
   if (!tmap_bf16(&tmX, X, K, M, 64, 128) || !tmap_bf16(&tmT, sT, ad->r, M, 64, 128) ||
-      !make_tmap(&tmCodes, W->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, K / 2, 32, 256, false))
+      !make_tmap(&tmCodes, W->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, K / 2, 32, 256, false) ||
+      !make_tmap(&tmCodesPair, W->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, K / 2, 32, 128, false))
     return QLORA_ERR_CUDA;
   GemmArgs g{};
   g.M_rows = (int)M;
@@ -302,6 +351,10 @@ qlora_status qlora_linear_fwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
   g.lora_b2 = static_cast<const __nv_bfloat16 *>(ad->B);
   g.lora_ld = ad->r;
   g.status = status_ptr(ws);
+  if (M >= kPairMinRows) {
+    s = launch_gemm_pair<false, kFusedMT>(tmX, tmT, tmCodesPair, g, dev, st);
+    if (s != QLORA_ERR_UNSUPPORTED_SHAPE) return s;
+  }
   return launch_gemm<false, false, true, 256, kFusedMT>(tmX, tmX, tmT, tmX, tmCodes, g, dev, sms, st);
 }
 
@@ -356,9 +409,10 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
   }
   // dX = dY W' + (s U) A
   {
-    CUtensorMap tmDY, tmU, tmCodes;
+    CUtensorMap tmDY, tmU, tmCodes, tmCodesPair;
     if (!tmap_bf16(&tmDY, dY, N, M, 64, 128) || !tmap_bf16(&tmU, sU_hi, r, M, 64, 128) ||
-        !make_tmap(&tmCodes, W->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, K / 2, 128, 64, false))
+        !make_tmap(&tmCodes, W->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, K / 2, 128, 64, false) ||
+        !make_tmap(&tmCodesPair, W->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, K / 2, 64, 64, false))
       return QLORA_ERR_CUDA;
     GemmArgs g{};
     g.M_rows = (int)M;
@@ -377,8 +431,11 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
     g.lora_b2 = static_cast<const __nv_bfloat16 *>(ad->A);
     g.lora_ld = K;
     g.status = status;
-    if ((s = launch_gemm<false, true, true, 256, kFusedMT>(tmDY, tmDY, tmU, tmDY, tmCodes, g, dev, sms, st)) != QLORA_OK)
-      return s;
+    s = M >= kPairMinRows ? launch_gemm_pair<true, kFusedMT>(tmDY, tmU, tmCodesPair, g, dev, st)
+                          : QLORA_ERR_UNSUPPORTED_SHAPE;
+    if (s == QLORA_ERR_UNSUPPORTED_SHAPE)
+      s = launch_gemm<false, true, true, 256, kFusedMT>(tmDY, tmDY, tmU, tmDY, tmCodes, g, dev, sms, st);
+    if (s != QLORA_OK) return s;
   }
   // dA^T [K, r] = X^T (s U_hi + s U_lo)  -> stored transposed into dA [r, K]
   {

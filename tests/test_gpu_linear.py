@@ -150,6 +150,16 @@ def test_backward_recomputes_t():
     check("dB", db, dbr)
 
 
+@pytest.mark.parametrize("n,k,m,r", [(1000, 320, 600, 16), (264, 640, 513, 128), (4104, 128, 1030, 8),
+                                     (512, 1024, 257, 64)])
+def test_cta_pair_path_ragged(n, k, m, r):
+    # from 257 tokens the fused forward / dX GEMMs run on CTA pairs (512-token
+    # tiles, 256 columns split between the two CTAs): ragged N, K and M
+    c = _custom(n, k, m, r, 11 * n + k + m + r)
+    for dt in (torch.float32, torch.bfloat16):
+        _check_all(c, *_run_fwd_bwd(c, dt, dt))
+
+
 @pytest.mark.parametrize("m", [4, 300])
 def test_b_zero_is_base_layer(m):
     c = _custom(512, 512, m, 64, 77, b_std=0.0)
@@ -192,8 +202,9 @@ def test_autograd_wrapper():
     check("dB", b.grad, dbr)
 
 
-def test_deterministic():
-    c = _custom(1024, 1024, 256, 64, 3)
+@pytest.mark.parametrize("m", [256, 300])
+def test_deterministic(m):
+    c = _custom(1024, 1024, m, 64, 3)
     r1 = _run_fwd_bwd(c, torch.float32, torch.float32)
     r2 = _run_fwd_bwd(c, torch.float32, torch.float32)
     for u, v in zip(r1, r2):
