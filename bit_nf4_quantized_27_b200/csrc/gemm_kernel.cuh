@@ -30,7 +30,12 @@ struct GemmArgs {
   int M_rows;        // rows of D (tiles of 128 * MT)
   int N_cols;        // cols of D (tiles of BN)
   int k_steps;       // main K steps of 64
-  int hilo;          // 1: a second pass of k_steps reuses A with B taken from tmB2
+  int hilo_cols;     // 1: a tile's B holds BN/2 columns of B (tmB) then the same
+                     //    columns of B2 (tmB2); D columns j and j + BN/2 are summed
+  int ksplit;        // K range split over this many CTAs (non-NF4, no LoRA steps); > 1
+                     // writes raw fp32 partial planes to `part` [ksplit][M_rows][N_cols]
+  float *part;
+  int k_per;         // K steps per split when ksplit > 1 (no split is empty)
   int lora_steps;    // extra K steps of 64 for the LoRA block (0 = none)
   int lora_r;        // LoRA rank (bounds the B2 rows/cols read by the dequant warps)
   // outputs (each optional): `out` (f32 or bf16, scaled by out_scale, optionally
@@ -226,6 +231,41 @@ __device__ __forceinline__ void store_chunk32(const GemmArgs &args, int row, int
   }
 }
 
+// Sums the ksplit fp32 partial planes of a split-K GEMM in plane order and
+// writes the outputs exactly as the GEMM epilogue does (out = v * out_scale;
+// hi = bf16(v * hl_scale), lo = bf16(v * hl_scale - hi)).  Two columns per thread.
+__global__ void splitk_finish_kernel(const GemmArgs args) {
+  const int64_t pairs = (int64_t)args.M_rows * args.N_cols / 2;
+  const int64_t plane = (int64_t)args.M_rows * args.N_cols;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < pairs; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t e = 2 * i;
+    float a = 0.0f, b = 0.0f;
+    for (int sp = 0; sp < args.ksplit; ++sp) {
+      const float2 p = *reinterpret_cast<const float2 *>(args.part + sp * plane + e);
+      a += p.x;
+      b += p.y;
+    }
+    const int64_t row = e / args.N_cols, col = e - row * args.N_cols;
+    if (args.out) {
+      if (args.out_f32) {
+        float *o = reinterpret_cast<float *>(args.out) + row * args.ldo + col;
+        o[0] = a * args.out_scale;
+        o[1] = b * args.out_scale;
+      } else {
+        *reinterpret_cast<uint32_t *>(reinterpret_cast<__nv_bfloat16 *>(args.out) + row * args.ldo + col) =
+            pack_bf16x2(a * args.out_scale, b * args.out_scale);
+      }
+    }
+    if (args.out_hi) {
+      const float x = a * args.hl_scale, y = b * args.hl_scale;
+      const uint32_t h = pack_bf16x2(x, y);
+      const uint32_t l = pack_bf16x2(x - bf16lo_to_f32(h), y - bf16hi_to_f32(h));
+      *reinterpret_cast<uint32_t *>(args.out_hi + row * args.ld_hl + col) = h;
+      *reinterpret_cast<uint32_t *>(args.out_lo + row * args.ld_hl + col) = l;
+    }
+  }
+}
+
 template <bool A_MN, bool B_MN, bool NF4, int BN, int MT>
 __global__ void __launch_bounds__(GemmCfg<A_MN, B_MN, NF4, BN, MT>::THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -268,7 +308,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   if (warp == 0 && lane == 0) {
     ptx::prefetch_tmap(&tmA);
     if (!NF4) ptx::prefetch_tmap(&tmB);
-    if (args.hilo) ptx::prefetch_tmap(&tmB2);
+    if (args.hilo_cols) ptx::prefetch_tmap(&tmB2);
     if (args.lora_steps) ptx::prefetch_tmap(&tmA2);
     if (NF4) ptx::prefetch_tmap(&tmCodes);
   }
@@ -281,15 +321,26 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  const int tile_n = args.hilo_cols ? BN / 2 : BN;  // output columns per tile
   const int num_m = (args.M_rows + C::BM * MT - 1) / (C::BM * MT);
-  const int num_n = (args.N_cols + BN - 1) / BN;
-  const int num_tiles = num_m * num_n;
+  const int num_n = (args.N_cols + tile_n - 1) / tile_n;
+  const int tiles_mn = num_m * num_n;
+  const int ksplit = args.ksplit > 1 ? args.ksplit : 1;
+  const int num_tiles = tiles_mn * ksplit;
   auto tile_of = [&](int w, int &m0, int &n0) {
-    m0 = (w % num_m) * C::BM * MT;
-    n0 = (w / num_m) * BN;
+    const int mn = w % tiles_mn;
+    m0 = (mn % num_m) * C::BM * MT;
+    n0 = (mn / num_m) * tile_n;
   };
-  const int main_steps = args.k_steps * (args.hilo ? 2 : 1);
+  const int main_steps = args.k_steps;
   const int steps = main_steps + args.lora_steps;
+  // K steps [k_begin, k_end) of tile w (its share of the split)
+  const int k_per = ksplit > 1 ? args.k_per : steps;
+  auto k_range = [&](int w, int &kb, int &ke) {
+    const int sp = w / tiles_mn;
+    kb = sp * k_per;
+    ke = min(steps, kb + k_per);
+  };
 
   auto fail = [&]() {
     raise_status(args.status, QLORA_ERR_TIMEOUT);
@@ -303,12 +354,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       int issued_a = 0, issued_c = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        int m0, n0;
+        int m0, n0, kb, ke;
         tile_of(tile, m0, n0);
-        for (int ks = 0; ks < steps && ok; ++ks) {
+        k_range(tile, kb, ke);
+        for (int ks = kb; ks < ke && ok; ++ks) {
           const bool lora = ks >= main_steps;
-          const bool second = !lora && ks >= args.k_steps;  // hi/lo second pass
-          const int kk = second ? ks - args.k_steps : ks;
+          const int kk = ks;
           if (NF4 && !lora) {
             if (!ptx::mbar_wait(&empty_c[sc], pc ^ 1, abort_flag)) { ok = false; break; }
             ptx::mbar_arrive_expect_tx(&full_c[sc], C::C_STAGE);
@@ -332,11 +383,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           }
           if (!NF4) {
             uint8_t *dB = sB + sa * C::B_STAGE;
-            const CUtensorMap *mb = second ? &tmB2 : &tmB;
             if (!B_MN) {
-              ptx::tma_load_2d(dB, mb, &full_a[sa], kk * 64, n0);
-            } else {
-              for (int t = 0; t < BN / 64; ++t) ptx::tma_load_2d(dB + t * 8192, mb, &full_a[sa], n0 + t * 64, kk * 64);
+              ptx::tma_load_2d(dB, &tmB, &full_a[sa], kk * 64, n0);
+            } else if (!args.hilo_cols) {
+              for (int t = 0; t < BN / 64; ++t) ptx::tma_load_2d(dB + t * 8192, &tmB, &full_a[sa], n0 + t * 64, kk * 64);
+            } else {  // columns n0.. of B, then the same columns of B2
+              constexpr int kHalfBlocks = BN >= 128 ? BN / 128 : 1;  // 64-column blocks per half
+              for (int t = 0; t < BN / 64; ++t) {
+                const int h = t / kHalfBlocks;
+                ptx::tma_load_2d(dB + t * 8192, h ? &tmB2 : &tmB, &full_a[sa], n0 + (t % kHalfBlocks) * 64, kk * 64);
+              }
             }
           }
           ++issued_a;
@@ -365,10 +421,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
         const int acc = it % C::NUM_ACC;
         const uint32_t acc_phase = (it / C::NUM_ACC) & 1;
+        int kb, ke;
+        k_range(tile, kb, ke);
         if (!ptx::mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag)) { ok = false; break; }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * C::ACC_COLS;
-        for (int ks = 0; ks < steps && ok; ++ks) {
+        for (int ks = kb; ks < ke && ok; ++ks) {
           const bool lora = ks >= main_steps;
           if (!ptx::mbar_wait(&full_a[sa], pa, abort_flag)) { ok = false; break; }
           if (NF4 && !ptx::mbar_wait(&full_b[sb], pb, abort_flag)) { ok = false; break; }
@@ -385,7 +443,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
               const uint64_t ad = a_mn ? ptx::smem_desc_sw128(a_base + t * 16384 + k16 * 2048, 8192, 1024)
                                        : ptx::smem_desc_sw128(a_base + t * 16384 + k16 * 32, 16, 1024);
               const uint32_t idesc = a_mn ? C::IDESC : (C::IDESC & ~(1u << 15));
-              ptx::mma_bf16(d_tmem + t * BN, ad, bd, idesc, (ks | k16) ? 1u : 0u);
+              ptx::mma_bf16(d_tmem + t * BN, ad, bd, idesc, (ks != kb || k16) ? 1u : 0u);
             }
           }
           ptx::mma_commit(&empty_a[sa]);
@@ -414,14 +472,33 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       ptx::tc_fence_after();
       int m0, n0;
       tile_of(tile, m0, n0);
+      const int sp = tile / tiles_mn;
       for (int t = 0; t < MT; ++t) {
         const int row = m0 + t * 128 + q * 32 + lane;
-        for (int cb = 0; cb < BN; cb += 32) {
+        for (int cb = 0; cb < tile_n; cb += 32) {
           uint32_t v[32];
-          ptx::tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS + t * BN + cb, v);
+          const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * C::ACC_COLS + t * BN + cb;
+          ptx::tmem_ld32(taddr, v);
           ptx::tmem_ld_wait();
+          if (args.hilo_cols) {  // add the B2 half of the tile
+            uint32_t w2[32];
+            ptx::tmem_ld32(taddr + BN / 2, w2);
+            ptx::tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(w2[j]));
+          }
           const int col0 = n0 + cb;
-          if (row < args.M_rows && col0 < args.N_cols) store_chunk32(args, row, col0, min(32, args.N_cols - col0), v);
+          if (row < args.M_rows && col0 < args.N_cols) {
+            if (ksplit > 1) {  // raw fp32 partial of this K share
+              float *o = args.part + ((int64_t)sp * args.M_rows + row) * args.N_cols + col0;
+              const int nc = min(32, args.N_cols - col0);
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (j < nc) o[j] = __uint_as_float(v[j]);
+            } else {
+              store_chunk32(args, row, col0, min(32, args.N_cols - col0), v);
+            }
+          }
         }
       }
       ptx::tc_fence_before();

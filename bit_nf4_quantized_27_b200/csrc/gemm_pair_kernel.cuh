@@ -109,13 +109,29 @@ gemm_nf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  // Tiles of 2*128*MT tokens x 256 columns, handed out round-robin to the
+  // clusters.  When the last round would leave at least half of the clusters
+  // idle, its tiles are split into halves of 256 tokens (one accumulator), so
+  // the last round takes half as long.
   const int num_m = (args.M_rows + 2 * C::BM * MT - 1) / (2 * C::BM * MT);
   const int num_n = (args.N_cols + C::BN - 1) / C::BN;
-  const int num_tiles = num_m * num_n;
   const int cluster = blockIdx.x >> 1, clusters = gridDim.x >> 1;
-  auto tile_of = [&](int w, int &m0, int &n0) {
-    m0 = (w % num_m) * 2 * C::BM * MT;
-    n0 = (w / num_m) * C::BN;
+  const int full_tiles = num_m * num_n;
+  const int rem = full_tiles % clusters;
+  const bool split = MT == 2 && rem > 0 && 2 * rem <= clusters;
+  const int main_tiles = split ? full_tiles - rem : full_tiles;
+  const int num_tiles = split ? main_tiles + 2 * rem : full_tiles;
+  auto tile_of = [&](int w, int &m0, int &n0, int &mt) {
+    if (w < main_tiles) {
+      m0 = (w % num_m) * 2 * C::BM * MT;
+      n0 = (w / num_m) * C::BN;
+      mt = MT;
+    } else {
+      const int f = main_tiles + ((w - main_tiles) >> 1);
+      m0 = (f % num_m) * 2 * C::BM * MT + 2 * C::BM * ((w - main_tiles) & 1);
+      n0 = (f / num_m) * C::BN;
+      mt = 1;
+    }
   };
   const int steps = args.k_steps + args.lora_steps;
   // operand row unit e (0..127) -> (W row offset wr, 64-feature block fb): fwd
@@ -144,8 +160,8 @@ gemm_nf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       int issued_a = 0, issued_c = 0;
       bool ok = true;
       for (int tile = cluster; tile < num_tiles && ok; tile += clusters) {
-        int m0, n0;
-        tile_of(tile, m0, n0);
+        int m0, n0, mt;
+        tile_of(tile, m0, n0, mt);
         const int nh = n0 + C::HB * static_cast<int>(rank);  // this CTA's first weight-operand row
         for (int ks = 0; ks < steps && ok; ++ks) {
           const bool lora = ks >= args.k_steps;
@@ -160,10 +176,10 @@ gemm_nf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
           }
           // empty_a is released by the even CTA's MMA commit, in both CTAs
           if (!ptx::mbar_wait(&empty_a[sa], pa ^ 1, abort_flag)) { ok = false; break; }
-          if (even) ptx::mbar_arrive_expect_tx(&full_a[sa], 2 * C::A_STAGE);
+          if (even) ptx::mbar_arrive_expect_tx(&full_a[sa], 2 * mt * C::BM * C::BK * 2);
           const uint32_t bar = ptx::mapa_shared(ptx::smem_addr(&full_a[sa]), 0);
           uint8_t *dA = sA + sa * C::A_STAGE;
-          for (int t = 0; t < MT; ++t) {
+          for (int t = 0; t < mt; ++t) {
             const int row = m0 + t * 2 * C::BM + C::BM * static_cast<int>(rank);
             if (lora) ptx::tma_load_2d_pair(dA + t * 16384, &tmA2, bar, (ks - args.k_steps) * 64, row);
             else ptx::tma_load_2d_pair(dA + t * 16384, &tmA, bar, ks * 64, row);
@@ -194,6 +210,8 @@ gemm_nf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       bool ok = true;
       const uint32_t sA0 = ptx::smem_addr(sA), sB0 = ptx::smem_addr(sB);
       for (int tile = cluster; tile < num_tiles && ok; tile += clusters, ++it) {
+        int m0_, n0_, mt;
+        tile_of(tile, m0_, n0_, mt);
         if (!ptx::mbar_wait(acc_empty, (it & 1) ^ 1, abort_flag)) { ok = false; break; }
         ptx::tc_fence_after();
         for (int ks = 0; ks < steps && ok; ++ks) {
@@ -208,6 +226,7 @@ gemm_nf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                                      : ptx::smem_desc_sw128(b_base + k16 * 32, 16, 1024);
 #pragma unroll
             for (int t = 0; t < MT; ++t) {
+              if (t >= mt) break;
               const uint64_t ad = ptx::smem_desc_sw128(a_base + t * 16384 + k16 * 32, 16, 1024);
               ptx::mma_bf16_pair(tmem_base + t * C::BN, ad, bd, C::IDESC, (ks | k16) ? 1u : 0u);
             }
@@ -235,9 +254,9 @@ gemm_nf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         break;
       }
       ptx::tc_fence_after();
-      int m0, n0;
-      tile_of(tile, m0, n0);
-      for (int t = 0; t < MT; ++t) {
+      int m0, n0, mt;
+      tile_of(tile, m0, n0, mt);
+      for (int t = 0; t < mt; ++t) {
         const int row = m0 + t * 2 * C::BM + C::BM * static_cast<int>(rank) + q * 32 + lane;
         for (int cb = 0; cb < C::BN; cb += 32) {
           uint32_t v[32];
@@ -280,8 +299,8 @@ gemm_nf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     bool ok = true;
     auto produce = [&]() -> bool {
       const bool lora = ks >= args.k_steps;
-      int m0_, n0;
-      tile_of(tile, m0_, n0);
+      int m0_, n0, mt_;
+      tile_of(tile, m0_, n0, mt_);
       const int nh = n0 + C::HB * static_cast<int>(rank);
       const uint32_t sb = static_cast<uint32_t>(u % C::SB), pb = static_cast<uint32_t>((u / C::SB) & 1);
       uint32_t o[32];
@@ -346,8 +365,8 @@ gemm_nf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     int tile = cluster, ks = 0, cu = 0;
     bool ok = true;
     auto index_of = [&](int ti, int k, int wr, int fb) -> int64_t {  // flat block index, -1 = none
-      int m0_, n0;
-      tile_of(ti, m0_, n0);
+      int m0_, n0, mt_;
+      tile_of(ti, m0_, n0, mt_);
       const int nh = n0 + C::HB * static_cast<int>(rank);
       int64_t wrow, kblk;
       if (!B_MN) { wrow = nh + wr; kblk = k; }

@@ -149,9 +149,10 @@ qlora_status launch_gemm(const CUtensorMap &tmA, const CUtensorMap &tmB, const C
   static qlora_status results[64];
   qlora_status s = set_smem(kernel, C::SMEM_BYTES, dev, flags, results);
   if (s != QLORA_OK) return s;
+  const int tile_n = args.hilo_cols ? BN / 2 : BN;
   const int num_m = (args.M_rows + C::BM * MT - 1) / (C::BM * MT);
-  const int num_n = (args.N_cols + BN - 1) / BN;
-  const int tiles = num_m * num_n;
+  const int num_n = (args.N_cols + tile_n - 1) / tile_n;
+  const int tiles = num_m * num_n * std::max(1, args.ksplit);
   const int grid = std::max(1, std::min(tiles, sms));
   kernel<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tmA, tmB, tmA2, tmB2, tmCodes, args);
   return launch_status();
@@ -173,8 +174,36 @@ bool valid_dtype(qlora_dtype d) { return d == QLORA_F32 || d == QLORA_BF16; }
 
 // T = X A^T for the tokens: writes s*T (bf16) to sT (if not null) and, if T_hi is
 // not null, T as the bf16 pair (T_hi, T_lo) with T_hi + T_lo = T to ~16 bits.
+// Rank-r GEMMs (T = X A^T, U = dY B): output tiles are few (M / 128), so when
+// the caller's workspace holds the partial planes the K range is split over up
+// to kMaxSplit CTAs per tile and the fp32 partials are summed, in split order,
+// by splitk_finish_kernel.
+constexpr int kMaxSplit = 8;
+inline size_t split_part_bytes(int64_t M, int32_t r) {
+  return align256(static_cast<size_t>(kMaxSplit) * static_cast<size_t>(M) * r * 4);
+}
+template <bool B_MN>
+qlora_status launch_rank_gemm(const CUtensorMap &tmA, const CUtensorMap &tmB, GemmArgs g, float *part, int dev,
+                              int sms, cudaStream_t st) {
+  const int tiles = ((g.M_rows + 127) / 128) * ((g.N_cols + 63) / 64);
+  int ks = part ? std::min(kMaxSplit, std::min(sms / std::max(1, tiles), g.k_steps / 4)) : 1;
+  if (ks > 1) {
+    g.k_per = (g.k_steps + ks - 1) / ks;
+    ks = (g.k_steps + g.k_per - 1) / g.k_per;  // every split gets at least one step
+  }
+  if (ks <= 1) return launch_gemm<false, B_MN, false, 64, 1>(tmA, tmB, tmA, tmA, tmA, g, dev, sms, st);
+  g.ksplit = ks;
+  g.part = part;
+  qlora_status s = launch_gemm<false, B_MN, false, 64, 1>(tmA, tmB, tmA, tmA, tmA, g, dev, sms, st);
+  if (s != QLORA_OK) return s;
+  const int64_t pairs = (int64_t)g.M_rows * g.N_cols / 2;
+  const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>((pairs + 255) / 256, (int64_t)sms * 8));
+  splitk_finish_kernel<<<grid, 256, 0, st>>>(g);
+  return launch_status();
+}
+
 qlora_status run_lora_down(const void *X, const qlora_lora *ad, int64_t M, int64_t K, float s, void *sT,
-                           void *T_hi, void *T_lo, uint32_t *status, int dev, int sms, cudaStream_t st) {
+                           void *T_hi, void *T_lo, float *part, uint32_t *status, int dev, int sms, cudaStream_t st) {
   CUtensorMap tmX, tmA;
   if (!tmap_bf16(&tmX, X, K, M, 64, 128) || !tmap_bf16(&tmA, ad->A, K, ad->r, 64, 64)) return QLORA_ERR_CUDA;
   GemmArgs g{};
@@ -190,9 +219,30 @@ qlora_status run_lora_down(const void *X, const qlora_lora *ad, int64_t M, int64
   g.ld_hl = ad->r;
   g.hl_scale = 1.0f;
   g.status = status;
-  return launch_gemm<false, false, false, 64, 1>(tmX, tmA, tmX, tmX, tmX, g, dev, sms, st);
+  return launch_rank_gemm<false>(tmX, tmA, g, part, dev, sms, st);
 }
 
+// Least workspace the entry points accept (no K splitting of the rank-r GEMMs).
+size_t min_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r, int for_backward) {
+  if (M <= 0 || N <= 0 || K <= 0 || r <= 0 || r > QLORA_MAX_RANK) return 0;
+  const size_t mr = align256(static_cast<size_t>(M) * r * 2);  // one bf16 [M, r] buffer
+  size_t bytes = QLORA_STATUS_BYTES;
+  if (!for_backward) {
+    bytes += mr;                                    // s*T
+    if (M <= kGemvMaxM) bytes += gemv_workspace_bytes(M, N, K);
+  } else {
+    bytes += 4 * mr;                                // s*U (hi, lo), recomputed T (hi, lo)
+  }
+  return bytes;
+}
+// Partial planes for K splitting, placed after the minimum workspace when the
+// caller passed room for them.
+float *split_part(void *ws, size_t ws_bytes, int64_t M, int64_t N, int64_t K, int32_t r, int for_backward) {
+  if (!for_backward && M <= kGemvMaxM) return nullptr;
+  const size_t lo = min_workspace_bytes(M, N, K, r, for_backward);
+  if (ws_bytes < lo + split_part_bytes(M, r)) return nullptr;
+  return reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + lo);
+}
 }  // namespace
 
 extern "C" {
@@ -218,16 +268,10 @@ size_t qlora_nf4_storage_bytes(int64_t rows, int64_t cols, size_t *codes_bytes, 
 }
 
 size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r, int for_backward) {
-  if (M <= 0 || N <= 0 || K <= 0 || r <= 0 || r > QLORA_MAX_RANK) return 0;
-  const size_t mr = align256(static_cast<size_t>(M) * r * 2);  // one bf16 [M, r] buffer
-  size_t bytes = QLORA_STATUS_BYTES;
-  if (!for_backward) {
-    bytes += mr;                                    // s*T
-    if (M <= kGemvMaxM) bytes += gemv_workspace_bytes(M, N, K);
-  } else {
-    bytes += 4 * mr;                                // s*U (hi, lo), recomputed T (hi, lo)
-  }
-  return bytes;
+  const size_t lo = min_workspace_bytes(M, N, K, r, for_backward);
+  if (lo == 0) return 0;
+  if (!for_backward && M <= kGemvMaxM) return lo;
+  return lo + split_part_bytes(M, r);
 }
 
 qlora_status qlora_nf4_quantize(const void *W, qlora_dtype w_dtype, const qlora_nf4_tensor *out, void *ws,
@@ -289,7 +333,7 @@ qlora_status qlora_linear_fwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
   if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(ws, 256) || (T_save && !aligned(T_save, 16)))
     return QLORA_ERR_MISALIGNED;
   const int64_t N = W->rows, K = W->cols;
-  if (ws_bytes < qlora_workspace_bytes(M, N, K, ad->r, 0)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  if (ws_bytes < min_workspace_bytes(M, N, K, ad->r, 0)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   int dev, sms;
   if ((s = check_device(&dev, &sms)) != QLORA_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -324,7 +368,8 @@ qlora_status qlora_linear_fwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
 
   {
     __nv_bfloat16 *th = static_cast<__nv_bfloat16 *>(T_save);
-    if ((s = run_lora_down(X, ad, M, K, sc, sT, th, th ? th + M * ad->r : nullptr, status_ptr(ws), dev, sms, st)) !=
+    if ((s = run_lora_down(X, ad, M, K, sc, sT, th, th ? th + M * ad->r : nullptr,
+                           split_part(ws, ws_bytes, M, N, K, ad->r, 0), status_ptr(ws), dev, sms, st)) !=
         QLORA_OK)
       return s;
   }
@@ -371,7 +416,7 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
       !aligned(ws, 256) || (T_saved && !aligned(T_saved, 16)))
     return QLORA_ERR_MISALIGNED;
   const int64_t N = W->rows, K = W->cols;
-  if (ws_bytes < qlora_workspace_bytes(M, N, K, ad->r, 1)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  if (ws_bytes < min_workspace_bytes(M, N, K, ad->r, 1)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   int dev, sms;
   if ((s = check_device(&dev, &sms)) != QLORA_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -382,12 +427,13 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
   void *sU_hi = wsb + QLORA_STATUS_BYTES;
   void *sU_lo = wsb + QLORA_STATUS_BYTES + mr;
   uint32_t *status = status_ptr(ws);
+  float *part = split_part(ws, ws_bytes, M, N, K, r, 1);
 
   const void *T_hi = T_saved;
   const void *T_lo = T_saved ? static_cast<const __nv_bfloat16 *>(T_saved) + M * r : nullptr;
   if (!T_saved) {
     void *th = wsb + QLORA_STATUS_BYTES + 2 * mr, *tl = wsb + QLORA_STATUS_BYTES + 3 * mr;
-    if ((s = run_lora_down(X, ad, M, K, sc, nullptr, th, tl, status, dev, sms, st)) != QLORA_OK) return s;
+    if ((s = run_lora_down(X, ad, M, K, sc, nullptr, th, tl, part, status, dev, sms, st)) != QLORA_OK) return s;
     T_hi = th;
     T_lo = tl;
   }
@@ -404,8 +450,7 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
     g.ld_hl = r;
     g.hl_scale = sc;
     g.status = status;
-    if ((s = launch_gemm<false, true, false, 64, 1>(tmDY, tmB, tmDY, tmDY, tmDY, g, dev, sms, st)) != QLORA_OK)
-      return s;
+    if ((s = launch_rank_gemm<true>(tmDY, tmB, g, part, dev, sms, st)) != QLORA_OK) return s;
   }
   // dX = dY W' + (s U) A
   {
@@ -447,14 +492,14 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
     g.M_rows = (int)K;
     g.N_cols = r;
     g.k_steps = (int)((M + 63) / 64);
-    g.hilo = 1;
+    g.hilo_cols = 1;
     g.out = dA;
     g.ldo = K;
     g.out_f32 = grad_dtype == QLORA_F32;
     g.out_transpose = 1;
     g.out_scale = 1.0f;
     g.status = status;
-    if ((s = launch_gemm<true, true, false, 64, 1>(tmXt, tmUh, tmXt, tmUl, tmXt, g, dev, sms, st)) != QLORA_OK)
+    if ((s = launch_gemm<true, true, false, 128, 1>(tmXt, tmUh, tmXt, tmUl, tmXt, g, dev, sms, st)) != QLORA_OK)
       return s;
   }
   // dB [N, r] = s dY^T (T_hi + T_lo)
@@ -467,13 +512,13 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
     g.M_rows = (int)N;
     g.N_cols = r;
     g.k_steps = (int)((M + 63) / 64);
-    g.hilo = 1;
+    g.hilo_cols = 1;
     g.out = dB;
     g.ldo = r;
     g.out_f32 = grad_dtype == QLORA_F32;
     g.out_scale = sc;
     g.status = status;
-    if ((s = launch_gemm<true, true, false, 64, 1>(tmDYt, tmTh, tmDYt, tmTl, tmDYt, g, dev, sms, st)) != QLORA_OK)
+    if ((s = launch_gemm<true, true, false, 128, 1>(tmDYt, tmTh, tmDYt, tmTl, tmDYt, g, dev, sms, st)) != QLORA_OK)
       return s;
   }
   return QLORA_OK;
@@ -513,7 +558,7 @@ qlora_status qlora_linear_fwd_noalloc(const qlora_nf4_tensor *W, const qlora_lor
   if (s != QLORA_OK) return s;
   if ((s = check_lora(adapter)) != QLORA_OK) return s;
   if (M < 1) return QLORA_ERR_INVALID_ARGUMENT;
-  const size_t need = qlora_workspace_bytes(M, W->rows, W->cols, adapter->r, 0);
+  const size_t need = min_workspace_bytes(M, W->rows, W->cols, adapter->r, 0);
   if (need == 0) return QLORA_ERR_INVALID_ARGUMENT;
   if (need > QLORA_NOALLOC_SCRATCH_BYTES) return QLORA_ERR_UNSUPPORTED_SHAPE;
   int dev, sms;

@@ -32,7 +32,7 @@
  *     be 16-byte aligned; ws must be 256-byte aligned.
  *   - The library never allocates, frees or synchronises (except
  *     qlora_read_status, which synchronises the stream it is given).  All scratch
- *     comes from the caller's workspace ws of at least qlora_workspace_bytes().
+ *     comes from the caller's workspace ws (qlora_workspace_bytes() tells how much).
  *     The first QLORA_STATUS_BYTES of ws hold a device status word.
  *   - Argument checks run on the host before any launch; a failed check returns an
  *     error code and launches nothing.  A failed launch returns QLORA_ERR_CUDA.
@@ -114,9 +114,14 @@ QLORA_API void qlora_nf4_codebook(float out[16]);
 QLORA_API size_t qlora_nf4_storage_bytes(int64_t rows, int64_t cols, size_t *codes_bytes,
                                size_t *scale_codes_bytes, size_t *c2_bytes);
 
-/* Workspace bytes needed by qlora_linear_fwd (for_backward = 0) or
- * qlora_linear_bwd (for_backward = 1) for M tokens, W [N, K] and rank r;
- * at least QLORA_STATUS_BYTES.  0 for invalid sizes. */
+/* Workspace bytes for qlora_linear_fwd (for_backward = 0) or qlora_linear_bwd
+ * (for_backward = 1) with M tokens, W [N, K] and rank r; 0 for invalid sizes.
+ * The entry points also accept less, down to QLORA_STATUS_BYTES + (256-byte
+ * rounded) M*r*2 bytes for the forward and QLORA_STATUS_BYTES + 4 * that for the
+ * backward (QLORA_ERR_WORKSPACE_TOO_SMALL below it); the size returned here adds
+ * fp32 partial planes that let the rank-r GEMMs (X A^T, dY B) split their K
+ * range over more CTAs when M > 16.  Results are the same either way to within
+ * float32 rounding order. */
 QLORA_API size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r, int for_backward);
 
 /* Quantise W [out->rows, out->cols] (float32 or bf16, row-major, device) to NF4

@@ -160,6 +160,32 @@ def test_cta_pair_path_ragged(n, k, m, r):
         _check_all(c, *_run_fwd_bwd(c, dt, dt))
 
 
+@pytest.mark.parametrize("n,k,m", [(20480, 256, 512), (256, 20480, 512), (10240, 320, 600)])
+def test_cta_pair_last_round_split(n, k, m):
+    # more 512-token tiles than resident CTA pairs, with a short last round: its
+    # tiles run as 256-token halves (forward: N = 20480 or 10240; dX: K = 20480)
+    c = _custom(n, k, m, 16, 3 * n + k + m)
+    _check_all(c, *_run_fwd_bwd(c, torch.float32, torch.float32))
+
+
+@pytest.mark.parametrize("n,k,m,r", [(1024, 1024, 512, 64), (512, 2048, 300, 16), (640, 4096, 2048, 128)])
+def test_minimum_workspace_without_k_split(n, k, m, r):
+    # the least workspace the entry points accept runs the rank-r GEMMs (X A^T,
+    # dY B) without splitting K; the reported size splits K over more CTAs
+    c = _custom(n, k, m, r, 5 * n + m)
+    qg, a, b, x, dy = c.gpu()
+    mr = (m * r * 2 + 255) // 256 * 256
+    assert bd.workspace_bytes(m, n, k, r, False) > 256 + mr
+    for fw, bw in ((256 + mr, 256 + 4 * mr), (None, None)):
+        wsf = bd.new_workspace(fw) if fw else None
+        wsb = bd.new_workspace(bw) if bw else None
+        y, t = bd.linear_fwd(qg, a, b, c.alpha, x, y_dtype=torch.float32, ws=wsf)
+        dx, da, db = bd.linear_bwd(qg, a, b, c.alpha, x, dy, t, dx_dtype=torch.float32, grad_dtype=torch.float32,
+                                   ws=wsb)
+        torch.cuda.synchronize()
+        _check_all(c, y, t, dx, da, db)
+
+
 @pytest.mark.parametrize("m", [4, 300])
 def test_b_zero_is_base_layer(m):
     c = _custom(512, 512, m, 64, 77, b_std=0.0)
