@@ -48,9 +48,10 @@ def load_peaks():
 # captures of the `cases` module's fwd_8192 / fwd_65b_up / fwd_65b_down.  The
 # figure belongs to the kernel sources it was measured on: it is reported only
 # while their digest still matches, else the traffic is null.
-FUSED_FWD_TRAFFIC_BYTES = 570.06e6
-FUSED_FWD_TRAFFIC_SOURCES = ("gemm_kernel.cuh", "sm100_ptx.cuh", "nf4_device.cuh", "qlora_nf4.cu")
-FUSED_FWD_TRAFFIC_DIGEST = "13f814ae0971338c"
+FUSED_FWD_TRAFFIC_BYTES = 594.85e6
+FUSED_FWD_TRAFFIC_SOURCES = ("gemm_pair_kernel.cuh", "gemm_kernel.cuh", "sm100_ptx.cuh", "nf4_device.cuh",
+                             "qlora_nf4.cu")
+FUSED_FWD_TRAFFIC_DIGEST = "36cb0a8f8fc5a857"
 
 
 def fused_fwd_traffic():
@@ -493,17 +494,22 @@ def main():
 
     fwd_tf = fl_f / (t_fwd * 1e-3) / 1e12
     bwd_tf = fl_b / (t_bwd * 1e-3) / 1e12
-    peak_tc = peaks["bf16_tflops_sustained"]
+    # The timed region is about 0.1 s with SM clocks at their maximum (see
+    # `clocks`), the conditions of the burst measurement; the sustained figure
+    # (a seconds-long loop that settled near 1.3 GHz) is reported beside it.
+    peak_tc = peaks["bf16_tflops"]
+    peak_sus = peaks["bf16_tflops_sustained"]
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(),
-        "roofline": {"bound": "tensor", "kernel": "NF4 fused tensor-core GEMM, forward call (T = X A^T + fused "
-                                                  "dequant GEMM with the LoRA K steps), all 7 layers",
+        "roofline": {"bound": "tensor", "kernel": "NF4 fused tensor-core GEMM on CTA pairs, forward call (T = X A^T "
+                                                  "with split K, then the fused dequant GEMM with the LoRA K steps), "
+                                                  "all 7 layers",
                      "achieved": fwd_tf, "peak": peak_tc, "unit": "TFLOP/s", "frac": fwd_tf / peak_tc,
                      "traffic": fused_fwd_traffic(), "traffic_unit": "bytes per fused forward launch",
-                     "peak_kind": f"{peaks_kind} bf16 dense, sustained",
-                     "step_frac": value / world / peak_tc},
+                     "peak_kind": f"{peaks_kind} bf16 dense, burst",
+                     "frac_of_sustained": fwd_tf / peak_sus, "step_frac": value / world / peak_tc},
         "breakdown_ms_per_step": {"quantize": t_q, "forward": t_fwd, "backward": t_bwd,
                                   "forward_TFLOP/s": fwd_tf, "backward_TFLOP/s": bwd_tf},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
