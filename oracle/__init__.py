@@ -38,4 +38,6 @@ from .nf4_oracle import (  # noqa: F401
     linear_fwd,
     linear_bwd,
     merged_weight,
+    merge_export,
+    adamw_step,
 )

@@ -38,6 +38,11 @@ Readings where the pages are silent or loose (each also listed in the design doc):
   256 blocks run over the flat block index and may span rows; packed byte i holds
   element 2i in its low nibble and element 2i+1 in its high nibble.
 * LoRA scale s = fl32(alpha) / fl32(r); y = X W'^T + s (X A^T) B^T.
+* Merged export: the 16-bit weight a page says merging needs is bf16, the
+  round-to-nearest-even of the exact W' + s B A (one rounding).
+* Adapter optimiser: the pages name Adam's per-parameter momentum and variance
+  but give no update rule; the step is decoupled-weight-decay Adam (AdamW,
+  Loshchilov and Hutter) with bias correction, the form torch.optim.AdamW uses.
 """
 
 from __future__ import annotations
@@ -357,3 +362,35 @@ def merged_weight(w_dq: np.ndarray, a: np.ndarray, b: np.ndarray, alpha: float, 
     """W' + s B A (float64): the merged deployment form [IBM; EZ, Delta W = B A]."""
     s = lora_scale(alpha, r)
     return np.asarray(w_dq, np.float64) + s * (np.asarray(b, np.float64) @ np.asarray(a, np.float64))
+
+
+def merge_export(codes: np.ndarray, scale_codes: np.ndarray, c2: np.ndarray, rows: int, cols: int,
+                 a: np.ndarray, b: np.ndarray, alpha: float, r: int) -> np.ndarray:
+    """The merged 16-bit weight, as float32 values of bf16: bf16_rne(W' + s B A).
+
+    [UL] "Trade-offs": merging the adapters into the base model first needs the
+    base dequantised to 16 bit; [IBM]: the trained low-rank update is merged into
+    the frozen weights for deployment.  W' + s B A is summed exactly (float64)
+    and rounded to bf16 once.
+    """
+    wd = dequantize(codes, scale_codes, c2, rows, cols)
+    return bf16_round(merged_weight(wd, a, b, alpha, r))
+
+
+def adamw_step(p: np.ndarray, g: np.ndarray, m: np.ndarray, v: np.ndarray, step: int, lr: float,
+               beta1: float, beta2: float, eps: float, weight_decay: float):
+    """One AdamW step on float64 copies; returns (p, m, v) after step number `step` (1-based).
+
+    m = beta1 m + (1 - beta1) g;  v = beta2 v + (1 - beta2) g^2;
+    p = p (1 - lr wd) - (lr / (1 - beta1^t)) m / (sqrt(v) / sqrt(1 - beta2^t) + eps).
+    [UL] "How QLoRA works": only the LoRA matrices are updated; [VN] "Paged
+    Optimizers": Adam keeps momentum and variance for every trained parameter.
+    """
+    p = np.asarray(p, np.float64)
+    g = np.asarray(g, np.float64)
+    m = beta1 * np.asarray(m, np.float64) + (1.0 - beta1) * g
+    v = beta2 * np.asarray(v, np.float64) + (1.0 - beta2) * g * g
+    bc1 = 1.0 - beta1 ** step
+    bc2 = 1.0 - beta2 ** step
+    p = p * (1.0 - lr * weight_decay) - (lr / bc1) * m / (np.sqrt(v) / math.sqrt(bc2) + eps)
+    return p, m, v

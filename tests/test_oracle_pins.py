@@ -442,3 +442,95 @@ def test_lora_scale_float32():
     assert O.lora_scale(16.0, 8) == 2.0
     assert O.lora_scale(16.0, 64) == 0.25
     assert O.lora_scale(1.0, 3) == float(np.float32(1.0) / np.float32(3.0))
+
+
+# ---------------------------------------------------------------------------
+# Merged export and the adapter optimiser step
+# ---------------------------------------------------------------------------
+def _quantised(n, k, seed, scale=0.02):
+    rng = np.random.default_rng(seed)
+    w = (rng.standard_normal((n, k)) * scale).astype(np.float32)
+    q = O.quantize(w, n, k)
+    return q, O.dequantize(q["codes"], q["scale_codes"], q["c2"], n, k)
+
+
+def test_merge_export_with_b_zero_is_the_dequantised_weight():
+    q, wd = _quantised(24, 128, 11)
+    a = np.random.default_rng(1).standard_normal((8, 128)).astype(np.float32)
+    got = O.merge_export(q["codes"], q["scale_codes"], q["c2"], 24, 128, a, np.zeros((24, 8), np.float32), 16.0, 8)
+    assert np.array_equal(got.view(np.uint32), wd.astype(np.float32).view(np.uint32))
+
+
+def test_merge_export_with_w_zero_is_one_bf16_rounding_of_the_update():
+    # integer-valued B and A small enough that s B A is exact in float32, so the
+    # float32 -> bf16 cast of torch (round to nearest even) is the reference
+    n, k, r = 16, 64, 8
+    rng = np.random.default_rng(2)
+    a = rng.integers(-300, 300, (r, k)).astype(np.float32)
+    b = rng.integers(-300, 300, (n, r)).astype(np.float32)
+    q = O.quantize(np.zeros((n, k), np.float32), n, k)
+    got = O.merge_export(q["codes"], q["scale_codes"], q["c2"], n, k, a, b, 16.0, r)
+    exact = (2.0 * (b.astype(np.float64) @ a.astype(np.float64))).astype(np.float32)
+    assert np.array_equal(exact.astype(np.float64), 2.0 * (b.astype(np.float64) @ a.astype(np.float64)))
+    want = torch.from_numpy(exact).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(got, want)
+    assert np.any(got != exact)  # the rounding is exercised
+
+
+def test_merged_export_reproduces_the_layer_forward():
+    q, wd = _quantised(32, 192, 3)
+    rng = np.random.default_rng(4)
+    a = (rng.standard_normal((8, 192)) / math.sqrt(192)).astype(np.float32)
+    b = (rng.standard_normal((32, 8)) * 0.01).astype(np.float32)
+    x = rng.standard_normal((5, 192)).astype(np.float32)
+    wm = O.merge_export(q["codes"], q["scale_codes"], q["c2"], 32, 192, a, b, 16.0, 8)
+    y, _ = O.linear_fwd(wd, a, b, x, 16.0, 8)
+    ym = x.astype(np.float64) @ wm.astype(np.float64).T
+    # the only difference is the merged weight's own bf16 rounding (2^-9 relative)
+    assert np.max(np.abs(ym - y)) <= 2.0 ** -8 * np.sqrt(np.sum(x.astype(np.float64) ** 2, axis=1)).max() * \
+        np.abs(wm).max()
+
+
+def _adamw_torch(p0, grads, lr, b1, b2, eps, wd):
+    p = torch.nn.Parameter(torch.from_numpy(p0.copy()))
+    opt = torch.optim.AdamW([p], lr=lr, betas=(b1, b2), eps=eps, weight_decay=wd)
+    for g in grads:
+        p.grad = torch.from_numpy(g.copy())
+        opt.step()
+    st = opt.state[p]
+    return p.detach().numpy(), st["exp_avg"].numpy(), st["exp_avg_sq"].numpy()
+
+
+def test_adamw_step_matches_torch_adamw_over_several_steps():
+    rng = np.random.default_rng(5)
+    p0 = rng.standard_normal(257)
+    grads = [rng.standard_normal(257) * (0.1 + i) for i in range(6)]
+    hp = dict(lr=3e-3, beta1=0.9, beta2=0.97, eps=1e-7, weight_decay=0.05)
+    p, m, v = p0, np.zeros_like(p0), np.zeros_like(p0)
+    for t, g in enumerate(grads, start=1):
+        p, m, v = O.adamw_step(p, g, m, v, t, **hp)
+    tp, tm, tv = _adamw_torch(p0, grads, hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"])
+    assert np.allclose(p, tp, rtol=1e-12, atol=1e-14)
+    assert np.allclose(m, tm, rtol=1e-12, atol=1e-14)
+    assert np.allclose(v, tv, rtol=1e-12, atol=1e-14)
+
+
+def test_adamw_step_closed_forms():
+    rng = np.random.default_rng(6)
+    p0 = rng.standard_normal(64)
+    # zero gradient and zero state: only the decoupled decay acts
+    p, m, v = O.adamw_step(p0, np.zeros(64), np.zeros(64), np.zeros(64), 1, 1e-2, 0.9, 0.999, 1e-8, 0.1)
+    assert np.array_equal(p, p0 * (1.0 - 1e-3)) and not m.any() and not v.any()
+    # first step without decay: the bias corrections cancel, the step is lr g / (|g| + eps)
+    g = rng.standard_normal(64)
+    p, _, _ = O.adamw_step(p0, g, np.zeros(64), np.zeros(64), 1, 1e-2, 0.9, 0.999, 1e-8, 0.0)
+    assert np.allclose(p, p0 - 1e-2 * g / (np.abs(g) + 1e-8), rtol=1e-14, atol=1e-16)
+
+
+def test_adamw_pin_catches_a_planted_sign_error():
+    rng = np.random.default_rng(7)
+    p0, g = rng.standard_normal(32), rng.standard_normal(32)
+    good, _, _ = O.adamw_step(p0, g, np.zeros(32), np.zeros(32), 1, 1e-2, 0.9, 0.999, 1e-8, 0.0)
+    bad = p0 + 1e-2 * g / (np.abs(g) + 1e-8)  # the update applied with the wrong sign
+    tp, _, _ = _adamw_torch(p0, [g], 1e-2, 0.9, 0.999, 1e-8, 0.0)
+    assert np.allclose(good, tp) and not np.allclose(bad, tp)
