@@ -377,6 +377,59 @@ def sub_quant(device, peaks):
     return res
 
 
+def sub_adapters(device, peaks):
+    """The steps after backward: merged export of an 8192x8192 NF4 weight with
+    an r = 64 adapter (CUDA graph over 4 weight copies), and one AdamW step over
+    the 65B-shaped block's adapters (flat fp32 with the bf16 copy).  GB/s of
+    algorithmic bytes against the measured HBM copy bandwidth."""
+    import torch
+
+    from bit_nf4_quantized_27_b200 import binding as bd
+
+    res = {}
+    n = k = 8192
+    r = 64
+    copies = 4
+    qs = []
+    for _ in range(copies):
+        w = (torch.randn(n, k, device=device) * 0.02).to(torch.bfloat16)
+        qs.append(bd.quantize(w))
+        del w
+    a = (torch.randn(r, k, device=device) / k ** 0.5).to(torch.bfloat16)
+    b = (torch.randn(n, r, device=device) * 0.01).to(torch.bfloat16)
+    outs = [torch.empty(n, k, dtype=torch.bfloat16, device=device) for _ in range(copies)]
+    for i in range(copies):
+        bd.merge(qs[i], a, b, 16.0, out=outs[i])
+    torch.cuda.synchronize()
+    reps = 2 * copies
+    us = graph_time_us(lambda: [bd.merge(qs[i % copies], a, b, 16.0, out=outs[i % copies]) for i in range(reps)]) / reps
+    nbytes = n * k * 2 + n * k // 2 + n * k // 64 + 4 * (n * k // 64 // 256) + 2 * r * (n + k)
+    res["merge_8192x8192_r64"] = {"us": us, "GB/s": nbytes / (us * 1e-6) / 1e9,
+                                  "frac_of_hbm": nbytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"],
+                                  "tensor_TFLOP/s": 2 * n * k * r / (us * 1e-6) / 1e12}
+    del qs, outs
+    torch.cuda.empty_cache()
+    npar = sum(r * kk + nn * r for nn, kk in ((8192, 8192),) * 4 + ((22016, 8192),) * 2 + ((8192, 22016),))
+    p, g, m, v = (torch.randn(npar, device=device) * 0.01 for _ in range(4))
+    v.abs_()
+    p16 = torch.empty(npar, dtype=torch.bfloat16, device=device)
+    for i in range(3):
+        bd.adamw_step(p, g, m, v, i + 1, 1e-4, weight_decay=0.01, p_bf16=p16)
+    torch.cuda.synchronize()
+    st, en = cuda_timer()
+    steps = 20
+    st.record()
+    for i in range(steps):
+        bd.adamw_step(p, g, m, v, i + 4, 1e-4, weight_decay=0.01, p_bf16=p16)
+    en.record()
+    torch.cuda.synchronize()
+    us = st.elapsed_time(en) * 1e3 / steps
+    nbytes = npar * (16 + 12 + 2)
+    res["adamw_65b_block_adapters"] = {"params": npar, "us": us, "GB/s": nbytes / (us * 1e-6) / 1e9,
+                                       "frac_of_hbm": nbytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"]}
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -521,7 +574,8 @@ def main():
         del host_x, host_dy
         layers.clear()
         torch.cuda.empty_cache()
-        line["sub"] = {"gemv_11008x4096_r64": sub_gemv(device, peaks), "quant_sweep": sub_quant(device, peaks)}
+        line["sub"] = {"gemv_11008x4096_r64": sub_gemv(device, peaks), "quant_sweep": sub_quant(device, peaks),
+                       "adapter_steps": sub_adapters(device, peaks)}
     if rank == 0 and world == 1 and not args.no_cpu:
         v, threads, desc, secs = oracle_sample()
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,

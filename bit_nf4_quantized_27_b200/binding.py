@@ -43,6 +43,11 @@ class LoraC(ctypes.Structure):
     _fields_ = [("r", ctypes.c_int32), ("alpha", ctypes.c_float), ("A", ctypes.c_void_p), ("B", ctypes.c_void_p)]
 
 
+class AdamWC(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float), ("eps", ctypes.c_float),
+                ("weight_decay", ctypes.c_float)]
+
+
 _lib = None
 
 
@@ -66,6 +71,8 @@ def lib():
         "qlora_linear_fwd": (ctypes.c_int, [pT, pL, vp, i64, vp, ctypes.c_int, vp, vp, sz, vp]),
         "qlora_linear_bwd": (ctypes.c_int, [pT, pL, vp, vp, i64, vp, vp, ctypes.c_int, vp, vp, ctypes.c_int, vp,
                                             sz, vp]),
+        "qlora_lora_merge": (ctypes.c_int, [pT, pL, vp, vp]),
+        "qlora_adamw_step": (ctypes.c_int, [vp, vp, vp, vp, vp, i64, ctypes.POINTER(AdamWC), i64, vp]),
         "qlora_clear_status": (ctypes.c_int, [vp, vp]),
         "qlora_read_status": (ctypes.c_int, [vp, vp]),
         "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -241,3 +248,26 @@ class QLoRALinearFunction(torch.autograd.Function):
         X, A, B, T = ctx.saved_tensors
         dX, dA, dB = linear_bwd(ctx.q, A, B, ctx.alpha, X, dY.contiguous().to(torch.bfloat16), T)
         return dX, dA, dB, None, None
+
+
+def merge(q: NF4Weight, A, B, alpha: float, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Merged export W_merged [N, K] bf16 = bf16(W' + (alpha/r) B A)."""
+    if out is None:
+        out = torch.empty(q.rows, q.cols, dtype=torch.bfloat16, device=A.device)
+    t, ad = q.c_struct(), _lora(A, B, alpha)
+    _check(lib().qlora_lora_merge(ctypes.byref(t), ctypes.byref(ad), _ptr(out), _stream(stream)), "qlora_lora_merge")
+    return out
+
+
+def adamw_step(p: torch.Tensor, g: torch.Tensor, m: torch.Tensor, v: torch.Tensor, step: int, lr: float,
+               beta1: float = 0.9, beta2: float = 0.999, eps: float = 1e-8, weight_decay: float = 0.0,
+               p_bf16: torch.Tensor | None = None, stream=None) -> None:
+    """One AdamW step in place on flat float32 tensors p, m, v with gradient g;
+    writes bf16(p) to p_bf16 if given."""
+    for t in (p, g, m, v):
+        assert t.dtype == torch.float32 and t.is_contiguous() and t.numel() == p.numel()
+    if p_bf16 is not None:
+        assert p_bf16.dtype == torch.bfloat16 and p_bf16.is_contiguous() and p_bf16.numel() == p.numel()
+    hp = AdamWC(lr, beta1, beta2, eps, weight_decay)
+    _check(lib().qlora_adamw_step(_ptr(p), _ptr(p_bf16), _ptr(g), _ptr(m), _ptr(v), p.numel(), ctypes.byref(hp),
+                                  step, _stream(stream)), "qlora_adamw_step")

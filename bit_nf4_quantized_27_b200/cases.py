@@ -11,6 +11,8 @@ CASE is one of:
   gemv_m1 / gemv_m4 / gemv_m16   decode forward, W 11008x4096, r=64
   quant_11008   quantise an 11008x4096 bf16 weight
   dequant_11008 dequantise it
+  merge_8192    merged export of an 8192x8192 NF4 weight with an r = 64 adapter
+  adamw_65b     AdamW step over the adapters of the 65B-shaped block (flat fp32)
 Inputs are drawn on the device from fixed seeds; every run exits 0 on success.
 """
 
@@ -73,6 +75,22 @@ def main(argv=None):
             else:
                 bd.dequantize(q, out=out)
         st = bd.read_status(ws)
+    elif c == "merge_8192":
+        w, _, a, b, _ = _layer(8192, 8192, 1)
+        q = bd.quantize(w)
+        del w
+        out = torch.empty(8192, 8192, dtype=torch.bfloat16, device="cuda")
+        for _ in range(args.reps):
+            bd.merge(q, a, b, 16.0, out=out)
+        st = 0
+    elif c == "adamw_65b":
+        n = sum(64 * k + nn * 64 for nn, k in ((8192, 8192),) * 4 + ((22016, 8192),) * 2 + ((8192, 22016),))
+        p, g, m, v = (torch.randn(n, device="cuda") * 0.01 for _ in range(4))
+        v.abs_()
+        p16 = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+        for i in range(args.reps):
+            bd.adamw_step(p, g, m, v, i + 1, 1e-4, weight_decay=0.01, p_bf16=p16)
+        st = 0
     else:
         raise SystemExit(f"unknown case {c}")
     torch.cuda.synchronize()

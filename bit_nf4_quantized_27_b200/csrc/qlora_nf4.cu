@@ -4,11 +4,13 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstring>
 #include <mutex>
 
 #include "gemm_kernel.cuh"
 #include "gemm_pair_kernel.cuh"
+#include "adapter_kernels.cuh"
 #include "gemv_kernel.cuh"
 #include "host_common.h"
 #include "qlora_nf4.h"
@@ -522,6 +524,59 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
       return s;
   }
   return QLORA_OK;
+}
+
+qlora_status qlora_lora_merge(const qlora_nf4_tensor *W, const qlora_lora *adapter, void *W_out,
+                              qlora_stream_t stream) {
+  qlora_status s = check_nf4(W);
+  if (s != QLORA_OK) return s;
+  if ((s = check_lora(adapter)) != QLORA_OK) return s;
+  if (!W_out) return QLORA_ERR_INVALID_ARGUMENT;
+  if (!aligned(W_out, 16)) return QLORA_ERR_MISALIGNED;
+  int dev, sms;
+  if ((s = check_device(&dev, &sms)) != QLORA_OK) return s;
+  const int bytes = static_cast<int>(merge_smem_bytes(adapter->r));
+  static std::once_flag flags[64];
+  static qlora_status results[64];
+  if ((s = set_smem(nf4_lora_merge_kernel, static_cast<int>(merge_smem_bytes(QLORA_MAX_RANK)), dev, flags,
+                    results)) != QLORA_OK)
+    return s;
+  const dim3 grid(static_cast<unsigned>((W->cols + kMergeTile - 1) / kMergeTile),
+                  static_cast<unsigned>((W->rows + kMergeTile - 1) / kMergeTile));
+  const float sc = adapter->alpha / static_cast<float>(adapter->r);
+  nf4_lora_merge_kernel<<<grid, kMergeThreads, bytes, reinterpret_cast<cudaStream_t>(stream)>>>(
+      W->codes, W->scale_codes, W->c2, W->rows, W->cols, static_cast<const __nv_bfloat16 *>(adapter->A),
+      static_cast<const __nv_bfloat16 *>(adapter->B), adapter->r, sc, static_cast<__nv_bfloat16 *>(W_out));
+  return launch_status();
+}
+
+qlora_status qlora_adamw_step(float *param, void *param_bf16, const float *grad, float *exp_avg, float *exp_avg_sq,
+                              int64_t n, const qlora_adamw_hparams *hp, int64_t step, qlora_stream_t stream) {
+  if (!param || !grad || !exp_avg || !exp_avg_sq || !hp || n < 1 || step < 1) return QLORA_ERR_INVALID_ARGUMENT;
+  if (!(hp->lr >= 0.0f) || !(hp->beta1 >= 0.0f && hp->beta1 < 1.0f) || !(hp->beta2 >= 0.0f && hp->beta2 < 1.0f) ||
+      !(hp->eps > 0.0f) || !(hp->weight_decay >= 0.0f) || !std::isfinite(hp->lr) || !std::isfinite(hp->weight_decay))
+    return QLORA_ERR_INVALID_ARGUMENT;
+  if (!aligned(param, 16) || !aligned(grad, 16) || !aligned(exp_avg, 16) || !aligned(exp_avg_sq, 16) ||
+      (param_bf16 && !aligned(param_bf16, 8)))
+    return QLORA_ERR_MISALIGNED;
+  int dev, sms;
+  qlora_status s;
+  if ((s = check_device(&dev, &sms)) != QLORA_OK) return s;
+  AdamWConsts c;
+  const double bc1 = 1.0 - std::pow(static_cast<double>(hp->beta1), static_cast<double>(step));
+  const double bc2 = 1.0 - std::pow(static_cast<double>(hp->beta2), static_cast<double>(step));
+  c.lr = hp->lr;
+  c.beta1 = hp->beta1;
+  c.beta2 = hp->beta2;
+  c.eps = hp->eps;
+  c.decay_factor = static_cast<float>(1.0 - static_cast<double>(hp->lr) * hp->weight_decay);
+  c.step_size = static_cast<float>(hp->lr / bc1);
+  c.sqrt_bc2 = static_cast<float>(std::sqrt(bc2));
+  const int64_t want = (n / 4 + 255) / 256;
+  const unsigned grid = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)sms * 8)));
+  adamw_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      param, static_cast<__nv_bfloat16 *>(param_bf16), grad, exp_avg, exp_avg_sq, n, c);
+  return launch_status();
 }
 
 }  // extern "C"

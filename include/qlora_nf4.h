@@ -187,6 +187,42 @@ QLORA_API qlora_status qlora_linear_fwd_noalloc(const qlora_nf4_tensor *W, const
                                                 const void *X, int64_t M, void *Y, qlora_dtype y_dtype,
                                                 void *T_save, qlora_stream_t stream);
 
+/* Merged export of a trained adapter ("QLoRA" glossary page, "Trade-offs":
+ * merging into the base model needs it dequantised to 16 bit; "What is LoRA?"
+ * (IBM): the low-rank update merges into the frozen weights for deployment):
+ *   W_out [N, K] bf16 = bf16_rne(W' + s B A),  s = alpha / r,
+ * with W' the dequantised NF4 weight, s B A from the bf16 adapter on tensor
+ * cores with float32 accumulation, the sum in float32, rounded to bf16 once.
+ * W_out: device, 16-byte aligned, caller-owned, overwritten.  Errors as for
+ * qlora_linear_fwd (invalid tensor or adapter, misalignment, no device). */
+QLORA_API qlora_status qlora_lora_merge(const qlora_nf4_tensor *W, const qlora_lora *adapter, void *W_out,
+                                        qlora_stream_t stream);
+
+/* AdamW hyper-parameters: learning rate lr >= 0, 0 <= beta1, beta2 < 1,
+ * eps > 0, decoupled weight decay >= 0. */
+typedef struct qlora_adamw_hparams {
+  float lr;
+  float beta1;
+  float beta2;
+  float eps;
+  float weight_decay;
+} qlora_adamw_hparams;
+
+/* One AdamW step (decoupled weight decay, bias-corrected; "Grokking QLoRA"
+ * (vnread), "Paged Optimizers": Adam keeps a momentum and a variance for every
+ * trained parameter) on n float32 parameters, in place:
+ *   m = b1 m + (1 - b1) g;  v = b2 v + (1 - b2) g^2;
+ *   p = p (1 - lr wd) - (lr / (1 - b1^t)) m / (sqrt(v) / sqrt(1 - b2^t) + eps)
+ * t = step >= 1.  param, grad, exp_avg, exp_avg_sq: device float32 [n], 16-byte
+ * aligned (m and v start at zero before step 1).  param_bf16: nullable device
+ * bf16 [n], 8-byte aligned; receives bf16(p), the copy the layer reads.  Used
+ * on the flat buffer of every layer's A and B after the data-parallel
+ * all-reduce of their gradients.  QLORA_ERR_INVALID_ARGUMENT for n < 1, step
+ * < 1, a missing pointer or hyper-parameters out of range. */
+QLORA_API qlora_status qlora_adamw_step(float *param, void *param_bf16, const float *grad, float *exp_avg,
+                                        float *exp_avg_sq, int64_t n, const qlora_adamw_hparams *hp, int64_t step,
+                                        qlora_stream_t stream);
+
 /* Zero the status word at the start of ws (enqueued on stream). */
 QLORA_API qlora_status qlora_clear_status(void *ws, qlora_stream_t stream);
 

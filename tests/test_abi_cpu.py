@@ -108,3 +108,26 @@ def test_device_level_literals_match_bit_patterns():
     assert len(bits) == 16 and len(vals) == 16
     assert bits == vals
     assert bits == [int(x) for x in O.nf4_levels().view(np.uint32)]
+
+
+def test_merge_and_adamw_argument_checks_without_gpu(L):
+    good = _t(64, 64)
+    ad = bd.LoraC(64, 16.0, 0x4000, 0x5000)
+    out = ctypes.c_void_p(0x6000)
+    assert L.qlora_lora_merge(ctypes.byref(good), ctypes.byref(ad), None, None) == 1
+    assert L.qlora_lora_merge(ctypes.byref(good), ctypes.byref(ad), ctypes.c_void_p(0x6008), None) == 3
+    assert L.qlora_lora_merge(ctypes.byref(good), ctypes.byref(bd.LoraC(12, 16.0, 0x4000, 0x5000)), out, None) == 1
+    assert L.qlora_lora_merge(ctypes.byref(_t(64, 65)), ctypes.byref(ad), out, None) == 2
+    p, g, m, v, h = (ctypes.c_void_p(a) for a in (0x10000, 0x20000, 0x30000, 0x40000, 0x50000))
+    hp = bd.AdamWC(1e-3, 0.9, 0.999, 1e-8, 0.01)
+    assert L.qlora_adamw_step(p, h, g, m, v, 0, ctypes.byref(hp), 1, None) == 1
+    assert L.qlora_adamw_step(p, h, g, m, v, 10, ctypes.byref(hp), 0, None) == 1
+    assert L.qlora_adamw_step(p, h, g, m, v, 10, ctypes.byref(bd.AdamWC(1e-3, 1.0, 0.999, 1e-8, 0.0)), 1, None) == 1
+    assert L.qlora_adamw_step(p, h, g, m, v, 10, ctypes.byref(bd.AdamWC(1e-3, 0.9, 0.999, 0.0, 0.0)), 1, None) == 1
+    assert L.qlora_adamw_step(p, h, None, m, v, 10, ctypes.byref(hp), 1, None) == 1
+    assert L.qlora_adamw_step(ctypes.c_void_p(0x10004), h, g, m, v, 10, ctypes.byref(hp), 1, None) == 3
+    assert L.qlora_adamw_step(p, ctypes.c_void_p(0x50002), g, m, v, 10, ctypes.byref(hp), 1, None) == 3
+    import torch
+    if not torch.cuda.is_available():
+        assert L.qlora_adamw_step(p, None, g, m, v, 10, ctypes.byref(hp), 1, None) == 8
+        assert L.qlora_lora_merge(ctypes.byref(good), ctypes.byref(ad), out, None) == 8
