@@ -37,6 +37,7 @@ from .nf4_oracle import (  # noqa: F401
     lora_scale,
     linear_fwd,
     linear_bwd,
+    linear_fwd_multi,
     merged_weight,
     merge_export,
     adamw_step,

@@ -358,6 +358,23 @@ def linear_bwd(w_dq: np.ndarray, a: np.ndarray, b: np.ndarray, x: np.ndarray,
     return dx, da, db
 
 
+def linear_fwd_multi(w_dq: np.ndarray, adapters, adapter_of_token, x: np.ndarray):
+    """Forward of one frozen base serving several adapters: token t uses adapter
+    adapters[adapter_of_token[t]] = (A, B, alpha, r), y_t = W' x_t + s_t (x_t A^T) B^T.
+
+    [IBM] (one shared base model, many small LoRA modules swapped per task);
+    [UL] "Trade-offs" (adapters small enough to store and swap per task).
+    Returns y [M, N] float64.
+    """
+    x = np.asarray(x)
+    out = []
+    for t in range(x.shape[0]):
+        a, b, alpha, r = adapters[adapter_of_token[t]]
+        y, _ = linear_fwd(w_dq, a, b, x[t:t + 1], alpha, r)
+        out.append(y[0])
+    return np.stack(out)
+
+
 def merged_weight(w_dq: np.ndarray, a: np.ndarray, b: np.ndarray, alpha: float, r: int):
     """W' + s B A (float64): the merged deployment form [IBM; EZ, Delta W = B A]."""
     s = lora_scale(alpha, r)

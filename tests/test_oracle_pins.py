@@ -534,3 +534,21 @@ def test_adamw_pin_catches_a_planted_sign_error():
     bad = p0 + 1e-2 * g / (np.abs(g) + 1e-8)  # the update applied with the wrong sign
     tp, _, _ = _adamw_torch(p0, [g], 1e-2, 0.9, 0.999, 1e-8, 0.0)
     assert np.allclose(good, tp) and not np.allclose(bad, tp)
+
+
+def test_multi_adapter_forward_reduces_and_separates():
+    w, a, b, x, _ = _tiny_linear(8, m=5, n=9, k=20, r=3)
+    rng = np.random.default_rng(9)
+    a2, b2 = rng.standard_normal(a.shape), rng.standard_normal(b.shape)
+    ads = [(a, b, 6.0, 3), (a2, b2, 2.0, 3)]
+    # one adapter for every token: the single-adapter forward
+    y1, _ = O.linear_fwd(w, a, b, x, 6.0, 3)
+    assert np.array_equal(O.linear_fwd_multi(w, ads, [0] * 5, x), y1)
+    # a token's output depends only on its own adapter
+    idx = [1, 0, 1, 1, 0]
+    ym = O.linear_fwd_multi(w, ads, idx, x)
+    y2, _ = O.linear_fwd(w, a2, b2, x, 2.0, 3)
+    for t, i in enumerate(idx):
+        assert np.array_equal(ym[t], (y1 if i == 0 else y2)[t])
+    # and two different adapters give different outputs
+    assert not np.allclose(ym[0], y1[0])
