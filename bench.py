@@ -346,6 +346,27 @@ def sub_gemv(device, peaks):
         out[f"m{m}"] = {"us_per_call": us, "GB/s": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
                         "GB/s_incl_adapters": (nf4 + act + (r * k + n * r) * 2) / (us * 1e-6) / 1e9,
                         "launches_per_call": 2, "timing": "CUDA graph of 64 calls, 8 weight copies"}
+    # 16 decode tokens, each with its own adapter on the same base
+    m = 16
+    ads = [((torch.randn(r, k, generator=g, device=device) / 64).to(torch.bfloat16),
+            (torch.randn(n, r, generator=g, device=device) * 0.01).to(torch.bfloat16), wl.alpha) for _ in range(m)]
+    x = torch.randn(m, k, generator=g, device=device).to(torch.bfloat16)
+    y = torch.empty(m, n, dtype=torch.bfloat16, device=device)
+    ws = bd.new_workspace(bd.workspace_bytes(m, n, k, r, False), device)
+    reps = 8 * copies
+    idx = list(range(m))
+
+    def calls_multi():
+        for i in range(reps):
+            bd.linear_fwd_multi(qs[i % copies], ads, idx, x, ws=ws, out=y)
+
+    us = graph_time_us(calls_multi) / reps
+    nf4 = n * k // 2 + n * k // 64 + 4 * ((n * k // 64 + 255) // 256)
+    act = m * k * 2 + m * n * 2
+    gbs = (nf4 + act) / (us * 1e-6) / 1e9
+    out["m16_16_adapters"] = {"us_per_call": us, "GB/s": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
+                              "GB/s_incl_adapters": (nf4 + act + m * (r * k + n * r) * 2) / (us * 1e-6) / 1e9,
+                              "launches_per_call": 2, "timing": "CUDA graph of 64 calls, 8 weight copies"}
     return out
 
 

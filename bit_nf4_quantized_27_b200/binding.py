@@ -71,6 +71,8 @@ def lib():
         "qlora_linear_fwd": (ctypes.c_int, [pT, pL, vp, i64, vp, ctypes.c_int, vp, vp, sz, vp]),
         "qlora_linear_bwd": (ctypes.c_int, [pT, pL, vp, vp, i64, vp, vp, ctypes.c_int, vp, vp, ctypes.c_int, vp,
                                             sz, vp]),
+        "qlora_linear_fwd_multi": (ctypes.c_int, [pT, pL, i32, ctypes.POINTER(i32), vp, i64, vp, ctypes.c_int, vp,
+                                                  sz, vp]),
         "qlora_lora_merge": (ctypes.c_int, [pT, pL, vp, vp]),
         "qlora_adamw_step": (ctypes.c_int, [vp, vp, vp, vp, vp, i64, ctypes.POINTER(AdamWC), i64, vp]),
         "qlora_clear_status": (ctypes.c_int, [vp, vp]),
@@ -271,3 +273,21 @@ def adamw_step(p: torch.Tensor, g: torch.Tensor, m: torch.Tensor, v: torch.Tenso
     hp = AdamWC(lr, beta1, beta2, eps, weight_decay)
     _check(lib().qlora_adamw_step(_ptr(p), _ptr(p_bf16), _ptr(g), _ptr(m), _ptr(v), p.numel(), ctypes.byref(hp),
                                   step, _stream(stream)), "qlora_adamw_step")
+
+
+def linear_fwd_multi(q: NF4Weight, adapters, adapter_of_token, X, y_dtype=torch.bfloat16,
+                     ws: torch.Tensor | None = None, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Decode forward of one base serving several adapters: adapters is a list of
+    (A, B, alpha) of one rank; token t uses adapters[adapter_of_token[t]]."""
+    M = X.shape[0]
+    r = adapters[0][0].shape[0]
+    Y = out if out is not None else torch.empty(M, q.rows, dtype=y_dtype, device=X.device)
+    arr = (LoraC * len(adapters))(*[_lora(a, b, alpha) for a, b, alpha in adapters])
+    idx = (ctypes.c_int32 * M)(*[int(i) for i in adapter_of_token])
+    if ws is None:
+        ws = new_workspace(workspace_bytes(M, q.rows, q.cols, r, False), X.device)
+    t = q.c_struct()
+    _check(lib().qlora_linear_fwd_multi(ctypes.byref(t), arr, len(adapters), idx, _ptr(X), M, _ptr(Y),
+                                        _dtype_code(Y.dtype), _ptr(ws), ws.numel(), _stream(stream)),
+           "qlora_linear_fwd_multi")
+    return Y

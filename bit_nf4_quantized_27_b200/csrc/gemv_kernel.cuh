@@ -33,6 +33,14 @@ constexpr int kGemvWarps = 16;
 constexpr int kGemvThreads = kGemvWarps * 32;
 constexpr int kGemvMaxRG = 10;  // row groups of 16 per CTA
 
+// Per-token adapters of a decode batch that serves several adapters on one base:
+// token t uses A[t] [r, K], B[t] [N, r] and scale s[t].
+struct MultiLora {
+  const __nv_bfloat16 *A[kGemvMaxM];
+  const __nv_bfloat16 *B[kGemvMaxM];
+  float s[kGemvMaxM];
+};
+
 struct GemvArgs {
   const uint8_t *codes;
   const uint8_t *scale_codes;
@@ -49,6 +57,8 @@ struct GemvArgs {
   uint32_t *status;
   int rg_per_cta;
   int stages;               // bulk kernel: depth of the shared-memory ring
+  int multi;                // 1: token t adds s[t] (x_t A_t^T) B_t^T with ml's adapters
+  MultiLora ml;
 };
 
 inline size_t gemv_workspace_bytes(int64_t, int64_t, int64_t) { return 0; }
@@ -688,7 +698,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   // waiting for the kernel that computes it.
   const int lora_rg = warp < my_rg ? warp : -1;
   uint32_t bfr[4][4];
-  if (lora_rg >= 0) {
+  if (lora_rg >= 0 && !a.multi) {
     const int64_t n0 = (int64_t)(rg0 + lora_rg) * 16;
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) {
@@ -703,7 +713,29 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   }
   __syncthreads();
   griddep_wait();
-  if (lora_rg >= 0) {
+  if (lora_rg >= 0 && a.multi) {
+    // one adapter per token: row (lane & 15) of this row group, half of the
+    // rank range per half-warp, combined by a shuffle (fixed order)
+    const int64_t n = (int64_t)(rg0 + lora_rg) * 16 + (lane & 15);
+    const int half = lane >> 4, hr = a.r / 2;  // r % 8 == 0: hr is a multiple of 4
+    float *rb = red_at(lora_rg);  // warp 0's slot
+    for (int t = 0; t < a.M; ++t) {
+      const __nv_bfloat16 *bt = a.ml.B[t] + n * a.r + half * hr;
+      const __nv_bfloat16 *st = a.sT + (int64_t)t * a.r + half * hr;
+      float acc = 0.0f;
+      for (int j = 0; j < hr; j += 4) {
+        const uint2 bv = __ldg(reinterpret_cast<const uint2 *>(bt + j));
+        const uint2 sv = __ldg(reinterpret_cast<const uint2 *>(st + j));
+        acc = fmaf(bf16lo_to_f32(bv.x), bf16lo_to_f32(sv.x), acc);
+        acc = fmaf(bf16hi_to_f32(bv.x), bf16hi_to_f32(sv.x), acc);
+        acc = fmaf(bf16lo_to_f32(bv.y), bf16lo_to_f32(sv.y), acc);
+        acc = fmaf(bf16hi_to_f32(bv.y), bf16hi_to_f32(sv.y), acc);
+      }
+      acc += __shfl_xor_sync(0xffffffffu, acc, 16);
+      if (half == 0) rb[(lane & 15) * TR + t] += acc;
+    }
+  }
+  if (lora_rg >= 0 && !a.multi) {
     const int64_t n0 = (int64_t)(rg0 + lora_rg) * 16;
     float acc[NG][4];
 #pragma unroll
@@ -859,6 +891,57 @@ __global__ void __launch_bounds__(kLoraDownThreads, 1) lora_down_small_kernel(
   }
 }
 
+// s_t T_t = s_t (x_t A_t^T) for decode tokens that each use their own adapter:
+// CTA (16-rank tile, token t), 256 threads splitting K in 8-element slices with
+// all 16 ranks' loads of a slice in flight; warp-shuffle then cross-warp sums
+// in a fixed order.  Writes s*T (bf16).
+constexpr int kLoraDownMultiThreads = 256;
+__global__ void __launch_bounds__(kLoraDownMultiThreads) lora_down_multi_kernel(
+    const __nv_bfloat16 *__restrict__ X, const MultiLora ml, int64_t K, int r, __nv_bfloat16 *__restrict__ sT) {
+  griddep_launch_dependents();
+  __shared__ float red[kLoraDownMultiThreads / 32][16];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int t = blockIdx.y, j0 = blockIdx.x * 16;
+  const __nv_bfloat16 *A = ml.A[t];
+  const __nv_bfloat16 *x = X + (int64_t)t * K;
+  float acc[16];
+#pragma unroll
+  for (int jj = 0; jj < 16; ++jj) acc[jj] = 0.0f;
+  for (int64_t k = (int64_t)tid * 8; k < K; k += kLoraDownMultiThreads * 8) {
+    const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(x + k));
+    const float xf[8] = {bf16lo_to_f32(xv.x), bf16hi_to_f32(xv.x), bf16lo_to_f32(xv.y), bf16hi_to_f32(xv.y),
+                         bf16lo_to_f32(xv.z), bf16hi_to_f32(xv.z), bf16lo_to_f32(xv.w), bf16hi_to_f32(xv.w)};
+    uint4 av[16];
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj)
+      av[jj] = (j0 + jj < r) ? __ldg(reinterpret_cast<const uint4 *>(A + (int64_t)(j0 + jj) * K + k))
+                             : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) {
+      const uint32_t w[4] = {av[jj].x, av[jj].y, av[jj].z, av[jj].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc[jj] = fmaf(bf16lo_to_f32(w[e]), xf[2 * e], acc[jj]);
+        acc[jj] = fmaf(bf16hi_to_f32(w[e]), xf[2 * e + 1], acc[jj]);
+      }
+    }
+  }
+#pragma unroll
+  for (int jj = 0; jj < 16; ++jj) {
+    float v = acc[jj];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) red[warp][jj] = v;
+  }
+  __syncthreads();
+  if (tid < 16 && j0 + tid < r) {
+    float v = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kLoraDownMultiThreads / 32; ++w) v += red[w][tid];
+    sT[(int64_t)t * r + j0 + tid] = __float2bfloat16_rn(v * ml.s[t]);
+  }
+}
+
 // Start of the dynamic shared-memory window of a kernel without static shared
 // memory: after the block's system reservation.  The bulk kernel recomputes its
 // layout from its real window start and reports an error if it does not fit.
@@ -892,6 +975,7 @@ inline qlora_status launch_gemv(GemvArgs g, const CUtensorMap *tm_codes, int dev
     if (g.stages == 0) bulk = false;
     else smem = gemv_bulk_smem_bytes(g.K, g.stages, g.M, base);
   }
+  if (!bulk && g.multi) return QLORA_ERR_UNSUPPORTED_SHAPE;  // per-token adapters: staged kernel only
   if (!bulk) {
     per = (num_rg + sms - 1) / sms;
     if (per > kGemvMaxRG) per = kGemvMaxRG;

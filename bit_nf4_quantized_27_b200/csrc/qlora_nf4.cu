@@ -526,6 +526,55 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
   return QLORA_OK;
 }
 
+qlora_status qlora_linear_fwd_multi(const qlora_nf4_tensor *W, const qlora_lora *adapters, int32_t n_adapters,
+                                    const int32_t *adapter_of_token, const void *X, int64_t M, void *Y,
+                                    qlora_dtype y_dtype, void *ws, size_t ws_bytes, qlora_stream_t stream) {
+  qlora_status s = check_nf4(W);
+  if (s != QLORA_OK) return s;
+  if (!adapters || n_adapters < 1 || !adapter_of_token || !X || !Y || !ws || M < 1 || M > kGemvMaxM ||
+      !valid_dtype(y_dtype))
+    return QLORA_ERR_INVALID_ARGUMENT;
+  const int r = adapters[0].r;
+  for (int32_t i = 0; i < n_adapters; ++i) {
+    if ((s = check_lora(&adapters[i])) != QLORA_OK) return s;
+    if (adapters[i].r != r) return QLORA_ERR_INVALID_ARGUMENT;
+  }
+  for (int64_t t = 0; t < M; ++t)
+    if (adapter_of_token[t] < 0 || adapter_of_token[t] >= n_adapters) return QLORA_ERR_INVALID_ARGUMENT;
+  if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
+  const int64_t N = W->rows, K = W->cols;
+  if (!gemv_bulk_ok(N, K)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (ws_bytes < min_workspace_bytes(M, N, K, r, 0)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  int dev, sms;
+  if ((s = check_device(&dev, &sms)) != QLORA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  GemvArgs g{};
+  for (int64_t t = 0; t < M; ++t) {
+    const qlora_lora &ad = adapters[adapter_of_token[t]];
+    g.ml.A[t] = static_cast<const __nv_bfloat16 *>(ad.A);
+    g.ml.B[t] = static_cast<const __nv_bfloat16 *>(ad.B);
+    g.ml.s[t] = ad.alpha / static_cast<float>(r);
+  }
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  __nv_bfloat16 *sT = reinterpret_cast<__nv_bfloat16 *>(wsb + QLORA_STATUS_BYTES);
+  lora_down_multi_kernel<<<dim3((r + 15) / 16, static_cast<unsigned>(M)), kLoraDownMultiThreads, 0, st>>>(
+      static_cast<const __nv_bfloat16 *>(X), g.ml, K, r, sT);
+  if ((s = launch_status()) != QLORA_OK) return s;
+  g.codes = W->codes; g.scale_codes = W->scale_codes; g.c2 = W->c2;
+  g.N = N; g.K = K; g.M = (int)M;
+  g.X = static_cast<const __nv_bfloat16 *>(X);
+  g.sT = sT;
+  g.B = g.ml.B[0];
+  g.r = r;
+  g.Y = Y; g.y_f32 = y_dtype == QLORA_F32;
+  g.status = status_ptr(ws);
+  g.multi = 1;
+  CUtensorMap tmc;
+  if (!tmap_codes_gemv(&tmc, W->codes, N, K, static_cast<uint32_t>((K < 4096 ? K : 4096) / 256)))
+    return QLORA_ERR_CUDA;
+  return launch_gemv(g, &tmc, dev, sms, st);
+}
+
 qlora_status qlora_lora_merge(const qlora_nf4_tensor *W, const qlora_lora *adapter, void *W_out,
                               qlora_stream_t stream) {
   qlora_status s = check_nf4(W);

@@ -187,6 +187,22 @@ QLORA_API qlora_status qlora_linear_fwd_noalloc(const qlora_nf4_tensor *W, const
                                                 const void *X, int64_t M, void *Y, qlora_dtype y_dtype,
                                                 void *T_save, qlora_stream_t stream);
 
+/* Decode forward of one NF4 base serving several adapters at once ("What is
+ * LoRA?" (IBM): one shared frozen base, many small LoRA modules swapped per task;
+ * "QLoRA" glossary page, "Trade-offs": adapters are small enough to store and
+ * swap per task).  Token t uses adapters[adapter_of_token[t]]:
+ *   Y[t] = X[t] W'^T + s_t (X[t] A_t^T) B_t^T,   s_t = alpha_t / r.
+ *   adapters          host array of n_adapters >= 1 adapters, all of one rank r
+ *   adapter_of_token  HOST int32 [M], values in [0, n_adapters)
+ *   X bf16 [M, K], Y [M, N] (y_dtype) device; 1 <= M <= 16
+ *   ws                device workspace, as qlora_linear_fwd's for M tokens
+ * Runs the staged decode kernel: N % 16 == 0, K % 256 == 0 and (K <= 4096 or
+ * K % 4096 == 0), else QLORA_ERR_UNSUPPORTED_SHAPE.  No T is saved (decode). */
+QLORA_API qlora_status qlora_linear_fwd_multi(const qlora_nf4_tensor *W, const qlora_lora *adapters,
+                                              int32_t n_adapters, const int32_t *adapter_of_token, const void *X,
+                                              int64_t M, void *Y, qlora_dtype y_dtype, void *ws, size_t ws_bytes,
+                                              qlora_stream_t stream);
+
 /* Merged export of a trained adapter ("QLoRA" glossary page, "Trade-offs":
  * merging into the base model needs it dequantised to 16 bit; "What is LoRA?"
  * (IBM): the low-rank update merges into the frozen weights for deployment):

@@ -131,3 +131,20 @@ def test_merge_and_adamw_argument_checks_without_gpu(L):
     if not torch.cuda.is_available():
         assert L.qlora_adamw_step(p, None, g, m, v, 10, ctypes.byref(hp), 1, None) == 8
         assert L.qlora_lora_merge(ctypes.byref(good), ctypes.byref(ad), out, None) == 8
+
+
+def test_multi_adapter_argument_checks_without_gpu(L):
+    good = _t(1024, 1024)
+    ads = (bd.LoraC * 2)(bd.LoraC(16, 16.0, 0x4000, 0x5000), bd.LoraC(16, 8.0, 0x6000, 0x7000))
+    idx = (ctypes.c_int32 * 3)(0, 1, 1)
+    X, Y, ws = ctypes.c_void_p(0x10000), ctypes.c_void_p(0x20000), ctypes.c_void_p(0x30000)
+    f = L.qlora_linear_fwd_multi
+    assert f(ctypes.byref(good), ads, 2, idx, X, 3, Y, 1, ws, 1 << 20, None) in (0, 8)  # valid (no GPU: 8)
+    bad_idx = (ctypes.c_int32 * 3)(0, 2, 1)
+    assert f(ctypes.byref(good), ads, 2, bad_idx, X, 3, Y, 1, ws, 1 << 20, None) == 1
+    assert f(ctypes.byref(good), ads, 2, idx, X, 17, Y, 1, ws, 1 << 20, None) == 1
+    assert f(ctypes.byref(good), ads, 0, idx, X, 3, Y, 1, ws, 1 << 20, None) == 1
+    mixed = (bd.LoraC * 2)(bd.LoraC(16, 16.0, 0x4000, 0x5000), bd.LoraC(32, 8.0, 0x6000, 0x7000))
+    assert f(ctypes.byref(good), mixed, 2, idx, X, 3, Y, 1, ws, 1 << 20, None) == 1
+    assert f(ctypes.byref(_t(1024, 576)), ads, 2, idx, X, 3, Y, 1, ws, 1 << 20, None) == 2
+    assert f(ctypes.byref(good), ads, 2, idx, X, 3, Y, 1, ws, 64, None) == 4

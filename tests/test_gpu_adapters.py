@@ -71,3 +71,39 @@ def test_adamw_matches_oracle_over_six_steps(n):
     assert np.all(np.abs(gm - rm) <= 2e-6 * mag_m)
     assert np.all(np.abs(gv - rv) <= 2e-6 * (np.abs(rv) + 1e-12))
     assert torch.equal(p16, p.to(torch.bfloat16))
+
+
+def _adapters(n, k, r, count, seed):
+    out = []
+    for i in range(count):
+        _, _, a, b, _ = I.custom(n, k, 1, r, seed + 7 * i)
+        out.append((a, b * (1 + i), 16.0 / (1 + i)))  # distinct B scale and alpha per adapter
+    return out
+
+
+def _check(name, got, ref):
+    g = got.float().cpu().numpy().astype(np.float64)
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    err = float(np.max(np.abs(g - ref)))
+    assert np.all(np.isfinite(g)) and err <= 1e-2 * rms, f"{name}: {err:.3e} vs {1e-2 * rms:.3e}"
+
+
+@pytest.mark.parametrize("n,k,m,r,count", [(11008, 4096, 1, 64, 2), (11008, 4096, 5, 64, 3), (11008, 4096, 16, 64, 16),
+                                           (1024, 1024, 9, 16, 4), (2048, 8192, 4, 128, 2), (512, 256, 3, 8, 3)])
+def test_multi_adapter_gemv_matches_oracle(n, k, m, r, count):
+    w, x, _, _, _ = I.custom(n, k, m, r, 9000 + n + m)
+    ads = _adapters(n, k, r, count, 9100 + k)
+    idx = [(3 * t + 1) % count for t in range(m)]
+    q = O.quantize(w.float().numpy(), n, k)
+    wd = O.dequantize(q["codes"], q["scale_codes"], q["c2"], n, k)
+    ref = O.linear_fwd_multi(wd, [(a.float().numpy(), b.float().numpy(), al, r) for a, b, al in ads], idx,
+                             x.float().numpy())
+    qg = bd.quantize(w.cuda())
+    y = bd.linear_fwd_multi(qg, [(a.cuda(), b.cuda(), al) for a, b, al in ads], idx, x.cuda(), y_dtype=torch.float32)
+    torch.cuda.synchronize()
+    _check(f"y {n}x{k} m={m}", y, ref)
+    # the adapters' own contribution, alone
+    y0 = bd.linear_fwd_multi(qg, [(a.cuda(), torch.zeros_like(b).cuda(), al) for a, b, al in ads], idx, x.cuda(),
+                             y_dtype=torch.float32)
+    torch.cuda.synchronize()
+    _check("lora part", y - y0, ref - x.float().numpy().astype(np.float64) @ wd.astype(np.float64).T)
