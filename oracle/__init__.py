@@ -38,6 +38,9 @@ from .nf4_oracle import (  # noqa: F401
     linear_fwd,
     linear_bwd,
     linear_fwd_multi,
+    unpack_keep,
+    linear_fwd_dropout,
+    linear_bwd_dropout,
     merged_weight,
     merge_export,
     adamw_step,

@@ -40,6 +40,8 @@ Readings where the pages are silent or loose (each also listed in the design doc):
 * LoRA scale s = fl32(alpha) / fl32(r); y = X W'^T + s (X A^T) B^T.
 * Merged export: the 16-bit weight a page says merging needs is bf16, the
   round-to-nearest-even of the exact W' + s B A (one rounding).
+* LoRA dropout acts on the adapter branch's input only: D(X) = X * keep / (1-p)
+  with a drawn keep mask passed in (bit j % 8 of byte j // 8 of each row).
 * Adapter optimiser: the pages name Adam's per-parameter momentum and variance
   but give no update rule; the step is decoupled-weight-decay Adam (AdamW,
   Loshchilov and Hutter) with bias correction, the form torch.optim.AdamW uses.
@@ -355,6 +357,47 @@ def linear_bwd(w_dq: np.ndarray, a: np.ndarray, b: np.ndarray, x: np.ndarray,
     dx = dy64 @ np.asarray(w_dq, dtype=np.float64) + s * (u @ a64)
     da = s * (u.T @ x64)
     db = s * (dy64.T @ np.asarray(t, dtype=np.float64))
+    return dx, da, db
+
+
+def unpack_keep(keep_bits: np.ndarray, m: int, k: int) -> np.ndarray:
+    """Keep mask [m, k] (bool) from its packed form: bit (j % 8) of byte j // 8 of row i."""
+    bits = np.asarray(keep_bits, np.uint8).reshape(m, k // 8)
+    return ((bits[:, :, None] >> np.arange(8, dtype=np.uint8)) & 1).reshape(m, k).astype(bool)
+
+
+def linear_fwd_dropout(w_dq: np.ndarray, a: np.ndarray, b: np.ndarray, x: np.ndarray, keep: np.ndarray,
+                       p: float, alpha: float, r: int):
+    """Forward with dropout on the LoRA input (lora_dropout):
+    y = X W'^T + s (D(X) A^T) B^T,  D(X) = X * keep / (1 - p).  Returns (y, T = D(X) A^T).
+
+    [EZ] "Low-Rank Adaptation (LoRA)": the LoRA configuration of its example sets
+    lora_dropout; the dropped input feeds only the adapter branch.  keep is the
+    drawn mask (passed in; 1 keeps an element).
+    """
+    s = lora_scale(alpha, r)
+    x64 = np.asarray(x, np.float64)
+    xd = x64 * np.asarray(keep, np.float64) / (1.0 - p)
+    t = xd @ np.asarray(a, np.float64).T
+    y = x64 @ np.asarray(w_dq, np.float64).T + s * (t @ np.asarray(b, np.float64).T)
+    return y, t
+
+
+def linear_bwd_dropout(w_dq: np.ndarray, a: np.ndarray, b: np.ndarray, x: np.ndarray, dy: np.ndarray,
+                       keep: np.ndarray, p: float, alpha: float, r: int):
+    """Gradients of linear_fwd_dropout for upstream dY, float64:
+    U = dY B;  dX = dY W' + s (U A) * keep / (1 - p);  dA = s U^T D(X);  dB = s dY^T D(X) A^T."""
+    s = lora_scale(alpha, r)
+    x64 = np.asarray(x, np.float64)
+    dy64 = np.asarray(dy, np.float64)
+    a64 = np.asarray(a, np.float64)
+    b64 = np.asarray(b, np.float64)
+    kp = np.asarray(keep, np.float64) / (1.0 - p)
+    xd = x64 * kp
+    u = dy64 @ b64
+    dx = dy64 @ np.asarray(w_dq, np.float64) + s * (u @ a64) * kp
+    da = s * (u.T @ xd)
+    db = s * (dy64.T @ (xd @ a64.T))
     return dx, da, db
 
 

@@ -553,3 +553,61 @@ def test_multi_adapter_forward_reduces_and_separates():
         assert np.allclose(ym[t], (y1 if i == 0 else y2)[t], rtol=1e-13, atol=1e-13)
     # and two different adapters give different outputs
     assert not np.allclose(ym[0], y1[0])
+
+
+def _dropout_case(seed, m=6, n=9, k=24, r=3, p=0.25):
+    rng = np.random.default_rng(seed)
+    w, a, b, x, dy = _tiny_linear(seed, m=m, n=n, k=k, r=r)
+    keep = rng.random((m, k)) >= p
+    return w, a, b, x, dy, keep, p
+
+
+def test_keep_mask_packing_layout():
+    rng = np.random.default_rng(1)
+    keep = rng.random((3, 40)) < 0.5
+    packed = np.zeros((3, 5), np.uint8)
+    for i in range(3):
+        for j in range(40):
+            if keep[i, j]:
+                packed[i, j // 8] |= np.uint8(1 << (j % 8))
+    assert np.array_equal(O.unpack_keep(packed, 3, 40), keep)
+
+
+def test_dropout_with_nothing_dropped_is_the_plain_layer():
+    w, a, b, x, dy, _, _ = _dropout_case(2)
+    keep = np.ones(x.shape, bool)
+    y, t = O.linear_fwd_dropout(w, a, b, x, keep, 0.0, 6.0, 3)
+    y0, t0 = O.linear_fwd(w, a, b, x, 6.0, 3)
+    assert np.allclose(y, y0, rtol=1e-14, atol=1e-14) and np.allclose(t, t0, rtol=1e-14, atol=1e-14)
+    for g1, g0 in zip(O.linear_bwd_dropout(w, a, b, x, dy, keep, 0.0, 6.0, 3), O.linear_bwd(w, a, b, x, dy, 6.0, 3)):
+        assert np.allclose(g1, g0, rtol=1e-13, atol=1e-13)
+
+
+def test_dropout_with_everything_dropped_removes_the_adapter():
+    w, a, b, x, dy, _, p = _dropout_case(3)
+    keep = np.zeros(x.shape, bool)
+    y, t = O.linear_fwd_dropout(w, a, b, x, keep, p, 6.0, 3)
+    assert not t.any() and np.allclose(y, x @ w.T, rtol=1e-14, atol=1e-14)
+    dx, da, db = O.linear_bwd_dropout(w, a, b, x, dy, keep, p, 6.0, 3)
+    assert not da.any() and not db.any() and np.allclose(dx, dy @ w, rtol=1e-14, atol=1e-14)
+
+
+def test_dropout_gradients_by_finite_differences():
+    w, a, b, x, dy, keep, p = _dropout_case(4)
+
+    def loss(x_, a_, b_):
+        y, _ = O.linear_fwd_dropout(w, a_, b_, x_, keep, p, 6.0, 3)
+        return float(np.sum(y * dy))
+
+    dx, da, db = O.linear_bwd_dropout(w, a, b, x, dy, keep, p, 6.0, 3)
+    h = 1e-6
+    for arr, grad, which in ((x, dx, 0), (a, da, 1), (b, db, 2)):
+        for idx in [(0, 0), (1, 2), (arr.shape[0] - 1, arr.shape[1] - 1), (2, arr.shape[1] // 2)]:
+            plus, minus = arr.copy(), arr.copy()
+            plus[idx] += h
+            minus[idx] -= h
+            args_p = [x, a, b]
+            args_m = [x, a, b]
+            args_p[which], args_m[which] = plus, minus
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * h)
+            assert abs(fd - grad[idx]) < 1e-6 * max(1.0, abs(fd))
