@@ -71,6 +71,11 @@ def lib():
         "qlora_linear_fwd": (ctypes.c_int, [pT, pL, vp, i64, vp, ctypes.c_int, vp, vp, sz, vp]),
         "qlora_linear_bwd": (ctypes.c_int, [pT, pL, vp, vp, i64, vp, vp, ctypes.c_int, vp, vp, ctypes.c_int, vp,
                                             sz, vp]),
+        "qlora_workspace_bytes_dropout": (sz, [i64, i64, i64, i32, ctypes.c_int]),
+        "qlora_linear_fwd_dropout": (ctypes.c_int, [pT, pL, vp, vp, ctypes.c_float, i64, vp, ctypes.c_int, vp, vp,
+                                                    sz, vp]),
+        "qlora_linear_bwd_dropout": (ctypes.c_int, [pT, pL, vp, vp, vp, ctypes.c_float, i64, vp, vp, ctypes.c_int,
+                                                    vp, vp, ctypes.c_int, vp, sz, vp]),
         "qlora_linear_fwd_multi": (ctypes.c_int, [pT, pL, i32, ctypes.POINTER(i32), vp, i64, vp, ctypes.c_int, vp,
                                                   sz, vp]),
         "qlora_lora_merge": (ctypes.c_int, [pT, pL, vp, vp]),
@@ -291,3 +296,43 @@ def linear_fwd_multi(q: NF4Weight, adapters, adapter_of_token, X, y_dtype=torch.
                                         _dtype_code(Y.dtype), _ptr(ws), ws.numel(), _stream(stream)),
            "qlora_linear_fwd_multi")
     return Y
+
+
+def workspace_bytes_dropout(m: int, n: int, k: int, r: int, backward: bool) -> int:
+    return int(lib().qlora_workspace_bytes_dropout(m, n, k, r, 1 if backward else 0))
+
+
+def linear_fwd_dropout(q: NF4Weight, A, B, alpha: float, X, keep: torch.Tensor, p: float, y_dtype=torch.bfloat16,
+                       save_t: bool = True, ws: torch.Tensor | None = None, stream=None):
+    """Forward with LoRA dropout on the adapter input; keep is the packed
+    uint8 [M, K/8] mask.  Returns (Y, T pair or None) as linear_fwd."""
+    M, K = X.shape
+    r = A.shape[0]
+    assert keep.dtype == torch.uint8 and keep.is_contiguous() and tuple(keep.shape) == (M, K // 8)
+    Y = torch.empty(M, q.rows, dtype=y_dtype, device=X.device)
+    T = torch.empty(2, M, r, dtype=torch.bfloat16, device=X.device) if save_t else None
+    if ws is None:
+        ws = new_workspace(workspace_bytes_dropout(M, q.rows, q.cols, r, False), X.device)
+    t, ad = q.c_struct(), _lora(A, B, alpha)
+    _check(lib().qlora_linear_fwd_dropout(ctypes.byref(t), ctypes.byref(ad), _ptr(X), _ptr(keep), float(p), M,
+                                          _ptr(Y), _dtype_code(Y.dtype), _ptr(T), _ptr(ws), ws.numel(),
+                                          _stream(stream)), "qlora_linear_fwd_dropout")
+    return Y, T
+
+
+def linear_bwd_dropout(q: NF4Weight, A, B, alpha: float, X, dY, keep: torch.Tensor, p: float, T=None,
+                       dx_dtype=torch.bfloat16, grad_dtype=torch.bfloat16, ws: torch.Tensor | None = None, stream=None):
+    """Gradients (dX, dA, dB) of linear_fwd_dropout for upstream dY."""
+    M, K = X.shape
+    r = A.shape[0]
+    dX = torch.empty(M, K, dtype=dx_dtype, device=X.device)
+    dA = torch.empty(r, K, dtype=grad_dtype, device=X.device)
+    dB = torch.empty(q.rows, r, dtype=grad_dtype, device=X.device)
+    if ws is None:
+        ws = new_workspace(workspace_bytes_dropout(M, q.rows, q.cols, r, True), X.device)
+    t, ad = q.c_struct(), _lora(A, B, alpha)
+    _check(lib().qlora_linear_bwd_dropout(ctypes.byref(t), ctypes.byref(ad), _ptr(X), _ptr(dY), _ptr(keep), float(p),
+                                          M, _ptr(T), _ptr(dX), _dtype_code(dx_dtype), _ptr(dA), _ptr(dB),
+                                          _dtype_code(grad_dtype), _ptr(ws), ws.numel(), _stream(stream)),
+           "qlora_linear_bwd_dropout")
+    return dX, dA, dB

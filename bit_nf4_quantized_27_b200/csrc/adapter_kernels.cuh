@@ -154,6 +154,27 @@ __global__ void __launch_bounds__(kMergeThreads) nf4_lora_merge_kernel(
 }
 
 // ---------------------------------------------------------------------------
+// LoRA dropout input: Xm = X * keep (bf16, exact: each element is X or 0), keep
+// packed one bit per element (bit k % 8 of byte k / 8 of each row).  The
+// 1 / (1 - p) factor is applied to the products computed from Xm.  One thread
+// per 8 elements (16 bytes of X, one mask byte).
+// ---------------------------------------------------------------------------
+__global__ void keep_mask_kernel(const __nv_bfloat16 *__restrict__ X, const uint8_t *__restrict__ keep,
+                                 int64_t n8, __nv_bfloat16 *__restrict__ Xm) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
+    const uint32_t b = keep[i];
+    uint4 v = __ldg(reinterpret_cast<const uint4 *>(X) + i);
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t lo = (b >> (2 * e)) & 1u ? 0x0000ffffu : 0u, hi = (b >> (2 * e + 1)) & 1u ? 0xffff0000u : 0u;
+      w[e] &= lo | hi;
+    }
+    reinterpret_cast<uint4 *>(Xm)[i] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // AdamW on flat float32 arrays (parameters, gradients, momentum, variance), in
 // the order of the definition:
 //   m = b1 m + (1 - b1) g;  v = b2 v + (1 - b2) g^2;

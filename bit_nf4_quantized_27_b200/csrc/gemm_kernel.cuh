@@ -36,6 +36,10 @@ struct GemmArgs {
                      // writes raw fp32 partial planes to `part` [ksplit][M_rows][N_cols]
   float *part;
   int k_per;         // K steps per split when ksplit > 1 (no split is empty)
+  // masked accumulate (non-transposed `out` only): out += v * out_scale * (keep bit ? keep_scale : 0),
+  // keep = [M_rows][N_cols / 8] bits, bit (col % 8) of byte col / 8
+  const uint8_t *keep;
+  float keep_scale;
   int lora_steps;    // extra K steps of 64 for the LoRA block (0 = none)
   int lora_r;        // LoRA rank (bounds the B2 rows/cols read by the dequant warps)
   // outputs (each optional): `out` (f32 or bf16, scaled by out_scale, optionally
@@ -149,9 +153,36 @@ __device__ __forceinline__ void load_row128(const __nv_bfloat16 *src, int valid_
 
 constexpr int kGemmDequantThreads = 256;  // NF4 producer threads (warps 8..15)
 
+// out[row, col0 + j] += v_j * out_scale * (keep bit ? keep_scale : 0), j < ncol.
+__device__ __forceinline__ void masked_accumulate32(const GemmArgs &args, int row, int col0, int ncol,
+                                                 const uint32_t (&v)[32]) {
+  const uint8_t *kp = args.keep + (int64_t)row * (args.N_cols / 8) + col0 / 8;
+  uint32_t bits = 0;
+#pragma unroll
+  for (int b = 0; b < 4; ++b)
+    if (8 * b < ncol) bits |= static_cast<uint32_t>(kp[b]) << (8 * b);
+  if (args.out_f32) {
+    float *o = reinterpret_cast<float *>(args.out) + (int64_t)row * args.ldo + col0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < ncol && ((bits >> j) & 1u)) o[j] += __uint_as_float(v[j]) * args.out_scale * args.keep_scale;
+  } else {
+    __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(args.out) + (int64_t)row * args.ldo + col0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < ncol && ((bits >> j) & 1u))
+        o[j] = __float2bfloat16_rn(__bfloat162float(o[j]) +
+                                   __uint_as_float(v[j]) * args.out_scale * args.keep_scale);
+  }
+}
+
 // Stores one 32-column chunk of accumulator row `row` (v = fp32 bit patterns).
 __device__ __forceinline__ void store_chunk32(const GemmArgs &args, int row, int col0, int ncol,
                                               const uint32_t (&v)[32]) {
+  if (args.keep) {
+    masked_accumulate32(args, row, col0, ncol, v);
+    return;
+  }
   const bool full = ncol == 32;
   if (args.out) {
     if (!args.out_transpose) {

@@ -809,14 +809,16 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
 // both bf16.  Inside a block, k is permuted identically for A and X (thread quad
 // q owns k in [16q, 16q + 16)), so each thread reads two 16-byte vectors per row
 // and block, and a warp has kLoraDownBlocks blocks of loads in flight before its
-// first MMA.  The partials are summed over the warps in a fixed order.  Writes
-// s*T (bf16) and, if T_hi is given, (T_hi, T_lo).
+// first MMA.  The partials are summed over the warps in a fixed order and
+// multiplied by t_scale (1, or 1 / (1 - p) for a dropped-out X).  Writes s*T
+// (bf16) and, if T_hi is given, (T_hi, T_lo).
 constexpr int kLoraDownThreads = 256;
 constexpr int kLoraDownBlocks = 4;
 template <int NG>
 __global__ void __launch_bounds__(kLoraDownThreads, 1) lora_down_small_kernel(
     const __nv_bfloat16 *__restrict__ X, const __nv_bfloat16 *__restrict__ A, int M, int64_t K, int r, float s,
-    __nv_bfloat16 *__restrict__ sT, __nv_bfloat16 *__restrict__ T_hi, __nv_bfloat16 *__restrict__ T_lo) {
+    __nv_bfloat16 *__restrict__ sT, __nv_bfloat16 *__restrict__ T_hi, __nv_bfloat16 *__restrict__ T_lo,
+    float t_scale) {
   griddep_launch_dependents();
   __shared__ float red[kLoraDownThreads / 32][16][kGemvMaxM];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -881,6 +883,7 @@ __global__ void __launch_bounds__(kLoraDownThreads, 1) lora_down_small_kernel(
     float v = 0.0f;
 #pragma unroll
     for (int w = 0; w < kLoraDownThreads / 32; ++w) v += red[w][jr][t];
+    v *= t_scale;  // 1, or 1 / (1 - p) when the input rows were dropped out
     const int64_t o = (int64_t)t * r + j0 + jr;
     sT[o] = __float2bfloat16_rn(v * s);
     if (T_hi) {

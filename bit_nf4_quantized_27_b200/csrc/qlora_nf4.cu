@@ -205,7 +205,8 @@ qlora_status launch_rank_gemm(const CUtensorMap &tmA, const CUtensorMap &tmB, Ge
 }
 
 qlora_status run_lora_down(const void *X, const qlora_lora *ad, int64_t M, int64_t K, float s, void *sT,
-                           void *T_hi, void *T_lo, float *part, uint32_t *status, int dev, int sms, cudaStream_t st) {
+                           void *T_hi, void *T_lo, float *part, uint32_t *status, int dev, int sms, cudaStream_t st,
+                           float t_scale = 1.0f) {
   CUtensorMap tmX, tmA;
   if (!tmap_bf16(&tmX, X, K, M, 64, 128) || !tmap_bf16(&tmA, ad->A, K, ad->r, 64, 64)) return QLORA_ERR_CUDA;
   GemmArgs g{};
@@ -215,11 +216,11 @@ qlora_status run_lora_down(const void *X, const qlora_lora *ad, int64_t M, int64
   g.out = sT;
   g.ldo = ad->r;
   g.out_f32 = 0;
-  g.out_scale = s;
+  g.out_scale = s * t_scale;
   g.out_hi = static_cast<__nv_bfloat16 *>(T_hi);
   g.out_lo = static_cast<__nv_bfloat16 *>(T_lo);
   g.ld_hl = ad->r;
-  g.hl_scale = 1.0f;
+  g.hl_scale = t_scale;
   g.status = status;
   return launch_rank_gemm<false>(tmX, tmA, g, part, dev, sms, st);
 }
@@ -245,6 +246,217 @@ float *split_part(void *ws, size_t ws_bytes, int64_t M, int64_t N, int64_t K, in
   if (ws_bytes < lo + split_part_bytes(M, r)) return nullptr;
   return reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + lo);
 }
+
+// Forward on a checked workspace: the base product reads X, the adapter branch
+// reads Xl (X, or its dropped-out copy) and scales T by t_scale; part is the
+// nullable K-split scratch.
+qlora_status fwd_impl(const qlora_nf4_tensor *W, const qlora_lora *ad, const void *X, const void *Xl, float t_scale,
+                      int64_t M, void *Y, qlora_dtype y_dtype, void *T_save, void *ws, float *part,
+                      qlora_stream_t stream) {
+  qlora_status s;
+  const int64_t N = W->rows, K = W->cols;
+  int dev, sms;
+  if ((s = check_device(&dev, &sms)) != QLORA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const float sc = ad->alpha / static_cast<float>(ad->r);
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  void *sT = wsb + QLORA_STATUS_BYTES;
+  const size_t mr = align256(static_cast<size_t>(M) * ad->r * 2);
+
+  if (M <= kGemvMaxM) {
+    __nv_bfloat16 *th = static_cast<__nv_bfloat16 *>(T_save);
+    auto down = M > 8 ? lora_down_small_kernel<2> : lora_down_small_kernel<1>;
+    down<<<(ad->r + 15) / 16, kLoraDownThreads, 0, st>>>(static_cast<const __nv_bfloat16 *>(Xl),
+                                                        static_cast<const __nv_bfloat16 *>(ad->A), (int)M, K, ad->r, sc,
+                                                        static_cast<__nv_bfloat16 *>(sT), th,
+                                                        th ? th + M * ad->r : nullptr, t_scale);
+    if ((s = launch_status()) != QLORA_OK) return s;
+    GemvArgs g{};
+    g.codes = W->codes; g.scale_codes = W->scale_codes; g.c2 = W->c2;
+    g.N = N; g.K = K; g.M = (int)M;
+    g.X = static_cast<const __nv_bfloat16 *>(X);
+    g.sT = static_cast<const __nv_bfloat16 *>(sT);
+    g.B = static_cast<const __nv_bfloat16 *>(ad->B);
+    g.r = ad->r;
+    g.Y = Y; g.y_f32 = y_dtype == QLORA_F32;
+    g.partial = reinterpret_cast<float *>(wsb + QLORA_STATUS_BYTES + mr);
+    g.status = status_ptr(ws);
+    CUtensorMap tmc;
+    const bool staged = gemv_bulk_ok(N, K) &&
+                        tmap_codes_gemv(&tmc, W->codes, N, K, static_cast<uint32_t>((K < 4096 ? K : 4096) / 256));
+    return launch_gemv(g, staged ? &tmc : nullptr, dev, sms, st);
+  }
+
+  {
+    __nv_bfloat16 *th = static_cast<__nv_bfloat16 *>(T_save);
+    if ((s = run_lora_down(Xl, ad, M, K, sc, sT, th, th ? th + M * ad->r : nullptr, part, status_ptr(ws), dev, sms,
+                           st, t_scale)) != QLORA_OK)
+      return s;
+  }
+
+  CUtensorMap tmX, tmCodes, tmT, tmCodesPair;
+  if (!tmap_bf16(&tmX, X, K, M, 64, 128) || !tmap_bf16(&tmT, sT, ad->r, M, 64, 128) ||
+      !make_tmap(&tmCodes, W->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, K / 2, 32, 256, false) ||
+      !make_tmap(&tmCodesPair, W->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, K / 2, 32, 128, false))
+    return QLORA_ERR_CUDA;
+  GemmArgs g{};
+  g.M_rows = (int)M;
+  g.N_cols = (int)N;
+  g.k_steps = (int)(K / 64);
+  g.lora_steps = (ad->r + 63) / 64;
+  g.lora_r = ad->r;
+  g.out = Y;
+  g.ldo = N;
+  g.out_f32 = y_dtype == QLORA_F32;
+  g.out_scale = 1.0f;
+  g.scale_codes = W->scale_codes;
+  g.c2 = W->c2;
+  g.w_rows = N;
+  g.w_cols = K;
+  g.lora_b2 = static_cast<const __nv_bfloat16 *>(ad->B);
+  g.lora_ld = ad->r;
+  g.status = status_ptr(ws);
+  if (M >= kPairMinRows) {
+    s = launch_gemm_pair<false, kFusedMT>(tmX, tmT, tmCodesPair, g, dev, st);
+    if (s != QLORA_ERR_UNSUPPORTED_SHAPE) return s;
+  }
+  return launch_gemm<false, false, true, 256, kFusedMT>(tmX, tmX, tmT, tmX, tmCodes, g, dev, sms, st);
+}
+
+// Backward on a checked workspace: dA and a recomputed T read Xl (X, or its
+// dropped-out copy) with t_scale; keep (nullable) masks the adapter term of dX.
+qlora_status bwd_impl(const qlora_nf4_tensor *W, const qlora_lora *ad, const void *X, const void *Xl, float t_scale,
+                      const void *keep, const void *dY, int64_t M, const void *T_saved, void *dX, qlora_dtype dx_dtype,
+                      void *dA, void *dB, qlora_dtype grad_dtype, void *ws, float *part, qlora_stream_t stream) {
+  qlora_status s;
+  const int64_t N = W->rows, K = W->cols;
+  (void)X;
+  int dev, sms;
+  if ((s = check_device(&dev, &sms)) != QLORA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const float sc = ad->alpha / static_cast<float>(ad->r);
+  const int r = ad->r;
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  const size_t mr = align256(static_cast<size_t>(M) * r * 2);
+  void *sU_hi = wsb + QLORA_STATUS_BYTES;
+  void *sU_lo = wsb + QLORA_STATUS_BYTES + mr;
+  uint32_t *status = status_ptr(ws);
+
+  const void *T_hi = T_saved;
+  const void *T_lo = T_saved ? static_cast<const __nv_bfloat16 *>(T_saved) + M * r : nullptr;
+  if (!T_saved) {
+    void *th = wsb + QLORA_STATUS_BYTES + 2 * mr, *tl = wsb + QLORA_STATUS_BYTES + 3 * mr;
+    if ((s = run_lora_down(Xl, ad, M, K, sc, nullptr, th, tl, part, status, dev, sms, st, t_scale)) != QLORA_OK)
+      return s;
+    T_hi = th;
+    T_lo = tl;
+  }
+  // U = dY B, kept as the bf16 pair (hi, lo) of s*U
+  {
+    CUtensorMap tmDY, tmB;
+    if (!tmap_bf16(&tmDY, dY, N, M, 64, 128) || !tmap_bf16(&tmB, ad->B, r, N, 64, 64)) return QLORA_ERR_CUDA;
+    GemmArgs g{};
+    g.M_rows = (int)M;
+    g.N_cols = r;
+    g.k_steps = (int)((N + 63) / 64);
+    g.out_hi = static_cast<__nv_bfloat16 *>(sU_hi);
+    g.out_lo = static_cast<__nv_bfloat16 *>(sU_lo);
+    g.ld_hl = r;
+    g.hl_scale = sc;
+    g.status = status;
+    if ((s = launch_rank_gemm<true>(tmDY, tmB, g, part, dev, sms, st)) != QLORA_OK) return s;
+  }
+  // dX = dY W' + (s U) A
+  {
+    CUtensorMap tmDY, tmU, tmCodes, tmCodesPair;
+    if (!tmap_bf16(&tmDY, dY, N, M, 64, 128) || !tmap_bf16(&tmU, sU_hi, r, M, 64, 128) ||
+        !make_tmap(&tmCodes, W->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, K / 2, 128, 64, false) ||
+        !make_tmap(&tmCodesPair, W->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, K / 2, 64, 64, false))
+      return QLORA_ERR_CUDA;
+    GemmArgs g{};
+    g.M_rows = (int)M;
+    g.N_cols = (int)K;
+    g.k_steps = (int)((N + 63) / 64);
+    g.lora_steps = keep ? 0 : (r + 63) / 64;  // with dropout the adapter term is added masked, below
+    g.lora_r = r;
+    g.out = dX;
+    g.ldo = K;
+    g.out_f32 = dx_dtype == QLORA_F32;
+    g.out_scale = 1.0f;
+    g.scale_codes = W->scale_codes;
+    g.c2 = W->c2;
+    g.w_rows = N;
+    g.w_cols = K;
+    g.lora_b2 = static_cast<const __nv_bfloat16 *>(ad->A);
+    g.lora_ld = K;
+    g.status = status;
+    s = M >= kPairMinRows ? launch_gemm_pair<true, kFusedMT>(tmDY, tmU, tmCodesPair, g, dev, st)
+                          : QLORA_ERR_UNSUPPORTED_SHAPE;
+    if (s == QLORA_ERR_UNSUPPORTED_SHAPE)
+      s = launch_gemm<false, true, true, 256, kFusedMT>(tmDY, tmDY, tmU, tmDY, tmCodes, g, dev, sms, st);
+    if (s != QLORA_OK) return s;
+  }
+  // dropout: dX += keep * ((s U) A) / (1 - p)
+  if (keep) {
+    CUtensorMap tmU, tmAl;
+    if (!tmap_bf16(&tmU, sU_hi, r, M, 64, 128) || !tmap_bf16(&tmAl, ad->A, K, r, 64, 64)) return QLORA_ERR_CUDA;
+    GemmArgs g{};
+    g.M_rows = (int)M;
+    g.N_cols = (int)K;
+    g.k_steps = (r + 63) / 64;
+    g.out = dX;
+    g.ldo = K;
+    g.out_f32 = dx_dtype == QLORA_F32;
+    g.out_scale = 1.0f;
+    g.keep = static_cast<const uint8_t *>(keep);
+    g.keep_scale = t_scale;
+    g.status = status;
+    if ((s = launch_gemm<false, true, false, 128, 1>(tmU, tmAl, tmU, tmU, tmU, g, dev, sms, st)) != QLORA_OK)
+      return s;
+  }
+  // dA^T [K, r] = X^T (s U_hi + s U_lo)  -> stored transposed into dA [r, K]
+  {
+    CUtensorMap tmXt, tmUh, tmUl;
+    if (!tmap_bf16(&tmXt, Xl, K, M, 64, 64) || !tmap_bf16(&tmUh, sU_hi, r, M, 64, 64) ||
+        !tmap_bf16(&tmUl, sU_lo, r, M, 64, 64))
+      return QLORA_ERR_CUDA;
+    GemmArgs g{};
+    g.M_rows = (int)K;
+    g.N_cols = r;
+    g.k_steps = (int)((M + 63) / 64);
+    g.hilo_cols = 1;
+    g.out = dA;
+    g.ldo = K;
+    g.out_f32 = grad_dtype == QLORA_F32;
+    g.out_transpose = 1;
+    g.out_scale = t_scale;
+    g.status = status;
+    if ((s = launch_gemm<true, true, false, 128, 1>(tmXt, tmUh, tmXt, tmUl, tmXt, g, dev, sms, st)) != QLORA_OK)
+      return s;
+  }
+  // dB [N, r] = s dY^T (T_hi + T_lo)
+  {
+    CUtensorMap tmDYt, tmTh, tmTl;
+    if (!tmap_bf16(&tmDYt, dY, N, M, 64, 64) || !tmap_bf16(&tmTh, T_hi, r, M, 64, 64) ||
+        !tmap_bf16(&tmTl, T_lo, r, M, 64, 64))
+      return QLORA_ERR_CUDA;
+    GemmArgs g{};
+    g.M_rows = (int)N;
+    g.N_cols = r;
+    g.k_steps = (int)((M + 63) / 64);
+    g.hilo_cols = 1;
+    g.out = dB;
+    g.ldo = r;
+    g.out_f32 = grad_dtype == QLORA_F32;
+    g.out_scale = sc;
+    g.status = status;
+    if ((s = launch_gemm<true, true, false, 128, 1>(tmDYt, tmTh, tmDYt, tmTl, tmDYt, g, dev, sms, st)) != QLORA_OK)
+      return s;
+  }
+  return QLORA_OK;
+}
+
+
 }  // namespace
 
 extern "C" {
@@ -336,73 +548,8 @@ qlora_status qlora_linear_fwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
     return QLORA_ERR_MISALIGNED;
   const int64_t N = W->rows, K = W->cols;
   if (ws_bytes < min_workspace_bytes(M, N, K, ad->r, 0)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
-  int dev, sms;
-  if ((s = check_device(&dev, &sms)) != QLORA_OK) return s;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const float sc = ad->alpha / static_cast<float>(ad->r);
-  uint8_t *wsb = static_cast<uint8_t *>(ws);
-  void *sT = wsb + QLORA_STATUS_BYTES;
-  const size_t mr = align256(static_cast<size_t>(M) * ad->r * 2);
-
-  if (M <= kGemvMaxM) {
-    __nv_bfloat16 *th = static_cast<__nv_bfloat16 *>(T_save);
-    auto down = M > 8 ? lora_down_small_kernel<2> : lora_down_small_kernel<1>;
-    down<<<(ad->r + 15) / 16, kLoraDownThreads, 0, st>>>(static_cast<const __nv_bfloat16 *>(X),
-                                                        static_cast<const __nv_bfloat16 *>(ad->A), (int)M, K, ad->r, sc,
-                                                        static_cast<__nv_bfloat16 *>(sT), th,
-                                                        th ? th + M * ad->r : nullptr);
-    if ((s = launch_status()) != QLORA_OK) return s;
-    GemvArgs g{};
-    g.codes = W->codes; g.scale_codes = W->scale_codes; g.c2 = W->c2;
-    g.N = N; g.K = K; g.M = (int)M;
-    g.X = static_cast<const __nv_bfloat16 *>(X);
-    g.sT = static_cast<const __nv_bfloat16 *>(sT);
-    g.B = static_cast<const __nv_bfloat16 *>(ad->B);
-    g.r = ad->r;
-    g.Y = Y; g.y_f32 = y_dtype == QLORA_F32;
-    g.partial = reinterpret_cast<float *>(wsb + QLORA_STATUS_BYTES + mr);
-    g.status = status_ptr(ws);
-    CUtensorMap tmc;
-    const bool staged = gemv_bulk_ok(N, K) &&
-                        tmap_codes_gemv(&tmc, W->codes, N, K, static_cast<uint32_t>((K < 4096 ? K : 4096) / 256));
-    return launch_gemv(g, staged ? &tmc : nullptr, dev, sms, st);
-  }
-
-  {
-    __nv_bfloat16 *th = static_cast<__nv_bfloat16 *>(T_save);
-    if ((s = run_lora_down(X, ad, M, K, sc, sT, th, th ? th + M * ad->r : nullptr,
-                           split_part(ws, ws_bytes, M, N, K, ad->r, 0), status_ptr(ws), dev, sms, st)) !=
-        QLORA_OK)
-      return s;
-  }
-
-  CUtensorMap tmX, tmCodes, tmT, tmCodesPair;
-  if (!tmap_bf16(&tmX, X, K, M, 64, 128) || !tmap_bf16(&tmT, sT, ad->r, M, 64, 128) ||
-      !make_tmap(&tmCodes, W->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, K / 2, 32, 256, false) ||
-      !make_tmap(&tmCodesPair, W->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, K / 2, 32, 128, false))
-    return QLORA_ERR_CUDA;
-  GemmArgs g{};
-  g.M_rows = (int)M;
-  g.N_cols = (int)N;
-  g.k_steps = (int)(K / 64);
-  g.lora_steps = (ad->r + 63) / 64;
-  g.lora_r = ad->r;
-  g.out = Y;
-  g.ldo = N;
-  g.out_f32 = y_dtype == QLORA_F32;
-  g.out_scale = 1.0f;
-  g.scale_codes = W->scale_codes;
-  g.c2 = W->c2;
-  g.w_rows = N;
-  g.w_cols = K;
-  g.lora_b2 = static_cast<const __nv_bfloat16 *>(ad->B);
-  g.lora_ld = ad->r;
-  g.status = status_ptr(ws);
-  if (M >= kPairMinRows) {
-    s = launch_gemm_pair<false, kFusedMT>(tmX, tmT, tmCodesPair, g, dev, st);
-    if (s != QLORA_ERR_UNSUPPORTED_SHAPE) return s;
-  }
-  return launch_gemm<false, false, true, 256, kFusedMT>(tmX, tmX, tmT, tmX, tmCodes, g, dev, sms, st);
+  return fwd_impl(W, ad, X, X, 1.0f, M, Y, y_dtype, T_save, ws, split_part(ws, ws_bytes, M, N, K, ad->r, 0),
+                  stream);
 }
 
 qlora_status qlora_linear_bwd(const qlora_nf4_tensor *W, const qlora_lora *ad, const void *X, const void *dY,
@@ -419,111 +566,87 @@ qlora_status qlora_linear_bwd(const qlora_nf4_tensor *W, const qlora_lora *ad, c
     return QLORA_ERR_MISALIGNED;
   const int64_t N = W->rows, K = W->cols;
   if (ws_bytes < min_workspace_bytes(M, N, K, ad->r, 1)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  return bwd_impl(W, ad, X, X, 1.0f, nullptr, dY, M, T_saved, dX, dx_dtype, dA, dB, grad_dtype, ws,
+                  split_part(ws, ws_bytes, M, N, K, ad->r, 1), stream);
+}
+
+size_t qlora_workspace_bytes_dropout(int64_t M, int64_t N, int64_t K, int32_t r, int for_backward) {
+  const size_t lo = min_workspace_bytes(M, N, K, r, for_backward);
+  if (lo == 0) return 0;
+  const size_t xm = align256(static_cast<size_t>(M) * static_cast<size_t>(K) * 2);
+  if (!for_backward && M <= kGemvMaxM) return lo + xm;
+  return lo + xm + split_part_bytes(M, r);
+}
+
+namespace {
+// X * keep into the workspace right after its minimum part; returns the copy and
+// the K-split scratch after it (null when the workspace has no room for it).
+qlora_status dropout_input(const void *X, const void *keep, int64_t M, int64_t N, int64_t K, int32_t r,
+                           int for_backward, void *ws, size_t ws_bytes, int sms, cudaStream_t st, void **Xm,
+                           float **part) {
+  const size_t lo = min_workspace_bytes(M, N, K, r, for_backward);
+  const size_t xm = align256(static_cast<size_t>(M) * static_cast<size_t>(K) * 2);
+  if (ws_bytes < lo + xm) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  uint8_t *wsb = static_cast<uint8_t *>(ws);
+  *Xm = wsb + lo;
+  *part = (for_backward || M > kGemvMaxM) && ws_bytes >= lo + xm + split_part_bytes(M, r)
+              ? reinterpret_cast<float *>(wsb + lo + xm)
+              : nullptr;
+  const int64_t n8 = M * K / 8;
+  const unsigned grid = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>((n8 + 255) / 256, (int64_t)sms * 8)));
+  keep_mask_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(X), static_cast<const uint8_t *>(keep), n8,
+                                         static_cast<__nv_bfloat16 *>(*Xm));
+  return launch_status();
+}
+}  // namespace
+
+qlora_status qlora_linear_fwd_dropout(const qlora_nf4_tensor *W, const qlora_lora *ad, const void *X, const void *keep,
+                                      float p, int64_t M, void *Y, qlora_dtype y_dtype, void *T_save, void *ws,
+                                      size_t ws_bytes, qlora_stream_t stream) {
+  qlora_status s = check_nf4(W);
+  if (s != QLORA_OK) return s;
+  if ((s = check_lora(ad)) != QLORA_OK) return s;
+  if (!X || !keep || !Y || !ws || M < 1 || M > (int64_t(1) << 30) || !valid_dtype(y_dtype) || !(p >= 0.0f && p < 1.0f))
+    return QLORA_ERR_INVALID_ARGUMENT;
+  if (W->rows % 8) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(X, 16) || !aligned(keep, 16) || !aligned(Y, 16) || !aligned(ws, 256) ||
+      (T_save && !aligned(T_save, 16)))
+    return QLORA_ERR_MISALIGNED;
+  const int64_t N = W->rows, K = W->cols;
+  if (ws_bytes < min_workspace_bytes(M, N, K, ad->r, 0)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   int dev, sms;
   if ((s = check_device(&dev, &sms)) != QLORA_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const float sc = ad->alpha / static_cast<float>(ad->r);
-  const int r = ad->r;
-  uint8_t *wsb = static_cast<uint8_t *>(ws);
-  const size_t mr = align256(static_cast<size_t>(M) * r * 2);
-  void *sU_hi = wsb + QLORA_STATUS_BYTES;
-  void *sU_lo = wsb + QLORA_STATUS_BYTES + mr;
-  uint32_t *status = status_ptr(ws);
-  float *part = split_part(ws, ws_bytes, M, N, K, r, 1);
+  void *Xm;
+  float *part;
+  if ((s = dropout_input(X, keep, M, N, K, ad->r, 0, ws, ws_bytes, sms, st, &Xm, &part)) != QLORA_OK) return s;
+  return fwd_impl(W, ad, X, Xm, 1.0f / (1.0f - p), M, Y, y_dtype, T_save, ws, part, stream);
+}
 
-  const void *T_hi = T_saved;
-  const void *T_lo = T_saved ? static_cast<const __nv_bfloat16 *>(T_saved) + M * r : nullptr;
-  if (!T_saved) {
-    void *th = wsb + QLORA_STATUS_BYTES + 2 * mr, *tl = wsb + QLORA_STATUS_BYTES + 3 * mr;
-    if ((s = run_lora_down(X, ad, M, K, sc, nullptr, th, tl, part, status, dev, sms, st)) != QLORA_OK) return s;
-    T_hi = th;
-    T_lo = tl;
-  }
-  // U = dY B, kept as the bf16 pair (hi, lo) of s*U
-  {
-    CUtensorMap tmDY, tmB;
-    if (!tmap_bf16(&tmDY, dY, N, M, 64, 128) || !tmap_bf16(&tmB, ad->B, r, N, 64, 64)) return QLORA_ERR_CUDA;
-    GemmArgs g{};
-    g.M_rows = (int)M;
-    g.N_cols = r;
-    g.k_steps = (int)((N + 63) / 64);
-    g.out_hi = static_cast<__nv_bfloat16 *>(sU_hi);
-    g.out_lo = static_cast<__nv_bfloat16 *>(sU_lo);
-    g.ld_hl = r;
-    g.hl_scale = sc;
-    g.status = status;
-    if ((s = launch_rank_gemm<true>(tmDY, tmB, g, part, dev, sms, st)) != QLORA_OK) return s;
-  }
-  // dX = dY W' + (s U) A
-  {
-    CUtensorMap tmDY, tmU, tmCodes, tmCodesPair;
-    if (!tmap_bf16(&tmDY, dY, N, M, 64, 128) || !tmap_bf16(&tmU, sU_hi, r, M, 64, 128) ||
-        !make_tmap(&tmCodes, W->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, K / 2, 128, 64, false) ||
-        !make_tmap(&tmCodesPair, W->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, K / 2, 64, 64, false))
-      return QLORA_ERR_CUDA;
-    GemmArgs g{};
-    g.M_rows = (int)M;
-    g.N_cols = (int)K;
-    g.k_steps = (int)((N + 63) / 64);
-    g.lora_steps = (r + 63) / 64;
-    g.lora_r = r;
-    g.out = dX;
-    g.ldo = K;
-    g.out_f32 = dx_dtype == QLORA_F32;
-    g.out_scale = 1.0f;
-    g.scale_codes = W->scale_codes;
-    g.c2 = W->c2;
-    g.w_rows = N;
-    g.w_cols = K;
-    g.lora_b2 = static_cast<const __nv_bfloat16 *>(ad->A);
-    g.lora_ld = K;
-    g.status = status;
-    s = M >= kPairMinRows ? launch_gemm_pair<true, kFusedMT>(tmDY, tmU, tmCodesPair, g, dev, st)
-                          : QLORA_ERR_UNSUPPORTED_SHAPE;
-    if (s == QLORA_ERR_UNSUPPORTED_SHAPE)
-      s = launch_gemm<false, true, true, 256, kFusedMT>(tmDY, tmDY, tmU, tmDY, tmCodes, g, dev, sms, st);
-    if (s != QLORA_OK) return s;
-  }
-  // dA^T [K, r] = X^T (s U_hi + s U_lo)  -> stored transposed into dA [r, K]
-  {
-    CUtensorMap tmXt, tmUh, tmUl;
-    if (!tmap_bf16(&tmXt, X, K, M, 64, 64) || !tmap_bf16(&tmUh, sU_hi, r, M, 64, 64) ||
-        !tmap_bf16(&tmUl, sU_lo, r, M, 64, 64))
-      return QLORA_ERR_CUDA;
-    GemmArgs g{};
-    g.M_rows = (int)K;
-    g.N_cols = r;
-    g.k_steps = (int)((M + 63) / 64);
-    g.hilo_cols = 1;
-    g.out = dA;
-    g.ldo = K;
-    g.out_f32 = grad_dtype == QLORA_F32;
-    g.out_transpose = 1;
-    g.out_scale = 1.0f;
-    g.status = status;
-    if ((s = launch_gemm<true, true, false, 128, 1>(tmXt, tmUh, tmXt, tmUl, tmXt, g, dev, sms, st)) != QLORA_OK)
-      return s;
-  }
-  // dB [N, r] = s dY^T (T_hi + T_lo)
-  {
-    CUtensorMap tmDYt, tmTh, tmTl;
-    if (!tmap_bf16(&tmDYt, dY, N, M, 64, 64) || !tmap_bf16(&tmTh, T_hi, r, M, 64, 64) ||
-        !tmap_bf16(&tmTl, T_lo, r, M, 64, 64))
-      return QLORA_ERR_CUDA;
-    GemmArgs g{};
-    g.M_rows = (int)N;
-    g.N_cols = r;
-    g.k_steps = (int)((M + 63) / 64);
-    g.hilo_cols = 1;
-    g.out = dB;
-    g.ldo = r;
-    g.out_f32 = grad_dtype == QLORA_F32;
-    g.out_scale = sc;
-    g.status = status;
-    if ((s = launch_gemm<true, true, false, 128, 1>(tmDYt, tmTh, tmDYt, tmTl, tmDYt, g, dev, sms, st)) != QLORA_OK)
-      return s;
-  }
-  return QLORA_OK;
+qlora_status qlora_linear_bwd_dropout(const qlora_nf4_tensor *W, const qlora_lora *ad, const void *X, const void *dY,
+                                      const void *keep, float p, int64_t M, const void *T_saved, void *dX,
+                                      qlora_dtype dx_dtype, void *dA, void *dB, qlora_dtype grad_dtype, void *ws,
+                                      size_t ws_bytes, qlora_stream_t stream) {
+  qlora_status s = check_nf4(W);
+  if (s != QLORA_OK) return s;
+  if ((s = check_lora(ad)) != QLORA_OK) return s;
+  if (!X || !dY || !keep || !dX || !dA || !dB || !ws || M < 1 || M > (int64_t(1) << 30) || !(p >= 0.0f && p < 1.0f))
+    return QLORA_ERR_INVALID_ARGUMENT;
+  if (!valid_dtype(dx_dtype) || !valid_dtype(grad_dtype)) return QLORA_ERR_INVALID_ARGUMENT;
+  if (W->rows % 8) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(X, 16) || !aligned(dY, 16) || !aligned(keep, 16) || !aligned(dX, 16) || !aligned(dA, 16) ||
+      !aligned(dB, 16) || !aligned(ws, 256) || (T_saved && !aligned(T_saved, 16)))
+    return QLORA_ERR_MISALIGNED;
+  const int64_t N = W->rows, K = W->cols;
+  if (ws_bytes < min_workspace_bytes(M, N, K, ad->r, 1)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  int dev, sms;
+  if ((s = check_device(&dev, &sms)) != QLORA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  void *Xm;
+  float *part;
+  if ((s = dropout_input(X, keep, M, N, K, ad->r, 1, ws, ws_bytes, sms, st, &Xm, &part)) != QLORA_OK) return s;
+  return bwd_impl(W, ad, X, Xm, 1.0f / (1.0f - p), keep, dY, M, T_saved, dX, dx_dtype, dA, dB, grad_dtype, ws, part,
+                  stream);
 }
 
 qlora_status qlora_linear_fwd_multi(const qlora_nf4_tensor *W, const qlora_lora *adapters, int32_t n_adapters,

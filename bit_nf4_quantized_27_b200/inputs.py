@@ -106,3 +106,13 @@ def custom(n: int, k: int, m: int, r: int, seed: int, w_std: float = 0.02,
     b = normal((n, r), b_std, seed + B_ID)
     dy = normal((m, n), 1.0, seed + DY_ID)
     return w, x, a, b, dy
+
+
+def keep_mask(m: int, k: int, p: float, seed: int) -> torch.Tensor:
+    """Drawn dropout keep mask for [m, k] (each element kept with probability
+    1 - p), packed one bit per element: bit (j % 8) of byte j // 8 of row i.
+    Returns uint8 [m, k // 8] (k % 8 == 0)."""
+    g = torch.Generator().manual_seed(seed)
+    keep = torch.rand((m, k), generator=g, dtype=torch.float64) >= p
+    weights = (1 << torch.arange(8, dtype=torch.int32))
+    return (keep.view(m, k // 8, 8).to(torch.int32) * weights).sum(-1).to(torch.uint8)

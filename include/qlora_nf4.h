@@ -187,6 +187,27 @@ QLORA_API qlora_status qlora_linear_fwd_noalloc(const qlora_nf4_tensor *W, const
                                                 const void *X, int64_t M, void *Y, qlora_dtype y_dtype,
                                                 void *T_save, qlora_stream_t stream);
 
+/* Forward and backward with LoRA dropout ("Mastering model fine-tuning"
+ * (ezsol.ir), "Low-Rank Adaptation (LoRA)": its LoRA configuration sets
+ * lora_dropout).  The adapter branch reads D(X) = X * keep / (1 - p):
+ *   Y  = X W'^T + s (D(X) A^T) B^T,  T = D(X) A^T (saved as by qlora_linear_fwd)
+ *   dX = dY W' + s ((dY B) A) * keep / (1 - p),  dA = s (dY B)^T D(X),  dB = s dY^T T
+ *   keep  device uint8 [M, K/8], 16-byte aligned: bit (k % 8) of byte k / 8 of
+ *         row m is 1 to keep X[m, k] (the drawn mask; the caller draws it)
+ *   p     drop probability, 0 <= p < 1
+ * Other arguments as qlora_linear_fwd / qlora_linear_bwd.  ws needs room for a
+ * masked copy of X as well: qlora_workspace_bytes_dropout() (the entry points
+ * accept down to the plain minimum plus that copy). */
+QLORA_API size_t qlora_workspace_bytes_dropout(int64_t M, int64_t N, int64_t K, int32_t r, int for_backward);
+QLORA_API qlora_status qlora_linear_fwd_dropout(const qlora_nf4_tensor *W, const qlora_lora *adapter, const void *X,
+                                                const void *keep, float p, int64_t M, void *Y, qlora_dtype y_dtype,
+                                                void *T_save, void *ws, size_t ws_bytes, qlora_stream_t stream);
+QLORA_API qlora_status qlora_linear_bwd_dropout(const qlora_nf4_tensor *W, const qlora_lora *adapter, const void *X,
+                                                const void *dY, const void *keep, float p, int64_t M,
+                                                const void *T_saved, void *dX, qlora_dtype dx_dtype, void *dA,
+                                                void *dB, qlora_dtype grad_dtype, void *ws, size_t ws_bytes,
+                                                qlora_stream_t stream);
+
 /* Decode forward of one NF4 base serving several adapters at once ("What is
  * LoRA?" (IBM): one shared frozen base, many small LoRA modules swapped per task;
  * "QLoRA" glossary page, "Trade-offs": adapters are small enough to store and

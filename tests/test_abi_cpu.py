@@ -148,3 +148,38 @@ def test_multi_adapter_argument_checks_without_gpu(L):
     assert f(ctypes.byref(good), mixed, 2, idx, X, 3, Y, 1, ws, 1 << 20, None) == 1
     assert f(ctypes.byref(_t(1024, 576)), ads, 2, idx, X, 3, Y, 1, ws, 1 << 20, None) == 2
     assert f(ctypes.byref(good), ads, 2, idx, X, 3, Y, 1, ws, 64, None) == 4
+
+
+def test_dropout_argument_checks_without_gpu(L):
+    good = _t(64, 64)
+    ad = bd.LoraC(64, 16.0, 0x4000, 0x5000)
+    X, keep, Y, ws = (ctypes.c_void_p(a) for a in (0x10000, 0x20000, 0x30000, 0x40000))
+    f = L.qlora_linear_fwd_dropout
+    big = 1 << 24
+    assert f(ctypes.byref(good), ctypes.byref(ad), X, keep, 1.0, 32, Y, 1, None, ws, big, None) == 1
+    assert f(ctypes.byref(good), ctypes.byref(ad), X, keep, -0.1, 32, Y, 1, None, ws, big, None) == 1
+    assert f(ctypes.byref(good), ctypes.byref(ad), X, None, 0.1, 32, Y, 1, None, ws, big, None) == 1
+    assert f(ctypes.byref(good), ctypes.byref(ad), X, ctypes.c_void_p(0x20008), 0.1, 32, Y, 1, None, ws, big,
+             None) == 3
+    assert f(ctypes.byref(good), ctypes.byref(ad), X, keep, 0.1, 32, Y, 1, None, ws, 64, None) == 4
+    b = L.qlora_linear_bwd_dropout
+    dX, dA, dB = (ctypes.c_void_p(a) for a in (0x50000, 0x60000, 0x70000))
+    assert b(ctypes.byref(good), ctypes.byref(ad), X, X, keep, 1.5, 32, None, dX, 1, dA, dB, 1, ws, big, None) == 1
+    assert b(ctypes.byref(good), ctypes.byref(ad), X, X, None, 0.1, 32, None, dX, 1, dA, dB, 1, ws, big, None) == 1
+    # the dropout workspace holds the masked copy of X on top of the plain one
+    for bwd in (0, 1):
+        assert L.qlora_workspace_bytes_dropout(300, 512, 1024, 64, bwd) >= \
+            L.qlora_workspace_bytes(300, 512, 1024, 64, bwd) + 300 * 1024 * 2
+
+
+def test_keep_mask_generator_packs_like_the_oracle():
+    import numpy as np
+    import torch
+
+    from bit_nf4_quantized_27_b200 import inputs as I
+
+    packed = I.keep_mask(5, 48, 0.3, 11)
+    assert packed.dtype == torch.uint8 and tuple(packed.shape) == (5, 6)
+    g = torch.Generator().manual_seed(11)
+    want = (torch.rand((5, 48), generator=g, dtype=torch.float64) >= 0.3).numpy()
+    assert np.array_equal(O.unpack_keep(packed.numpy(), 5, 48), want)

@@ -266,3 +266,41 @@ def test_llama7b_block_layers_full_size(layer):
 
 def test_65b_block_q_full_size():
     _sampled(I.L65B_BLOCK, 0, nrows=24)
+
+
+@pytest.mark.parametrize("n,k,m,r,p", [(328, 576, 4, 64, 0.1), (1024, 1024, 300, 16, 0.25), (512, 512, 200, 64, 0.5),
+                                       (4104, 128, 1030, 8, 0.05), (640, 4096, 2048, 128, 0.1)])
+def test_lora_dropout_matches_oracle(n, k, m, r, p):
+    c = _custom(n, k, m, r, 13 * n + k + m)
+    keep = I.keep_mask(m, k, p, 99 + m)
+    kb = O.unpack_keep(keep.numpy(), m, k)
+    qg, a, b, x, dy = c.gpu()
+    for dt in (torch.float32, torch.bfloat16):
+        y, t = bd.linear_fwd_dropout(qg, a, b, c.alpha, x, keep.cuda(), p, y_dtype=dt)
+        dx, da, db = bd.linear_bwd_dropout(qg, a, b, c.alpha, x, dy, keep.cuda(), p, t, dx_dtype=dt, grad_dtype=dt)
+        torch.cuda.synchronize()
+        yr, tr = O.linear_fwd_dropout(c.wd, c.af, c.bf, c.xf, kb, p, c.alpha, c.r)
+        check("y", y, yr)
+        check("T", t[0].float() + t[1].float(), tr)
+        dxr, dar, dbr = O.linear_bwd_dropout(c.wd, c.af, c.bf, c.xf, c.dyf, kb, p, c.alpha, c.r)
+        check("dX", dx, dxr)
+        if dt == torch.float32:
+            # the adapter's share of dX alone (about 1% of it), the masked term: it
+            # multiplies A by the bf16 rounding of s U, so each element is within
+            # 2^-8 of (|s U| |A|) * keep / (1 - p) of the exact term, plus the float32
+            # accumulation error of the base product dY W' it is separated from
+            base = c.dyf.astype(np.float64) @ c.wd.astype(np.float64)
+            su = O.lora_scale(c.alpha, c.r) * (c.dyf.astype(np.float64) @ c.bf.astype(np.float64))
+            bound = 2.0 ** -8 * (np.abs(su) @ np.abs(c.af.astype(np.float64))) * kb / (1 - p) + \
+                n * 2.0 ** -24 * (np.abs(c.dyf.astype(np.float64)) @ np.abs(c.wd.astype(np.float64)))
+            term = dx.double().cpu().numpy() - base
+            term_ref = dxr - base
+            assert np.all(np.abs(term - term_ref) <= bound + 1e-6 * np.sqrt(np.mean(term_ref ** 2)))
+        check("dA", da, dar)
+        check("dB", db, dbr)
+    # backward recomputing T from the masked input
+    dx2, da2, db2 = bd.linear_bwd_dropout(qg, a, b, c.alpha, x, dy, keep.cuda(), p, None, dx_dtype=torch.float32,
+                                          grad_dtype=torch.float32)
+    torch.cuda.synchronize()
+    check("dB (T recomputed)", db2, dbr)
+    check("dA (T recomputed)", da2, dar)
