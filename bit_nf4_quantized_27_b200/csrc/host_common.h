@@ -89,9 +89,13 @@ inline int code_of(float x) {
   return bi;
 }
 
+// Cell of x: round-to-nearest of x*32 + 32, read from the low mantissa bits of
+// fl32(x*32 + 32 + 1.5*2^23) (one fused multiply-add, exact integer spacing
+// there); 0..64 for x in [-1, 1].
+constexpr float kCellMagic = 12582912.0f + 32.0f;  // 1.5 * 2^23 + 32
 inline int cell_of(float x) {
-  const float v = std::fmaf(x, 32.0f, 32.0f);
-  return static_cast<int>(v);  // truncation toward zero
+  const float v = std::fmaf(x, 32.0f, kCellMagic);
+  return static_cast<int>(v - 12582912.0f);
 }
 
 struct HostCellTable {

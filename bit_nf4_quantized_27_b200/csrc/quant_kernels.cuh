@@ -14,10 +14,12 @@
 // Code search.  The code of x = fl32(w / S) is argmin_j fl32(|x - L_j|), lowest j
 // on ties.  It is a non-decreasing step function of x with 15 switch points t_j
 // (the largest float32 whose code is <= j).  The kernel cuts [-1, 1] into 65 cells
-// of width 1/32 (cell = trunc(fl32(x * 32 + 32))), narrower than the closest pair
-// of switch points, and keeps per cell the switch point nearest to it and the code
-// just below that point: code = base + (x > thr).  The table is built on the host
-// from the same float32 definition.  To avoid a division per weight, the fast path
+// of width 1/32, narrower than the closest pair of switch points: the cell is the
+// nearest integer to x * 32 + 32, taken from the low mantissa bits of
+// fl32(x * 32 + 32 + 1.5 * 2^23) (one FMA, no conversion).  It keeps per cell the
+// switch point nearest to it and the code just below that point (one 8-byte
+// entry): code = base + (x > thr).  The table is built on the host from the same
+// float32 definition and the same cell formula.  To avoid a division per weight, the fast path
 // uses x' = w * fl32(1/S), which is within 2 ulp of fl32(w / S); whenever x' lies
 // within 4 ulp of the cell's switch point, the exact quotient (IEEE division) is
 // used instead, so the result is always the code of fl32(w / S).
@@ -34,10 +36,16 @@ struct CodeCellTable {
   uint32_t base[kCells];  // code of x <= thr
 };
 
+// Cell 0..64 of x in [-1, 1] (the unsigned min keeps any other input in range).
+__device__ __forceinline__ uint32_t code_cell(float x) {
+  const float v = __fmaf_rn(x, 32.0f, 12582912.0f + 32.0f);
+  return min(__float_as_uint(v) - 0x4B400000u, static_cast<uint32_t>(kCells - 1));
+}
+
 // Exact code of a normalised weight x in [-1, 1] (x already equal to fl32(w / S)).
-__device__ __forceinline__ uint32_t code_from_table(float x, const float *s_thr, const uint32_t *s_base) {
-  const int cell = __float2int_rz(__fmaf_rn(x, 32.0f, 32.0f));
-  return s_base[cell] + (x > s_thr[cell] ? 1u : 0u);
+__device__ __forceinline__ uint32_t code_from_table(float x, const float2 *s_tab) {
+  const float2 e = s_tab[code_cell(x)];
+  return __float_as_uint(e.y) + (x > e.x ? 1u : 0u);
 }
 
 template <typename TIn>
@@ -87,16 +95,12 @@ nf4_quantize_kernel(const TIn *__restrict__ W, int64_t nblocks, uint8_t *__restr
   constexpr int BPI = kQuantThreads / LPB;               // blocks per CTA iteration
   constexpr int ITERS = kGroup / BPI;
 
-  __shared__ float s_thr[kCells];
-  __shared__ uint32_t s_base[kCells];
+  __shared__ float2 s_tab[kCells];  // (switch point, base code bits)
   __shared__ float s_absmax[kGroup];
   __shared__ float s_wmax[kQuantThreads / 32];
 
   const int tid = threadIdx.x;
-  if (tid < kCells) {
-    s_thr[tid] = table.thr[tid];
-    s_base[tid] = table.base[tid];
-  }
+  if (tid < kCells) s_tab[tid] = make_float2(table.thr[tid], __uint_as_float(table.base[tid]));
   const int64_t g = blockIdx.x;
   const int64_t blk0 = g * kGroup;
   const int nblk = static_cast<int>(nblocks - blk0 < kGroup ? nblocks - blk0 : kGroup);
@@ -139,14 +143,13 @@ nf4_quantize_kernel(const TIn *__restrict__ W, int64_t nblocks, uint8_t *__restr
 #pragma unroll
       for (int i = 0; i < EPL; ++i) {
         const float xa = __fmul_rn(w[i], rS);
-        const int cell = __float2int_rz(__fmaf_rn(xa, 32.0f, 32.0f));
-        const float t = s_thr[min(max(cell, 0), kCells - 1)];
-        c[i] = s_base[min(max(cell, 0), kCells - 1)] + (xa > t ? 1u : 0u);
-        slow |= (__float_as_uint(xa) - __float_as_uint(t) + 4u) <= 8u;
+        const float2 e = s_tab[code_cell(xa)];
+        c[i] = __float_as_uint(e.y) + (xa > e.x ? 1u : 0u);
+        slow |= (__float_as_uint(xa) - __float_as_uint(e.x) + 4u) <= 8u;
       }
       if (slow) {
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) c[i] = code_from_table(__fdiv_rn(w[i], S), s_thr, s_base);
+        for (int i = 0; i < EPL; ++i) c[i] = code_from_table(__fdiv_rn(w[i], S), s_tab);
       }
 #pragma unroll
       for (int i = 0; i < EPL; ++i) packed |= c[i] << (4 * i);
