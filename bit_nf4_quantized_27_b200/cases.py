@@ -9,6 +9,7 @@ CASE is one of:
   fwd_65b_up / bwd_65b_up       22016x8192 (gate/up of the 65B-shaped block), 4096 tokens
   fwd_65b_down / bwd_65b_down   8192x22016 (down of the 65B-shaped block), 4096 tokens
   gemv_m1 / gemv_m4 / gemv_m16   decode forward, W 11008x4096, r=64
+  gemv_multi16  decode forward of 16 tokens, each with its own r=64 adapter
   quant_11008   quantise an 11008x4096 bf16 weight
   dequant_11008 dequantise it
   merge_8192    merged export of an 8192x8192 NF4 weight with an r = 64 adapter
@@ -56,6 +57,17 @@ def main(argv=None):
             else:
                 bd.linear_bwd(q, a, b, 16.0, x, dy, t, ws=ws_b)
         st = bd.read_status(ws_f) or bd.read_status(ws_b)
+    elif c == "gemv_multi16":
+        w, x, _, _, _ = _layer(11008, 4096, 16)
+        q = bd.quantize(w)
+        ads = []
+        for i in range(16):
+            _, _, a, b, _ = _layer(11008, 4096, 1, seed=100 + i)
+            ads.append((a, b, 16.0))
+        ws = bd.new_workspace(bd.workspace_bytes(16, 11008, 4096, 64, False))
+        for _ in range(args.reps):
+            bd.linear_fwd_multi(q, ads, list(range(16)), x, ws=ws)
+        st = bd.read_status(ws)
     elif c.startswith("gemv"):
         m = int(c.split("_m")[1])
         w, x, a, b, _ = _layer(11008, 4096, m)

@@ -41,6 +41,13 @@ struct MultiLora {
   float s[kGemvMaxM];
 };
 
+constexpr int kBulkMaxRG = 5;
+constexpr int kBulkMaxStages = 6;
+// Shared-memory placement of the staged kernel's buffers (absolute shared addresses).
+struct BulkLayout {
+  uint32_t lut, red[kBulkMaxRG], stage[kBulkMaxStages], bar, end;
+};
+
 struct GemvArgs {
   const uint8_t *codes;
   const uint8_t *scale_codes;
@@ -58,6 +65,8 @@ struct GemvArgs {
   int rg_per_cta;
   int stages;               // bulk kernel: depth of the shared-memory ring
   int multi;                // 1: token t adds s[t] (x_t A_t^T) B_t^T with ml's adapters
+  BulkLayout lay;           // bulk kernel: placement computed on the host for a window at lay_base
+  uint32_t lay_base;
   MultiLora ml;
 };
 
@@ -349,19 +358,21 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_lora_kernel(const Ge
 }
 
 // ---------------------------------------------------------------------------
-// Bulk-staged variant: each 16-row group's codes (16 x CH/2 contiguous bytes)
-// and block scales (16 x CH/64 bytes) arrive in shared memory through
-// cp.async.bulk into a 2-stage ring, so DRAM sees long contiguous reads and
-// up to 68 KB stays in flight per SM without holding registers.  Requirements:
-// N % 16 == 0, K % 256 == 0 and (K <= 4096 or K % 4096 == 0); CH = min(K, 4096).
+// Bulk-staged variant: each 16-row group's codes (16 x CH/2 bytes, one 3-D TMA
+// copy) and block scales (16 x CH/64 bytes, one bulk copy) arrive in shared
+// memory in a ring of up to kBulkMaxStages stages, so DRAM sees long contiguous
+// reads and up to about 130 KB stays in flight per SM without holding
+// registers.  Both copies carry an L2 evict-first policy: a decode step reads
+// each weight once.  Requirements: N % 16 == 0, K % 256 == 0 and (K <= 4096 or
+// K % 4096 == 0); CH = min(K, 4096).
 // ---------------------------------------------------------------------------
-constexpr int kBulkMaxRG = 5;
 
-__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+__device__ __forceinline__ void bulk_g2s_hint(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
+                                              uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
           static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
-      "l"(src), "r"(bytes), "r"(static_cast<uint32_t>(__cvta_generic_to_shared(bar)))
+      "l"(src), "r"(bytes), "r"(static_cast<uint32_t>(__cvta_generic_to_shared(bar))), "l"(policy)
       : "memory");
 }
 
@@ -376,7 +387,6 @@ inline bool gemv_bulk_ok(int64_t N, int64_t K) {
 // row-group partial sums and the barriers are placed before the table where
 // they fit and after it otherwise.
 constexpr uint32_t kBulkLutBytes = 256 * 256;
-constexpr int kBulkMaxStages = 6;
 constexpr uint32_t kBulkSmemLimit = 232448;  // opt-in dynamic shared memory per CTA
 
 // A stage holds one 16-row group's codes for a chunk of CH = min(K, 4096)
@@ -397,10 +407,8 @@ __host__ __device__ inline uint32_t gemv_bulk_red_bytes(int M) {
 }
 
 // Placement of the bulk kernel's buffers around the 64 KB-aligned table, for a
-// dynamic window starting at shared address `base`.
-struct BulkLayout {
-  uint32_t lut, red[kBulkMaxRG], stage[kBulkMaxStages], bar, end;
-};
+// dynamic window starting at shared address `base` (computed on the host and
+// passed to the kernel, which checks that its window starts there).
 __host__ __device__ inline BulkLayout gemv_bulk_layout(uint32_t base, uint32_t stage_bytes, int stages,
                                                        uint32_t red_bytes) {
   BulkLayout L;
@@ -446,11 +454,14 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   const int TR = gemv_bulk_red_tokens(a.M);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, q = lane & 3;
+  if (tid == 0) ptx::prefetch_tmap(&tm_codes);
 
-  // ---- layout around the 64 KB-aligned table
+  // ---- layout around the 64 KB-aligned table, placed by the host for the
+  // window start it expects (recomputing it here costs a noticeable share of a
+  // decode call's few microseconds)
   const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw));
-  const BulkLayout Lay = gemv_bulk_layout(base, gemv_bulk_stage_bytes(a.K), S, gemv_bulk_red_bytes(a.M));
-  if (S < 2 || S > kBulkMaxStages || Lay.end > base + static_cast<uint32_t>(dyn_bytes)) {
+  const BulkLayout &Lay = a.lay;
+  if (base != a.lay_base || S < 2 || S > kBulkMaxStages || Lay.end > base + static_cast<uint32_t>(dyn_bytes)) {
     if (tid == 0) raise_status(a.status, QLORA_ERR_CUDA);  // the host sized the window for another start
     return;
   }
@@ -481,20 +492,23 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   const int nw = static_cast<int>(CH / 256);  // warps with columns in a chunk
   const bool active = warp < nw;
 
-  // producer (thread 0): stage u = (chunk u / my_rg, row group u % my_rg)
+  // producer (thread 0): stage u = (chunk u / my_rg, row group u % my_rg); the
+  // codes and block scales are read once per call, so they enter L2 as evict-first
+  const uint64_t policy = ptx::l2_evict_first_policy();
   auto issue = [&](int u) {
     const int ch = u / my_rg, i = u % my_rg;
     const int slot = u % S;
     uint8_t *st = stage_at(slot);
     const int64_t n0 = (int64_t)(rg0 + i) * 16;
     ptx::mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(16 * CH / 2 + 16 * CH / 64));
-    ptx::tma_load_3d(st, &tm_codes, &full[slot], 0, static_cast<int32_t>(n0), ch * static_cast<int32_t>(CH / 256));
+    ptx::tma_load_3d_hint(st, &tm_codes, &full[slot], 0, static_cast<int32_t>(n0),
+                          ch * static_cast<int32_t>(CH / 256), policy);
     if (CH == a.K) {
-      bulk_g2s(st + 16 * CH / 2, a.scale_codes + n0 * nbk, static_cast<uint32_t>(16 * nbk), &full[slot]);
+      bulk_g2s_hint(st + 16 * CH / 2, a.scale_codes + n0 * nbk, static_cast<uint32_t>(16 * nbk), &full[slot], policy);
     } else {
       for (int rw = 0; rw < 16; ++rw)
-        bulk_g2s(st + 16 * CH / 2 + rw * (CH / 64), a.scale_codes + (n0 + rw) * nbk + ch * (CH / 64),
-                 static_cast<uint32_t>(CH / 64), &full[slot]);
+        bulk_g2s_hint(st + 16 * CH / 2 + rw * (CH / 64), a.scale_codes + (n0 + rw) * nbk + ch * (CH / 64),
+                      static_cast<uint32_t>(CH / 64), &full[slot], policy);
     }
   };
   if (tid == 0) {
@@ -681,14 +695,15 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
       }
       return true;
     };
-    float ca[2], cb[2];
-    if (my_rg > 0) c2_of(0, ca);
-    for (int i = 0; i < my_rg && ok; i += 2) {
-      if (i + 1 < my_rg) c2_of(i + 1, cb);
-      ok = process(i, ca);
-      if (!ok || i + 1 >= my_rg) break;
-      if (i + 2 < my_rg) c2_of(i + 2, ca);
-      ok = process(i + 1, cb);
+    // one copy of the row-group body (the loop is not unrolled), so the
+    // instruction footprint of the steady state stays small
+    float cn[2] = {0.0f, 0.0f};
+    if (my_rg > 0) c2_of(0, cn);
+#pragma unroll 1
+    for (int i = 0; i < my_rg && ok; ++i) {
+      const float cc[2] = {cn[0], cn[1]};
+      if (i + 1 < my_rg) c2_of(i + 1, cn);
+      ok = process(i, cc);
     }
   }
   if (!ok && lane == 0) raise_status(a.status, QLORA_ERR_TIMEOUT);
@@ -976,7 +991,11 @@ inline qlora_status launch_gemv(GemvArgs g, const CUtensorMap *tm_codes, int dev
     const uint32_t base = dyn_smem_base(dev);
     g.stages = gemv_bulk_stages(g.K, g.M, base, per * static_cast<int>(g.K / CH));
     if (g.stages == 0) bulk = false;
-    else smem = gemv_bulk_smem_bytes(g.K, g.stages, g.M, base);
+    else {
+      smem = gemv_bulk_smem_bytes(g.K, g.stages, g.M, base);
+      g.lay = gemv_bulk_layout(base, gemv_bulk_stage_bytes(g.K), g.stages, gemv_bulk_red_bytes(g.M));
+      g.lay_base = base;
+    }
   }
   if (!bulk && g.multi) return QLORA_ERR_UNSUPPORTED_SHAPE;  // per-token adapters: staged kernel only
   if (!bulk) {
