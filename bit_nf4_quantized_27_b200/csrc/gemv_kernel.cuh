@@ -114,7 +114,17 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2_scaled(uint32_t v, float inv
   return *reinterpret_cast<const uint32_t *>(&h);
 }
 
-__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Waits for the preceding kernel (programmatic dependent launch) and returns 0.
+// Reads of what that kernel writes (s T) take their address from the result, so
+// the compiler cannot schedule them before the wait (a read-only .nc load
+// declares the data constant for the whole kernel, which lets it move).  They
+// are .ca loads: the data no longer changes once the wait returns, and caching
+// it in L1 keeps every warp of every CTA from going to the same L2 lines.
+__device__ __forceinline__ uint32_t griddep_wait_token() {
+  uint32_t z;
+  asm volatile("griddepcontrol.wait;\n\tmov.u32 %0, 0;" : "=r"(z) : : "memory");
+  return z;
+}
 __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
@@ -303,7 +313,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_lora_kernel(const Ge
 
   // LoRA up-projection on tensor cores: rows = 16 weight rows (A = B_lora rows),
   // cols = tokens (B = (s T)^T), K = r.  Needs s T from the preceding kernel.
-  griddep_wait();
+  const __nv_bfloat16 *const sT = a.sT + griddep_wait_token();
   for (int i = warp; i < my_rg; i += kGemvWarps) {
     const int64_t n0 = (int64_t)(rg0 + i) * 16;
     float acc[NG][4];
@@ -324,9 +334,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_lora_kernel(const Ge
         const int t = g + 8 * ng;
         uint32_t b0 = 0, b1 = 0;
         if (t < a.M) {
-          const uint32_t *src = reinterpret_cast<const uint32_t *>(a.sT + (int64_t)t * a.r + j0 + 2 * q);
-          if (j0 + 2 * q < a.r) b0 = __ldg(src);
-          if (j0 + 8 + 2 * q < a.r) b1 = __ldg(src + 4);
+          const unsigned *src = reinterpret_cast<const unsigned *>(sT + (int64_t)t * a.r + j0 + 2 * q);
+          if (j0 + 2 * q < a.r) b0 = __ldca(src);
+          if (j0 + 8 + 2 * q < a.r) b1 = __ldca(src + 4);
         }
         mma_16816(acc[ng], af[0], af[1], af[2], af[3], b0, b1);
       }
@@ -727,7 +737,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
     }
   }
   __syncthreads();
-  griddep_wait();
+  const __nv_bfloat16 *const sT = a.sT + griddep_wait_token();
   if (lora_rg >= 0 && a.multi) {
     // one adapter per token: row (lane & 15) of this row group, half of the
     // rank range per half-warp, combined by a shuffle (fixed order)
@@ -736,11 +746,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
     float *rb = red_at(lora_rg);  // warp 0's slot
     for (int t = 0; t < a.M; ++t) {
       const __nv_bfloat16 *bt = a.ml.B[t] + n * a.r + half * hr;
-      const __nv_bfloat16 *st = a.sT + (int64_t)t * a.r + half * hr;
+      const __nv_bfloat16 *st = sT + (int64_t)t * a.r + half * hr;
       float acc = 0.0f;
       for (int j = 0; j < hr; j += 4) {
         const uint2 bv = __ldg(reinterpret_cast<const uint2 *>(bt + j));
-        const uint2 sv = __ldg(reinterpret_cast<const uint2 *>(st + j));
+        const uint2 sv = __ldca(reinterpret_cast<const uint2 *>(st + j));
         acc = fmaf(bf16lo_to_f32(bv.x), bf16lo_to_f32(sv.x), acc);
         acc = fmaf(bf16hi_to_f32(bv.x), bf16hi_to_f32(sv.x), acc);
         acc = fmaf(bf16lo_to_f32(bv.y), bf16lo_to_f32(sv.y), acc);
@@ -763,9 +773,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
 #pragma unroll
       for (int ng = 0; ng < NG; ++ng) {
         const int t = g + 8 * ng;
-        const uint32_t *src = reinterpret_cast<const uint32_t *>(a.sT + (int64_t)t * a.r + j0 + 2 * q);
-        bt[jj][ng][0] = (t < a.M && j0 + 2 * q < a.r) ? __ldg(src) : 0u;
-        bt[jj][ng][1] = (t < a.M && j0 + 8 + 2 * q < a.r) ? __ldg(src + 4) : 0u;
+        const unsigned *src = reinterpret_cast<const unsigned *>(sT + (int64_t)t * a.r + j0 + 2 * q);
+        bt[jj][ng][0] = (t < a.M && j0 + 2 * q < a.r) ? __ldca(src) : 0u;
+        bt[jj][ng][1] = (t < a.M && j0 + 8 + 2 * q < a.r) ? __ldca(src + 4) : 0u;
       }
     }
 #pragma unroll
@@ -788,9 +798,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
         const int t = g + 8 * ng;
         uint32_t b0 = 0, b1 = 0;
         if (t < a.M) {
-          const uint32_t *src = reinterpret_cast<const uint32_t *>(a.sT + (int64_t)t * a.r + j0 + 2 * q);
-          if (j0 + 2 * q < a.r) b0 = __ldg(src);
-          if (j0 + 8 + 2 * q < a.r) b1 = __ldg(src + 4);
+          const unsigned *src = reinterpret_cast<const unsigned *>(sT + (int64_t)t * a.r + j0 + 2 * q);
+          if (j0 + 2 * q < a.r) b0 = __ldca(src);
+          if (j0 + 8 + 2 * q < a.r) b1 = __ldca(src + 4);
         }
         mma_16816(acc[ng], af[0], af[1], af[2], af[3], b0, b1);
       }
