@@ -280,8 +280,10 @@ def run_step(layers, wl, flat, world, timing=None, ready=None):
 
 
 def launches_per_step(nlayers):
-    # per layer: quantise 1; forward 2 (T, fused GEMM); backward 4 (U, dX, dA, dB)
-    return nlayers * 7
+    # per layer of the 65B-shaped block: quantise 1; forward 3 (T with split K and
+    # its finishing sum, fused GEMM); backward 5 (U with split K and its finishing
+    # sum, dX, dA, dB) -- 63 per step, as the ncu launch list of the step shows
+    return nlayers * 9
 
 
 def graph_time_us(calls, reps=5):
@@ -614,7 +616,7 @@ def main():
                 "ms_per_step": ms_e2e,
                 "copies": "per layer from pinned memory on a copy stream, overlapping the step's compute; "
                           "gradients read back after the step"},
-        "gpu_launches": launches_per_step(len(layers)) * args.steps + (0 if world == 1 else 0),
+        "gpu_launches": launches_per_step(len(layers)) * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and not args.no_sub:
