@@ -264,8 +264,9 @@ def test_llama7b_block_layers_full_size(layer):
     _sampled(I.LLAMA7B_BLOCK, layer)
 
 
-def test_65b_block_q_full_size():
-    _sampled(I.L65B_BLOCK, 0, nrows=24)
+@pytest.mark.parametrize("layer", [0, 4, 6], ids=["q", "gate", "down"])
+def test_65b_block_layers_full_size(layer):
+    _sampled(I.L65B_BLOCK, layer, nrows=24)
 
 
 @pytest.mark.parametrize("n,k,m,r,p", [(328, 576, 4, 64, 0.1), (1024, 1024, 300, 16, 0.25), (512, 512, 200, 64, 0.5),
