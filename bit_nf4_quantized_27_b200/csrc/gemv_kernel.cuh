@@ -1,9 +1,12 @@
 // Small-M (decode-shaped) forward of the NF4 linear layer with LoRA, M <= 16:
 //   Y [M, N] = X W'^T + (s T) B^T,   T = X A^T computed by lora_down_small_kernel.
 //
-// HBM-bound: the packed codes (0.5 B/weight) dominate the traffic, so the kernel
-// streams them straight from HBM into registers with 8-byte vector loads and
-// decodes in registers.  Each byte (two codes) indexes a 256-entry table of fp16
+// HBM-bound: the packed codes (0.5 B/weight) dominate the traffic.  Two kernels
+// share the decode below: nf4_gemv_bulk_kernel (the one used whenever
+// N % 16 == 0 and K % 256 == 0, with K <= 4096 or a multiple of 4096) stages
+// each 16-row group's codes and scales in shared memory by TMA; the fallback
+// nf4_gemv_lora_kernel, for other shapes, loads them from HBM into registers with
+// 8-byte vector loads.  Each byte (two codes) indexes a 256-entry table of fp16
 // level pairs (L[lo], L[hi]) kept in shared memory with one copy per lane (each
 // lane reads its own bank, so lookups never conflict); the pair is directly one
 // register of an m16n8k16 tensor-core A fragment (rows = 16 weight rows).  The
@@ -129,6 +132,8 @@ __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Fallback for shapes the staged kernel does not take: codes and scales are
+// loaded straight into registers.
 // smem: table [256][32] u32 | red [rg][16 warps][16 rows][16 tokens] f32
 template <int NG>
 __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_lora_kernel(const GemvArgs a) {
