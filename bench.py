@@ -174,8 +174,15 @@ def run_reference(args, rank):
         if i >= args.warmup:
             vals.append(v)
     value = statistics.median(vals)
+    from bit_nf4_quantized_27_b200 import inputs as I
+
+    wl = I.L65B_BLOCK
+    step_flops = sum(sum(layer_flops(wl.m, ly.n, ly.k, wl.r)) for ly in wl.layers)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+            "steps": args.steps, "warmup": args.warmup,
+            # one full step of the workload at the sample's measured rate
+            "ms_per_step": step_flops / (value * 1e12) * 1e3, "ms_per_step_kind": "extrapolated from the sample",
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc},
