@@ -26,6 +26,8 @@
 // shared memory and are summed in a fixed order (deterministic).
 #pragma once
 
+#include <mutex>
+
 #include "nf4_device.cuh"
 #include "sm100_ptx.cuh"
 
