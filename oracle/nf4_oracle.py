@@ -45,6 +45,27 @@ Readings where the pages are silent or loose (each also listed in the design doc):
 * Adapter optimiser: the pages name Adam's per-parameter momentum and variance
   but give no update rule; the step is decoupled-weight-decay Adam (AdamW,
   Loshchilov and Hutter) with bias correction, the form torch.optim.AdamW uses.
+
+What pins each function to something other than itself (tests/test_oracle_pins.py;
+no function here is left unpinned):
+
+* norm_ppf: statistics.NormalDist and scipy's ndtri; the erf-based CDF inverts it.
+* nf4_levels: structure (sorted, exact 0 and +-1) and the snippet's float32 build.
+* assign_codes / quantize: the page's worked example (printed MSEs, codes equal to
+  torch's argmin), an exact-rational brute force, constructed ties, exact levels,
+  all-zero blocks and groups, the ~16% MSE gain over evenly spaced levels.
+* pack_codes / unpack_codes: the byte layout.
+* e4m3_encode / e4m3_decode: the format's spec points, torch's float8 cast.
+* double_quantize / dequantize: the scale error bound, requantise idempotence,
+  one rounding of level times scale, the storage-overhead closed form.
+* linear_fwd / linear_bwd: brute-force loops, central finite differences, B = 0,
+  W = 0, the merged form.
+* merged_weight / merge_export: B = 0 gives the dequantised weight bit for bit,
+  W = 0 gives one bf16 rounding of the update, the layer's forward.
+* adamw_step: torch.optim.AdamW over several steps, closed forms, a planted error.
+* linear_fwd_multi: reduces to linear_fwd per token, adapters kept apart.
+* unpack_keep / linear_fwd_dropout / linear_bwd_dropout: the mask layout, p = 0
+  and everything dropped, central finite differences.
 """
 
 from __future__ import annotations
