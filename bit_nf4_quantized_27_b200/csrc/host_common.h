@@ -102,6 +102,7 @@ struct HostCellTable {
   float thr[65];
   uint32_t base[65];
   float switch_points[15];
+  uint32_t min_edge_ulps;  // fewest float32 steps between a switch point and a cell edge
   bool ok;
 };
 
@@ -133,6 +134,20 @@ inline const HostCellTable &cell_table() {
       }
       b[k] = key_f32(hi);
     }
+    // The kernel picks the cell from x' = w * fl32(1/S), within 2 ulp of
+    // fl32(w / S), and checks only the chosen cell's switch point for a 4-ulp
+    // band: that is exact only while no switch point lies near a cell edge,
+    // where x' and the exact quotient could fall into different cells.  Keep
+    // every switch point more than kEdgeUlps float32 steps from every edge.
+    constexpr uint32_t kEdgeUlps = 8;
+    t.min_edge_ulps = 0xffffffffu;
+    for (int j = 0; j < 15; ++j)
+      for (int k = 0; k <= 66; ++k) {
+        const uint32_t a = f32_key(t.switch_points[j]), e = f32_key(b[k]);
+        const uint32_t d = a > e ? a - e : e - a;
+        if (d < t.min_edge_ulps) t.min_edge_ulps = d;
+      }
+    if (t.min_edge_ulps <= kEdgeUlps) t.ok = false;
     for (int k = 0; k < 65; ++k) {
       const double lo = b[k], hi = b[k + 1];
       int inside = 0, best = 0;

@@ -117,3 +117,38 @@ def test_requantise_idempotent_on_gpu():
     ws = bd.new_workspace(bd.STATUS_BYTES)
     q2 = bd.quantize(wd, ws=ws)
     assert torch.equal(q.codes, q2.codes)
+
+
+def test_every_float32_in_the_unit_interval():
+    # Every float32 x in [-1, 1] (both zeros included, 2 130 706 434 values) goes
+    # through the kernel with S = 1, so x = w / S exactly: 63 values per block of
+    # 64 next to a 1.0 that fixes the block's absmax.  The expected code is the
+    # number of the oracle's switch points below x (the switch points come from
+    # bisecting the oracle's own code assignment).
+    from tests.test_host_layout import _oracle_switch_points
+
+    thr = torch.tensor(_oracle_switch_points(), dtype=torch.int64).to(torch.int32).view(torch.float32).cuda()
+    ws = bd.new_workspace(bd.STATUS_BYTES)
+    per = 63
+    nblk = 1 << 22                                  # blocks per chunk: 264 M values, 1 GiB of input
+    top = 0x3F800000                                # bits of 1.0
+    checked = 0
+    for sign in (0, 0x80000000):
+        for start in range(0, top + 1, per * nblk):
+            n = min(per * nblk, top + 1 - start)
+            nb = (n + per - 1) // per
+            bits = torch.arange(start, start + nb * per, dtype=torch.int64, device="cuda")
+            bits = torch.minimum(bits, torch.tensor(top, device="cuda")) | sign
+            x = bits.to(torch.int64).view(-1)
+            x = torch.where(x >= 1 << 31, x - (1 << 32), x).to(torch.int32).view(torch.float32).view(nb, per)
+            w = torch.cat([torch.ones(nb, 1, device="cuda"), x], dim=1).contiguous()
+            q = bd.quantize(w, ws=ws)
+            p = q.codes.view(nb, 32)
+            codes = torch.stack([p & 15, p >> 4], dim=2).view(nb, 64)[:, 1:]
+            want = torch.searchsorted(thr, x.contiguous(), side="left", out_int32=True)
+            bad = (codes.to(torch.int32) != want).sum().item()
+            assert bad == 0, (hex(sign), start, bad)
+            checked += n
+            del bits, x, w, q, p, codes, want
+    assert bd.read_status(ws) == 0
+    assert checked == 2 * (top + 1)

@@ -76,6 +76,29 @@ def test_levels_close_to_snippet_float32_build():
     assert np.sum(ours != theirs) <= 12
 
 
+def _levels_from_library_ppf(ppf):
+    """The snippet's construction with a library quantile in float64, each level
+    rounded once to float32 (the table reading the kernels embed)."""
+    off = 0.9677083
+    pos = [ppf(off + k * (0.5 - off) / 8.0) for k in range(8)]
+    neg = [-ppf(off + k * (0.5 - off) / 7.0) for k in range(7)]
+    vals = sorted(neg + [0.0] + pos)
+    return np.array([v / max(vals) for v in vals], dtype=np.float64).astype(F32)
+
+
+def test_levels_equal_two_library_builds_bit_for_bit():
+    # Python's statistics.NormalDist and scipy's ndtri (Cephes) are written
+    # independently of the oracle's AS241; with the exact construction rounded
+    # once, all three give the same 16 float32 bit patterns.  L[1] sits 0.497 ulp
+    # from a rounding boundary, so a slip in the oracle's quantile, in the
+    # offsets' spacing or in the normalisation changes at least one pattern.
+    ours = O.nf4_levels().view(np.uint32)
+    nd = _levels_from_library_ppf(statistics.NormalDist().inv_cdf).view(np.uint32)
+    cephes = _levels_from_library_ppf(lambda p: float(scipy.special.ndtri(p))).view(np.uint32)
+    assert np.array_equal(nd, cephes)
+    assert np.array_equal(ours, nd), [hex(int(v)) for v in ours]
+
+
 # ---------------------------------------------------------------------------
 # The page's worked example
 # ---------------------------------------------------------------------------
@@ -294,6 +317,74 @@ def test_double_quant_scale_error_bound():
     for gi in range(q["c2"].size):
         blk = slice(gi * 256, (gi + 1) * 256)
         assert q["scale_codes"][blk].max() == 0x7E
+
+
+_E4M3_EXACT = [Fraction(float(v)) for v in O.e4m3_decode(np.arange(0x7F))]  # 0x00 .. 0x7E
+
+
+def _e4m3_rne_exact(x: Fraction) -> int:
+    """E4M3 code of a non-negative rational: nearest value, ties to the code with
+    an even last mantissa bit, saturating at 448 (exact arithmetic)."""
+    if x >= _E4M3_EXACT[-1]:
+        return 0x7E
+    hi = next(i for i, v in enumerate(_E4M3_EXACT) if v >= x)
+    if _E4M3_EXACT[hi] == x or hi == 0:
+        return hi
+    lo = hi - 1
+    d_lo, d_hi = x - _E4M3_EXACT[lo], _E4M3_EXACT[hi] - x
+    if d_lo != d_hi:
+        return lo if d_lo < d_hi else hi
+    return lo if lo % 2 == 0 else hi
+
+
+def _near_tie_scales(c2: np.float32, rng) -> np.ndarray:
+    """float32 scales S whose quotient S / c2 lies within a few float32 ulps of
+    E4M3 rounding midpoints, so that rounding the quotient to float32 first
+    (or not) decides the E4M3 code."""
+    out = []
+    mids = [(a + b) / 2 for a, b in zip(_E4M3_EXACT[:-1], _E4M3_EXACT[1:])]
+    for mid in rng.choice(len(mids), 24, replace=False):
+        s0 = np.float32(float(mids[mid] * Fraction(float(c2))))
+        for k in range(-3, 4):
+            s = s0
+            for _ in range(abs(k)):
+                s = np.nextafter(s, np.float32(np.inf if k > 0 else 0))
+            out.append(s)
+    return np.array(out, F32)
+
+
+def test_double_quantize_exact_rational():
+    # c2 = fl32(max S / 448) and q = E4M3_rne(fl32(S / c2)), re-derived in exact
+    # rational arithmetic on three groups, the last one ragged (100 blocks), with
+    # scales placed where the quotient lands on or next to an E4M3 midpoint once
+    # rounded to float32: rounding S / c2 in float64, or keeping c2 in float64,
+    # changes codes here.
+    rng = np.random.default_rng(29)
+    groups = []
+    for size in (256, 256, 100):
+        m = np.float32(rng.uniform(0.01, 0.08))
+        c2 = F32(float(_fl32(Fraction(float(m)) / 448)))
+        s = _near_tie_scales(c2, rng)
+        s = s[(s > 0) & (s < m)][: size - 1]
+        fill = (rng.uniform(0.0, 1.0, size - 1 - s.size) * m).astype(F32)
+        g = np.concatenate([[m], s, fill]).astype(F32)
+        rng.shuffle(g)
+        groups.append(g)
+    scales = np.concatenate(groups)
+    q, c2 = O.double_quantize(scales)
+    assert c2.size == 3 and q.size == 612
+    mids = {a / 2 + b / 2 for a, b in zip(_E4M3_EXACT[:-1], _E4M3_EXACT[1:])}
+    ties_hit = 0
+    for gi, g in enumerate(groups):
+        m = max(Fraction(float(v)) for v in g)
+        c2_exact = _fl32(m / 448)
+        assert Fraction(float(c2[gi])) == c2_exact
+        for bi, sv in enumerate(g):
+            x = _fl32(Fraction(float(sv)) / c2_exact)
+            want = _e4m3_rne_exact(x)
+            ties_hit += x in mids
+            assert q[gi * 256 + bi] == want, (gi, bi, float(sv))
+    assert ties_hit >= 5  # the construction really reaches exact float32 midpoints
 
 
 def test_storage_overhead_closed_form(golden_dir):
