@@ -760,17 +760,20 @@ qlora_status qlora_adamw_step(float *param, void *param_bf16, const float *grad,
 static __device__ __align__(256) uint8_t g_noalloc_scratch[QLORA_NOALLOC_SCRATCH_BYTES];
 
 namespace {
+// Only a successful lookup is cached: a lookup that fails (for example one made
+// during a stream capture) is retried by the next call on that device.
 qlora_status noalloc_scratch(int dev, void **out) {
-  static std::once_flag flags[64];
+  static std::mutex mu;
   static void *addr[64];
-  static cudaError_t err[64];
-  std::call_once(flags[dev], [&] {
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
     void *p = nullptr;
-    err[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return QLORA_ERR_CUDA;
+    }
     addr[dev] = p;
-    cudaGetLastError();
-  });
-  if (err[dev] != cudaSuccess || !addr[dev]) return QLORA_ERR_CUDA;
+  }
   *out = addr[dev];
   return QLORA_OK;
 }

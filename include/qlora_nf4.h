@@ -181,7 +181,11 @@ QLORA_API qlora_status qlora_linear_bwd(const qlora_nf4_tensor *W, const qlora_l
  * device current); make that first call before any stream capture.  Every call
  * on a device shares the one array and the contents left by the last call: calls
  * that overlap on the GPU (different streams, or other threads) race on it, so
- * serialise them.  Device-side status of these calls is not readable. */
+ * serialise them.  Device-side status of these calls is not readable: when a
+ * kernel of such a call records a device-side error (a bounded wait that gave
+ * up), the call has still returned QLORA_OK and Y and T_save are undefined.
+ * A failed address lookup returns QLORA_ERR_CUDA and is retried by the next
+ * call. */
 #define QLORA_NOALLOC_SCRATCH_BYTES (256u + 2u * 1024u * 1024u)
 QLORA_API qlora_status qlora_linear_fwd_noalloc(const qlora_nf4_tensor *W, const qlora_lora *adapter,
                                                 const void *X, int64_t M, void *Y, qlora_dtype y_dtype,

@@ -38,6 +38,22 @@ def test_rejects_sizes_beyond_its_scratch():
              None, None) == 2
 
 
+@pytest.mark.parametrize("m,expect_size_error", [(16384, False), (16385, True)])
+def test_size_limit_boundary(m, expect_size_error):
+    # 256 status bytes + M * 64 * 2 bytes of s*T: 16384 tokens at rank 64 fill the
+    # scratch exactly, one token more does not.  X is NULL, so a call that gets
+    # past the size check stops at a later host check (no device here, or the
+    # NULL X) and launches nothing.
+    f = _fn()
+    t = bd.NF4TensorC(64, 64, 0x1000, 0x2000, 0x3000)
+    ad = bd.LoraC(64, 16.0, 0x4000, 0x5000)
+    rc = f(ctypes.byref(t), ctypes.byref(ad), None, m, ctypes.c_void_p(0x7000), 1, None, None)
+    if expect_size_error:
+        assert rc == 2
+    else:
+        assert rc in (1, 8), rc  # QLORA_ERR_INVALID_ARGUMENT (NULL X) or QLORA_ERR_NO_DEVICE
+
+
 def _close(got: torch.Tensor, want: torch.Tensor):
     g = got.float().cpu().numpy().astype(np.float64)
     w = want.float().cpu().numpy().astype(np.float64)
