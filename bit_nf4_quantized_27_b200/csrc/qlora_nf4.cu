@@ -11,10 +11,12 @@
 #include "gemm_kernel.cuh"
 #include "gemm_pair_kernel.cuh"
 #include "adapter_kernels.cuh"
+#include "decode_kernel.cuh"
 #include "gemv_kernel.cuh"
 #include "host_common.h"
 #include "qlora_nf4.h"
 #include "quant_kernels.cuh"
+#include "selftest_kernel.cuh"
 
 using namespace qlora;
 
@@ -62,19 +64,37 @@ bool make_tmap(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, uint32_t
 }
 
 // NF4 codes [N][K/2 bytes] as a 3-D map (128 bytes, N rows, K/256 chunks of 128
-// bytes), box 128 x 16 rows x `chunks`, 128-byte swizzle: the decode GEMV's
+// bytes), box 128 x `rows` x `chunks`, 128-byte swizzle: the decode kernels'
 // stage layout [chunk][row][128 B].
-bool tmap_codes_gemv(CUtensorMap *m, const void *codes, int64_t N, int64_t K, uint32_t chunks) {
+bool tmap_codes_gemv(CUtensorMap *m, const void *codes, int64_t N, int64_t K, uint32_t chunks, uint32_t rows = 16) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(K / 256)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K / 2), 128};
-  const cuuint32_t box[3] = {128, 16, chunks};
+  const cuuint32_t box[3] = {128, rows, chunks};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(codes), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// LoRA B [N, r] bf16 as a 3-D map (64 ranks, N rows, r/64 chunks of 128 bytes;
+// for r <= 64 one chunk whose ranks past r read as zeros), box 64 x `rows` x
+// chunks with the 128-byte swizzle: the decode kernel's per-unit B-row layout
+// [chunk][row][128 B].
+bool tmap_brows(CUtensorMap *m, const void *B, int64_t N, int r, uint32_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const uint32_t chunks = r <= 64 ? 1u : static_cast<uint32_t>(r / 64);
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(r <= 64 ? r : 64), static_cast<cuuint64_t>(N), chunks};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(r) * 2, 128};
+  const cuuint32_t box[3] = {64, rows, chunks};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult res = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(B), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return res == CUDA_SUCCESS;
 }
 
 bool tmap_bf16(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
@@ -231,8 +251,11 @@ size_t min_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r, int for_b
   const size_t mr = align256(static_cast<size_t>(M) * r * 2);  // one bf16 [M, r] buffer
   size_t bytes = QLORA_STATUS_BYTES;
   if (!for_backward) {
-    bytes += mr;                                    // s*T
-    if (M <= kGemvMaxM) bytes += gemv_workspace_bytes(M, N, K);
+    // s*T: [M, r] bf16, or for the one-kernel decode path its tagged MMA
+    // fragment entries (ceil(r/16) k-steps x two token halves x 32 lanes x 4
+    // values x 8 bytes)
+    const size_t frag = static_cast<size_t>((r + 15) / 16) * 2048;
+    bytes += M <= kGemvMaxM ? std::max(mr, align256(frag)) : mr;
   } else {
     bytes += 4 * mr;                                // s*U (hi, lo), recomputed T (hi, lo)
   }
@@ -263,6 +286,49 @@ qlora_status fwd_impl(const qlora_nf4_tensor *W, const qlora_lora *ad, const voi
   void *sT = wsb + QLORA_STATUS_BYTES;
   const size_t mr = align256(static_cast<size_t>(M) * ad->r * 2);
 
+  if (M <= kGemvMaxM && Xl == X && aligned(W->scale_codes, 16) && ad->r % 8 == 0 && aligned(X, 16) &&
+      aligned(ad->A, 16) && aligned(ad->B, 16)) {
+    // one kernel per call: T, the fused dequant GEMV and the LoRA term
+    const DecodePlan p = decode_plan(N, K, static_cast<int>(M), ad->r, sms, decode_smem_base(dev));
+    CUtensorMap tmc, tmb;
+    if (p.ok &&
+        tmap_codes_gemv(&tmc, W->codes, N, K, static_cast<uint32_t>(p.WPR), static_cast<uint32_t>(16 * p.RPS)) &&
+        tmap_brows(&tmb, ad->B, N, ad->r, static_cast<uint32_t>(16 * p.RPS))) {
+      DecodeArgs g{};
+      g.codes = W->codes;
+      g.scale_codes = W->scale_codes;
+      g.c2 = W->c2;
+      g.X = static_cast<const __nv_bfloat16 *>(X);
+      g.A = static_cast<const __nv_bfloat16 *>(ad->A);
+      g.B = static_cast<const __nv_bfloat16 *>(ad->B);
+      g.N = N;
+      g.K = K;
+      g.M = static_cast<int>(M);
+      g.r = ad->r;
+      g.s = sc;
+      g.Y = Y;
+      g.y_f32 = y_dtype == QLORA_F32;
+      g.stf_g = reinterpret_cast<uint64_t *>(sT);
+      __nv_bfloat16 *th = static_cast<__nv_bfloat16 *>(T_save);
+      g.T_hi = th;
+      g.T_lo = th ? th + M * ad->r : nullptr;
+      g.status = status_ptr(ws);
+      g.bar_count = status_ptr(ws) + 1;
+      g.bar_gen = status_ptr(ws) + 2;
+      g.G = p.G;
+      g.units = p.units;
+      g.units_max = p.units_max;
+      g.WPR = p.WPR;
+      g.RPS = p.RPS;
+      g.stages = p.stages;
+      g.F = p.F;
+      g.stf_bytes = p.stf_bytes;
+      g.brow_unit_bytes = p.brow_unit_bytes;
+      g.lay = p.lay;
+      g.lay_base = p.base;
+      return launch_decode(p, g, tmc, tmb, dev, st);
+    }
+  }
   if (M <= kGemvMaxM) {
     __nv_bfloat16 *th = static_cast<__nv_bfloat16 *>(T_save);
     auto down = M > 8 ? lora_down_small_kernel<2> : lora_down_small_kernel<1>;
@@ -798,9 +864,22 @@ qlora_status qlora_linear_fwd_noalloc(const qlora_nf4_tensor *W, const qlora_lor
   return qlora_linear_fwd(W, adapter, X, M, Y, y_dtype, T_save, scratch, QLORA_NOALLOC_SCRATCH_BYTES, stream);
 }
 
+qlora_status qlora_selftest_bounded_wait(void *ws, uint32_t limit_us, qlora_stream_t stream) {
+  if (!ws || limit_us < 1 || limit_us > 2000000u) return QLORA_ERR_INVALID_ARGUMENT;
+  if (!aligned(ws, 256)) return QLORA_ERR_MISALIGNED;
+  qlora_status s;
+  if ((s = check_device(nullptr, nullptr)) != QLORA_OK) return s;
+  // the copy in flight reads the workspace header itself (QLORA_STATUS_BYTES)
+  static_assert(kSelftestCopyBytes <= QLORA_STATUS_BYTES, "the copy stays inside the header");
+  bounded_wait_selftest_kernel<<<1, kSelftestThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t *>(ws), status_ptr(ws), static_cast<uint64_t>(limit_us) * 1000u);
+  return launch_status();
+}
+
 qlora_status qlora_clear_status(void *ws, qlora_stream_t stream) {
   if (!ws) return QLORA_ERR_INVALID_ARGUMENT;
-  return cudaMemsetAsync(ws, 0, sizeof(uint32_t), reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+  // words 0 (status) and 1 (arrival count); word 2 (generation) is kept
+  return cudaMemsetAsync(ws, 0, 2 * sizeof(uint32_t), reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
              ? QLORA_OK
              : QLORA_ERR_CUDA;
 }

@@ -33,7 +33,13 @@
  *   - The library never allocates, frees or synchronises (except
  *     qlora_read_status, which synchronises the stream it is given).  All scratch
  *     comes from the caller's workspace ws (qlora_workspace_bytes() tells how much).
- *     The first QLORA_STATUS_BYTES of ws hold a device status word.
+ *     The first QLORA_STATUS_BYTES of ws hold a device status word and two
+ *     counters of the one-kernel decode forward (an arrival count and a call
+ *     generation).  A new workspace must start zeroed (at least its first
+ *     QLORA_STATUS_BYTES and, for the forward with M <= 16, the s*T entries
+ *     after them: allocate it zeroed).  Every completed call leaves the arrival
+ *     count at zero; after a call whose kernel did not complete, or one that
+ *     recorded QLORA_ERR_TIMEOUT, call qlora_clear_status before reusing ws.
  *   - Argument checks run on the host before any launch; a failed check returns an
  *     error code and launches nothing.  A failed launch returns QLORA_ERR_CUDA.
  *     Errors found on the device (non-finite weights, a bounded wait that timed
@@ -264,8 +270,21 @@ QLORA_API qlora_status qlora_adamw_step(float *param, void *param_bf16, const fl
                                         float *exp_avg_sq, int64_t n, const qlora_adamw_hparams *hp, int64_t step,
                                         qlora_stream_t stream);
 
-/* Zero the status word at the start of ws (enqueued on stream). */
+/* Zero the status word and the decode forward's arrival count at the start of
+ * ws (enqueued on stream).  The call generation is kept: the decode forward's
+ * s*T entries in ws are tagged with it, and a generation that went backwards
+ * could make a previous call's entries look current. */
 QLORA_API qlora_status qlora_clear_status(void *ws, qlora_stream_t stream);
+
+/* Test hook for the device-side error path (no counterpart on the QLoRA pages).
+ * Launches one CTA that runs the protocol every pipelined kernel of the library
+ * follows when a bounded wait gives up: it waits on a barrier that nothing
+ * completes for limit_us microseconds (1 .. 2,000,000), records
+ * QLORA_ERR_TIMEOUT in the status word of ws, lets its other warps leave, waits
+ * for the copy it has in flight (a read of the first QLORA_STATUS_BYTES of ws)
+ * and frees its tensor memory.  The GPU context stays usable afterwards.
+ * QLORA_ERR_INVALID_ARGUMENT for a NULL ws or a limit out of range. */
+QLORA_API qlora_status qlora_selftest_bounded_wait(void *ws, uint32_t limit_us, qlora_stream_t stream);
 
 /* Synchronise `stream`, read the status word at the start of ws and return the
  * first error it records (QLORA_OK if none).  The word is left unchanged. */

@@ -305,3 +305,87 @@ def test_lora_dropout_matches_oracle(n, k, m, r, p):
     torch.cuda.synchronize()
     check("dB (T recomputed)", db2, dbr)
     check("dA (T recomputed)", da2, dar)
+
+
+@pytest.mark.parametrize("n,k,m,r", [(1000, 256, 1, 8), (1000, 768, 7, 24), (2040, 1280, 16, 64),
+                                     (3080, 3840, 11, 40), (11008, 4096, 2, 16), (256, 4096, 16, 256)])
+def test_one_kernel_decode_shapes(n, k, m, r):
+    # the one-kernel decode path: rows not a multiple of 16, K giving 1, 3, 5, 15
+    # and 16 warps per row group, ranks below a k-step (r % 16 != 0) and two
+    # 64-rank chunks
+    c = _custom(n, k, m, r, 13 * n + k + m + r)
+    qg, a, b, x, _ = c.gpu()
+    ws = bd.new_workspace(bd.workspace_bytes(m, n, k, r, False))
+    for dt in (torch.float32, torch.bfloat16):
+        y, t = bd.linear_fwd(qg, a, b, c.alpha, x, y_dtype=dt, ws=ws)
+        yr, tr = c.ref_fwd()
+        check(f"y {n}x{k} m={m} r={r}", y, yr)
+        check(f"T {n}x{k} m={m} r={r}", t[0].float() + t[1].float(), tr)
+    assert bd.read_status(ws) == 0
+
+
+def test_decode_lora_term_alone():
+    # W = 0 (every code 7): y = s (X A^T) B^T, the LoRA path alone, on the decode
+    # kernel at 1, 9 and 16 tokens
+    for m in (1, 9, 16):
+        c = _custom(2048, 1024, m, 64, 71 + m, b_std=0.5)
+        c.w = torch.zeros_like(c.w)
+        c.wd = np.zeros_like(c.wd)
+        qg, a, b, x, _ = c.gpu()
+        y, _ = bd.linear_fwd(qg, a, b, c.alpha, x, y_dtype=torch.float32)
+        yr, _ = c.ref_fwd()
+        check(f"lora alone m={m}", y, yr)
+
+
+def test_decode_consecutive_calls_share_a_workspace():
+    # Calls on one workspace, alternating two weights (different grids), with new
+    # tokens each time: the grid barrier's generation moves on every call and its
+    # count returns to zero; the results stay bit-identical for repeated inputs.
+    c1 = _custom(4096, 2048, 4, 64, 501)
+    c2 = _custom(1536, 4096, 16, 32, 502)
+    g1, g2 = c1.gpu(), c2.gpu()
+    ws = bd.new_workspace(max(bd.workspace_bytes(16, 4096, 4096, 64, False), 4096))
+    first = {}
+    for it in range(6):
+        for name, c, gp in (("a", c1, g1), ("b", c2, g2)):
+            qg, a, b, x, _ = gp
+            xi = x if it % 2 == 0 else x.flip(0).contiguous()
+            y, _ = bd.linear_fwd(qg, a, b, c.alpha, xi, y_dtype=torch.float32, ws=ws)
+            key = (name, it % 2)
+            if key in first:
+                assert torch.equal(y, first[key]), key
+            else:
+                first[key] = y.clone()
+                xr = c.xf if it % 2 == 0 else c.xf[::-1]
+                yr, _ = O.linear_fwd(c.wd, c.af, c.bf, xr, c.alpha, c.r)
+                check(f"y {name} {it}", y, yr)
+    assert bd.read_status(ws) == 0
+    hdr = ws[:16].view(torch.int32).cpu()
+    assert int(hdr[1]) == 0  # barrier count back to zero
+
+
+def test_decode_graph_replay():
+    # 24 calls captured in one CUDA graph (consecutive kernels overlap through
+    # programmatic dependent launch), replayed twice, against eager results
+    c = _custom(11008, 4096, 1, 64, 777)
+    qg, a, b, x, _ = c.gpu()
+    ws = bd.new_workspace(bd.workspace_bytes(16, 11008, 4096, 64, False))
+    xs = [torch.randn(1, 4096, device="cuda").to(torch.bfloat16) for _ in range(3)]
+    ys = [torch.empty(1, 11008, dtype=torch.float32, device="cuda") for _ in range(24)]
+    want = [bd.linear_fwd(qg, a, b, c.alpha, xs[i % 3], y_dtype=torch.float32, ws=ws)[0].clone() for i in range(3)]
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            for i in range(24):
+                bd.linear_fwd(qg, a, b, c.alpha, xs[i % 3], ws=ws, out=ys[i], save_t=False)
+    for _ in range(2):
+        for y in ys:
+            y.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        for i, y in enumerate(ys):
+            assert torch.equal(y, want[i % 3]), (i, float((y - want[i % 3]).abs().max()))
+    del g
+    assert bd.read_status(ws) == 0

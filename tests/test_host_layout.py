@@ -82,3 +82,20 @@ def test_quantiser_cell_table(tmp_path):
     assert lines["ok"] == "1" and int(lines["min_edge_ulps"]) > 8
     got = [int(ln.split()[2], 16) for ln in r.stdout.splitlines() if ln.startswith("switch")]
     assert got == _oracle_switch_points()
+
+
+@pytest.mark.skipif(shutil.which("nvcc") is None and not os.path.exists("/usr/local/cuda/bin/nvcc"),
+                    reason="nvcc not available")
+def test_decode_plans(tmp_path):
+    # the one-kernel decode path: every plan fits, is aligned, has no overlapping
+    # buffers, and its CTAs cover every row exactly once
+    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    exe = tmp_path / "decode_plan_check"
+    src = os.path.join(ROOT, "tests", "host", "decode_plan_check.cu")
+    b = subprocess.run([nvcc, "-std=c++17", "-O1", "-gencode", "arch=compute_100a,code=sm_100a", "-I",
+                        os.path.join(ROOT, "include"), "-o", str(exe), src], capture_output=True, text=True,
+                       timeout=600)
+    assert b.returncode == 0, b.stderr[-3000:]
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stdout[-3000:]
+    assert " 0 failures" in r.stdout
