@@ -80,6 +80,7 @@ def lib():
                                                   sz, vp]),
         "qlora_lora_merge": (ctypes.c_int, [pT, pL, vp, vp]),
         "qlora_adamw_step": (ctypes.c_int, [vp, vp, vp, vp, vp, i64, ctypes.POINTER(AdamWC), i64, vp]),
+        "qlora_selftest_bounded_wait": (ctypes.c_int, [vp, ctypes.c_uint32, vp]),
         "qlora_clear_status": (ctypes.c_int, [vp, vp]),
         "qlora_read_status": (ctypes.c_int, [vp, vp]),
         "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -229,6 +230,12 @@ def linear_bwd(q: NF4Weight, A, B, alpha: float, X, dY, T=None, dx_dtype=torch.b
                                   _dtype_code(dX.dtype), _ptr(dA), _ptr(dB), _dtype_code(dA.dtype), _ptr(ws),
                                   ws.numel(), _stream(stream)), "qlora_linear_bwd")
     return dX, dA, dB
+
+
+def selftest_bounded_wait(ws: torch.Tensor, limit_us: int, stream=None):
+    """Runs the device-side give-up protocol once: records QLORA_ERR_TIMEOUT in ws."""
+    _check(lib().qlora_selftest_bounded_wait(_ptr(ws), int(limit_us), _stream(stream)),
+           "qlora_selftest_bounded_wait")
 
 
 def clear_status(ws: torch.Tensor, stream=None):

@@ -85,6 +85,17 @@ def test_valid_call_without_gpu_reports_no_device(L):
     assert L.qlora_nf4_quantize(W, 1, ctypes.byref(_t(64, 64)), ws, None) == 8
 
 
+def test_selftest_argument_checks_without_gpu(L):
+    ws = ctypes.c_void_p(0x20000)
+    assert L.qlora_selftest_bounded_wait(None, 1000, None) == 1
+    assert L.qlora_selftest_bounded_wait(ws, 0, None) == 1
+    assert L.qlora_selftest_bounded_wait(ws, 2000001, None) == 1
+    assert L.qlora_selftest_bounded_wait(ctypes.c_void_p(0x20010), 1000, None) == 3
+    import torch
+    if not torch.cuda.is_available():
+        assert L.qlora_selftest_bounded_wait(ws, 1000, None) == 8
+
+
 def test_status_strings(L):
     for code in range(9):
         assert L.qlora_status_string(code)
