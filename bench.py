@@ -128,18 +128,18 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # CPU oracle baseline (bounded sample of the same step)
 # ---------------------------------------------------------------------------
-def oracle_sample(seconds_budget=20.0, rows=2048, toks=1024):
-    """Runs the oracle on row/token slices of the 65B-shaped block's layers:
-    quantise a `rows`-row slice of each weight, then forward+backward of `toks`
-    tokens through it, layer after layer until `seconds_budget` is spent.
-    Returns (TFLOP/s, threads, description, seconds)."""
+def oracle_sample(seconds_budget=20.0, rows=2048, toks=1024, wl=None):
+    """Runs the oracle on row/token slices of a block's layers (the 65B-shaped
+    block unless `wl` names another): quantise a `rows`-row slice of each weight,
+    then forward+backward of `toks` tokens through it, layer after layer until
+    `seconds_budget` is spent.  Returns (TFLOP/s, threads, description, seconds)."""
     import numpy as np
     from threadpoolctl import threadpool_info
 
     import oracle as O
     from bit_nf4_quantized_27_b200 import inputs as I
 
-    wl = I.L65B_BLOCK
+    wl = I.L65B_BLOCK if wl is None else wl
     flops, t_total, done = 0.0, 0.0, []
     for li, ly in enumerate(wl.layers):
         w = I.normal((rows, ly.k), 0.02, I.seed_for(wl.wid, I.W_ID, li)).float().numpy()
@@ -159,7 +159,7 @@ def oracle_sample(seconds_budget=20.0, rows=2048, toks=1024):
         if t_total > seconds_budget:
             break
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    desc = (f"oracle (numpy float64) on layers {','.join(done)} of the 65B-shaped block, each a {rows}-row slice of W "
+    desc = (f"oracle (numpy float64) on layers {','.join(done)} of {wl.name}, each a {rows}-row slice of W "
             f"quantised then forward+backward of {toks} tokens; FLOPs counted as for the GPU step")
     return flops / t_total / 1e12, threads, desc, t_total
 
@@ -244,10 +244,12 @@ def build_block(wl, device, rank, gen_seed_offset=0):
     return layers, flat
 
 
-def run_step(layers, wl, flat, world, timing=None, ready=None):
+def run_step(layers, wl, flat, world, timing=None, ready=None, quant=True):
     """One block step on the current stream.  `ready` = (x_events, dy_events):
     layer i's forward waits for x_events[i] and its backward for dy_events[i]
-    (the end-to-end step copies each layer's inputs on a copy stream)."""
+    (the end-to-end step copies each layer's inputs on a copy stream).  With
+    quant=False the weights quantised by an earlier step are reused (the
+    training step proper: QLoRA quantises the frozen weights once, at load)."""
     import torch
 
     from bit_nf4_quantized_27_b200 import binding as bd
@@ -258,7 +260,8 @@ def run_step(layers, wl, flat, world, timing=None, ready=None):
         if ev:
             e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
             e0.record()
-        bd.quantize(d["w"], out=d["q"], ws=d["ws_f"])
+        if quant:
+            bd.quantize(d["w"], out=d["q"], ws=d["ws_f"])
         if ev:
             e1.record()
         if ready is not None:
@@ -325,9 +328,9 @@ def graph_time_us(calls, reps=5):
 
 def sub_gemv(device, peaks):
     """Decode-shaped forward (W 11008x4096, M in {1,4,16}, r=64): GB/s over the
-    NF4 codes + scales + activations.  64 calls per CUDA graph, rotating over 8
-    weight copies (186 MB, larger than L2), so every call reads its weights from
-    HBM."""
+    NF4 codes + scales + activations.  68 calls per CUDA graph, rotating over 17
+    weight copies (395 MB, more than three times L2), so every call reads its
+    weights from HBM."""
     import torch
 
     from bit_nf4_quantized_27_b200 import binding as bd
@@ -335,7 +338,7 @@ def sub_gemv(device, peaks):
 
     wl = I.GEMV
     n, k, r = 11008, 4096, 64
-    copies = 8
+    copies = 17
     g = torch.Generator(device=device)
     g.manual_seed(I.seed_for(wl.wid, I.W_ID))
     qs = []
@@ -351,7 +354,7 @@ def sub_gemv(device, peaks):
         y = torch.empty(m, n, dtype=torch.bfloat16, device=device)
         t = torch.empty(2, m, r, dtype=torch.bfloat16, device=device)
         ws = bd.new_workspace(bd.workspace_bytes(m, n, k, r, False), device)
-        reps = 8 * copies
+        reps = 4 * copies
 
         def calls():
             for i in range(reps):
@@ -363,7 +366,7 @@ def sub_gemv(device, peaks):
         gbs = (nf4 + act) / (us * 1e-6) / 1e9
         out[f"m{m}"] = {"us_per_call": us, "GB/s": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
                         "GB/s_incl_adapters": (nf4 + act + (r * k + n * r) * 2) / (us * 1e-6) / 1e9,
-                        "launches_per_call": 2, "timing": "CUDA graph of 64 calls, 8 weight copies"}
+                        "launches_per_call": 1, "timing": f"CUDA graph of {reps} calls, {copies} weight copies"}
     # 16 decode tokens, each with its own adapter on the same base
     m = 16
     ads = [((torch.randn(r, k, generator=g, device=device) / 64).to(torch.bfloat16),
@@ -371,7 +374,7 @@ def sub_gemv(device, peaks):
     x = torch.randn(m, k, generator=g, device=device).to(torch.bfloat16)
     y = torch.empty(m, n, dtype=torch.bfloat16, device=device)
     ws = bd.new_workspace(bd.workspace_bytes(m, n, k, r, False), device)
-    reps = 8 * copies
+    reps = 4 * copies
     idx = list(range(m))
 
     def calls_multi():
@@ -384,8 +387,109 @@ def sub_gemv(device, peaks):
     gbs = (nf4 + act) / (us * 1e-6) / 1e9
     out["m16_16_adapters"] = {"us_per_call": us, "GB/s": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
                               "GB/s_incl_adapters": (nf4 + act + m * (r * k + n * r) * 2) / (us * 1e-6) / 1e9,
-                              "launches_per_call": 2, "timing": "CUDA graph of 64 calls, 8 weight copies"}
+                              "launches_per_call": 2, "timing": f"CUDA graph of {reps} calls, {copies} weight copies"}
     return out
+
+
+def sub_block7b(device, peaks, steps=10, warmup=3):
+    """The Llama-7B block (q, k, v, o 4096x4096, gate/up 4096->11008, down
+    11008->4096; 2048 tokens, r = 64 on every layer): forward + backward of all
+    seven layers, with the per-step quantisation and without it (the training
+    step proper, weights quantised once at load); TFLOP/s of algorithmic FLOPs
+    against the bf16 dense peak, and the oracle timed on a bounded sample of
+    the same layers.  Inputs total about 1 GB, larger than L2."""
+    import torch
+
+    from bit_nf4_quantized_27_b200 import inputs as I
+
+    wl = I.LLAMA7B_BLOCK
+    layers, flat = build_block(wl, device, 0)
+    fl_f = sum(layer_flops(wl.m, d["n"], d["k"], wl.r)[0] for d in layers)
+    fl_b = sum(layer_flops(wl.m, d["n"], d["k"], wl.r)[1] for d in layers)
+    for _ in range(warmup):
+        run_step(layers, wl, flat, 1)
+    torch.cuda.synchronize()
+    res = {"flops_per_step": fl_f + fl_b, "layers": [d["name"] for d in layers], "tokens": wl.m, "lora_r": wl.r}
+    for quant in (True, False):
+        timing = {"quant": [], "fwd": [], "bwd": []}
+        s, e = cuda_timer()
+        s.record()
+        for _ in range(steps):
+            run_step(layers, wl, flat, 1, timing, quant=quant)
+        e.record()
+        torch.cuda.synchronize()
+        ms = s.elapsed_time(e) / steps
+        t_fwd = sum(a.elapsed_time(b) for a, b in timing["fwd"]) / steps
+        t_bwd = sum(a.elapsed_time(b) for a, b in timing["bwd"]) / steps
+        tag = "" if quant else "_no_quant"
+        res["ms_per_step" + tag] = ms
+        res["TFLOP/s" + tag] = (fl_f + fl_b) / (ms * 1e-3) / 1e12
+        res["frac_of_bf16" + tag] = res["TFLOP/s" + tag] / peaks["bf16_tflops"]
+        if quant:
+            res["quantize_ms"] = sum(a.elapsed_time(b) for a, b in timing["quant"]) / steps
+        res["forward_ms" + tag] = t_fwd
+        res["backward_ms" + tag] = t_bwd
+        res["forward_TFLOP/s" + tag] = fl_f / (t_fwd * 1e-3) / 1e12
+        res["backward_TFLOP/s" + tag] = fl_b / (t_bwd * 1e-3) / 1e12
+    res["timing"] = f"CUDA events over {steps} steps after {warmup} warm-up steps"
+    del layers, flat
+    torch.cuda.empty_cache()
+    v, threads, desc, secs = oracle_sample(seconds_budget=8.0, rows=1024, toks=512, wl=wl)
+    res["cpu_oracle"] = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc,
+                         "seconds": secs}
+    return res
+
+
+def sub_tiny(device, peaks, reps=64):
+    """The tiny layer (W 256x256 float32, 16 tokens, r = 8, alpha = 16): quantise +
+    forward + backward per call, as CUDA-graph replays (the work is a few MFLOP,
+    so the figure is a latency; launch-bound), next to the oracle on the same
+    inputs."""
+    import time as _time
+
+    import torch
+
+    import oracle as O
+    from bit_nf4_quantized_27_b200 import binding as bd
+    from bit_nf4_quantized_27_b200 import inputs as I
+
+    wl = I.TINY
+    w, x, a, b, dy = I.weight(wl), I.activations(wl), I.lora_a(wl), I.lora_b(wl), I.grad_output(wl)
+    n, k = w.shape
+    m, r = x.shape[0], a.shape[0]
+    wc, xc, ac, bc, dyc = (t.to(device) for t in (w, x, a, b, dy))
+    q = bd.NF4Weight(n, k, device)
+    wsq = bd.new_workspace(bd.STATUS_BYTES, device)
+    wsf = bd.new_workspace(bd.workspace_bytes(m, n, k, r, False), device)
+    wsb = bd.new_workspace(bd.workspace_bytes(m, n, k, r, True), device)
+    y = torch.empty(m, n, dtype=torch.bfloat16, device=device)
+    t = torch.empty(2, m, r, dtype=torch.bfloat16, device=device)
+    dx = torch.empty(m, k, dtype=torch.bfloat16, device=device)
+    da = torch.empty(r, k, dtype=torch.float32, device=device)
+    db = torch.empty(n, r, dtype=torch.float32, device=device)
+
+    def calls():
+        for _ in range(reps):
+            bd.quantize(wc, out=q, ws=wsq)
+            bd.linear_fwd(q, ac, bc, wl.alpha, xc, ws=wsf, out=y, t_out=t)
+            bd.linear_bwd(q, ac, bc, wl.alpha, xc, dyc, t, ws=wsb, outs=(dx, da, db), grad_dtype=torch.float32)
+
+    us = graph_time_us(calls) / reps
+    fl = sum(layer_flops(m, n, k, r))
+    wf, xf, af, bf, dyf = (t_.float().numpy() for t_ in (w, x, a, b, dy))
+    times = []
+    for _ in range(20):
+        t0 = _time.perf_counter()
+        qo = O.quantize(wf, n, k)
+        wd = O.dequantize(qo["codes"], qo["scale_codes"], qo["c2"], n, k)
+        _, to = O.linear_fwd(wd, af, bf, xf, wl.alpha, r)
+        O.linear_bwd(wd, af, bf, xf, dyf, wl.alpha, r, to)
+        times.append(time.perf_counter() - t0)
+    cpu_us = statistics.median(times) * 1e6
+    return {"us_per_call": us, "TFLOP/s": fl / (us * 1e-6) / 1e12, "flops_per_call": fl,
+            "bound": "launch latency (one quantise, one forward and the backward kernels per call)",
+            "timing": f"CUDA graph of {reps} calls (quantise + forward + backward)",
+            "cpu_oracle": {"us_per_call": cpu_us, "kind": "oracle", "sample": "the whole call, median of 20"}}
 
 
 def sub_quant(device, peaks):
@@ -397,7 +501,7 @@ def sub_quant(device, peaks):
 
     res = {}
     for n, k in ((4096, 4096), (11008, 4096)):
-        copies = 4 if n > 4096 else 8
+        copies = 4 if n > 4096 else 10  # 453 MB / 420 MB touched per rotation, over 3x L2
         ws_ = [(torch.randn(n, k, device=device) * 0.02).to(torch.bfloat16) for _ in range(copies)]
         qs = [bd.NF4Weight(n, k, device) for _ in range(copies)]
         outs = [torch.empty(n, k, dtype=torch.bfloat16, device=device) for _ in range(copies)]
@@ -535,17 +639,25 @@ def main():
     for _ in range(args.steps):
         run_step(layers, wl, flat, world, timing)
     e.record()
+    # the training step proper: the weights stay quantised from the steps above
+    s_nq, e_nq = cuda_timer()
+    s_nq.record()
+    for _ in range(args.steps):
+        run_step(layers, wl, flat, world, quant=False)
+    e_nq.record()
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
     ms = s.elapsed_time(e) / args.steps
+    ms_nq = s_nq.elapsed_time(e_nq) / args.steps
     if world > 1:
         import torch.distributed as dist
 
-        t = torch.tensor([ms], device=device)
+        t = torch.tensor([ms, ms_nq], device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms, ms_nq = (float(v) for v in t.tolist())
     value = world * (fl_f + fl_b) / (ms * 1e-3) / 1e12
+    value_nq = world * (fl_f + fl_b) / (ms_nq * 1e-3) / 1e12
     t_fwd = sum(a.elapsed_time(b) for a, b in timing["fwd"]) / args.steps
     t_bwd = sum(a.elapsed_time(b) for a, b in timing["bwd"]) / args.steps
     t_q = sum(a.elapsed_time(b) for a, b in timing["quant"]) / args.steps
@@ -619,6 +731,9 @@ def main():
                      "frac_of_sustained": fwd_tf / peak_sus, "step_frac": value / world / peak_tc},
         "breakdown_ms_per_step": {"quantize": t_q, "forward": t_fwd, "backward": t_bwd,
                                   "forward_TFLOP/s": fwd_tf, "backward_TFLOP/s": bwd_tf},
+        "train_step_no_quant": {"ms_per_step": ms_nq, "TFLOP/s": value_nq,
+                                "frac_of_bf16": value_nq / world / peak_tc,
+                                "note": "weights quantised once at load (QLoRA), forward + backward of the 7 layers"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": ms_e2e,
                 "copies": "per layer from pinned memory on a copy stream, overlapping the step's compute; "
@@ -631,7 +746,9 @@ def main():
         layers.clear()
         torch.cuda.empty_cache()
         line["sub"] = {"gemv_11008x4096_r64": sub_gemv(device, peaks), "quant_sweep": sub_quant(device, peaks),
-                       "adapter_steps": sub_adapters(device, peaks)}
+                       "adapter_steps": sub_adapters(device, peaks),
+                       "block_7b_m2048_r64": sub_block7b(device, peaks),
+                       "tiny_256x256_m16_r8": sub_tiny(device, peaks)}
     if rank == 0 and world == 1 and not args.no_cpu:
         v, threads, desc, secs = oracle_sample()
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
