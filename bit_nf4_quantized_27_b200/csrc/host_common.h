@@ -134,11 +134,12 @@ inline const HostCellTable &cell_table() {
       }
       b[k] = key_f32(hi);
     }
-    // The kernel picks the cell from x' = w * fl32(1/S), within 2 ulp of
-    // fl32(w / S), and checks only the chosen cell's switch point for a 4-ulp
-    // band: that is exact only while no switch point lies near a cell edge,
-    // where x' and the exact quotient could fall into different cells.  Keep
-    // every switch point more than kEdgeUlps float32 steps from every edge.
+    // The kernel picks the cell from x' = fl32(w * r), r an approximate
+    // reciprocal of S, within 6 ulp of fl32(w / S), and checks only the chosen
+    // cell's switch point for an 8-ulp band: that is exact only while no switch
+    // point lies within 6 ulp of a cell edge, where x' and the exact quotient
+    // could fall into different cells.  Keep every switch point more than
+    // kEdgeUlps float32 steps from every edge.
     constexpr uint32_t kEdgeUlps = 8;
     t.min_edge_ulps = 0xffffffffu;
     for (int j = 0; j < 15; ++j)

@@ -593,10 +593,15 @@ qlora_status qlora_nf4_dequantize(const qlora_nf4_tensor *w, void *W_out, qlora_
   const int64_t want = (nchunks + kDequantThreads - 1) / kDequantThreads;
   const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)sms * 16));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (out_dtype == QLORA_BF16)
-    nf4_dequantize_kernel<__nv_bfloat16><<<grid, kDequantThreads, 0, st>>>(
-        w->codes, w->scale_codes, w->c2, nchunks, static_cast<__nv_bfloat16 *>(W_out));
-  else
+  if (out_dtype == QLORA_BF16) {
+    // one warp step per 1024 weights; enough CTAs for about two steps per warp
+    const int64_t nweights = w->rows * w->cols;
+    const int64_t wsteps = (nweights + 1023) / 1024;
+    const int64_t ctas = (wsteps + 2 * kDequantWarps - 1) / (2 * kDequantWarps);
+    const unsigned gb = (unsigned)std::max<int64_t>(1, std::min<int64_t>(ctas, (int64_t)1 << 20));
+    nf4_dequantize_bf16_kernel<<<gb, kDequantThreads, 0, st>>>(w->codes, w->scale_codes, w->c2, nweights,
+                                                               static_cast<__nv_bfloat16 *>(W_out));
+  } else
     nf4_dequantize_kernel<float><<<grid, kDequantThreads, 0, st>>>(w->codes, w->scale_codes, w->c2, nchunks,
                                                                    static_cast<float *>(W_out));
   return launch_status();

@@ -19,10 +19,14 @@
 // fl32(x * 32 + 32 + 1.5 * 2^23) (one FMA, no conversion).  It keeps per cell the
 // switch point nearest to it and the code just below that point (one 8-byte
 // entry): code = base + (x > thr).  The table is built on the host from the same
-// float32 definition and the same cell formula.  To avoid a division per weight, the fast path
-// uses x' = w * fl32(1/S), which is within 2 ulp of fl32(w / S); whenever x' lies
-// within 4 ulp of the cell's switch point, the exact quotient (IEEE division) is
-// used instead, so the result is always the code of fl32(w / S).
+// float32 definition and the same cell formula; each lane reads its own copy of
+// it (entry k of lane l at (32 k + l) * 8 bytes), so the lookups of a warp never
+// collide in a bank.  To avoid a division per weight, the fast path uses
+// x' = fl32(w * r) with r the hardware reciprocal approximation of S (absolute
+// error at most 2^-23 for S in [1, 2), so relative error at most 2^-22): x' is
+// within 6 ulp of fl32(w / S).  Whenever x' lies within 8 ulp of the cell's
+// switch point, the exact quotient (IEEE division) is used instead, so the
+// result is always the code of fl32(w / S).
 #pragma once
 
 #include "nf4_device.cuh"
@@ -42,9 +46,17 @@ __device__ __forceinline__ uint32_t code_cell(float x) {
   return min(__float_as_uint(v) - 0x4B400000u, static_cast<uint32_t>(kCells - 1));
 }
 
-// Exact code of a normalised weight x in [-1, 1] (x already equal to fl32(w / S)).
-__device__ __forceinline__ uint32_t code_from_table(float x, const float2 *s_tab) {
-  const float2 e = s_tab[code_cell(x)];
+// Entry (switch point, base code bits) at shared address `addr`.
+__device__ __forceinline__ float2 lds_f2(uint32_t addr) {
+  float2 v;
+  asm("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+  return v;
+}
+
+// Exact code of a normalised weight x in [-1, 1] (x already equal to fl32(w / S));
+// tab_lane = shared address of this lane's entry 0.
+__device__ __forceinline__ uint32_t code_from_table(float x, uint32_t tab_lane) {
+  const float2 e = lds_f2(tab_lane + code_cell(x) * 256u);
   return __float_as_uint(e.y) + (x > e.x ? 1u : 0u);
 }
 
@@ -95,12 +107,17 @@ nf4_quantize_kernel(const TIn *__restrict__ W, int64_t nblocks, uint8_t *__restr
   constexpr int BPI = kQuantThreads / LPB;               // blocks per CTA iteration
   constexpr int ITERS = kGroup / BPI;
 
-  __shared__ float2 s_tab[kCells];  // (switch point, base code bits)
+  __shared__ __align__(16) float2 s_tab[kCells * 32];  // (switch point, base code bits), one copy per lane
   __shared__ float s_absmax[kGroup];
   __shared__ float s_wmax[kQuantThreads / 32];
 
   const int tid = threadIdx.x;
-  if (tid < kCells) s_tab[tid] = make_float2(table.thr[tid], __uint_as_float(table.base[tid]));
+  for (int e = tid; e < kCells * 32; e += kQuantThreads)
+    s_tab[e] = make_float2(table.thr[e >> 5], __uint_as_float(table.base[e >> 5]));
+  const uint32_t tab_lane = static_cast<uint32_t>(__cvta_generic_to_shared(s_tab)) + (tid & 31) * 8u;
+  // cell k's entry from the bits of fl32(x * 32 + 32 + 1.5 * 2^23): (bits - 0x4B400000) * 256 + tab_lane,
+  // one multiply-add in 32-bit arithmetic (|x'| <= 1 + 2 ulp keeps the cell in 0..64)
+  const uint32_t tab_off = tab_lane - 0x4B400000u * 256u;
   const int64_t g = blockIdx.x;
   const int64_t blk0 = g * kGroup;
   const int nblk = static_cast<int>(nblocks - blk0 < kGroup ? nblocks - blk0 : kGroup);
@@ -137,19 +154,21 @@ nf4_quantize_kernel(const TIn *__restrict__ W, int64_t nblocks, uint8_t *__restr
     if (S == 0.0f || !finite) {
       packed = 0x77777777u & ((1ull << (4 * EPL)) - 1);  // exact-zero level everywhere
     } else {
-      const float rS = __frcp_rn(S);
-      bool slow = !(rS < 3.0e38f);  // subnormal S: reciprocal overflows
+      float rS;
+      asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rS) : "f"(S));
+      bool slow = !(rS < 3.0e38f);  // subnormal S (flushed): every code takes the exact path
+      if (slow) rS = 0.0f;          // (and the fast path's cells stay in range)
       uint32_t c[EPL];
 #pragma unroll
       for (int i = 0; i < EPL; ++i) {
         const float xa = __fmul_rn(w[i], rS);
-        const float2 e = s_tab[code_cell(xa)];
+        const float2 e = lds_f2(__float_as_uint(__fmaf_rn(xa, 32.0f, 12582912.0f + 32.0f)) * 256u + tab_off);
         c[i] = __float_as_uint(e.y) + (xa > e.x ? 1u : 0u);
-        slow |= (__float_as_uint(xa) - __float_as_uint(e.x) + 4u) <= 8u;
+        slow |= (__float_as_uint(xa) - __float_as_uint(e.x) + 8u) <= 16u;
       }
       if (slow) {
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) c[i] = code_from_table(__fdiv_rn(w[i], S), s_tab);
+        for (int i = 0; i < EPL; ++i) c[i] = code_from_table(__fdiv_rn(w[i], S), tab_lane);
       }
 #pragma unroll
       for (int i = 0; i < EPL; ++i) packed |= c[i] << (4 * i);
@@ -219,6 +238,62 @@ nf4_dequantize_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restri
       float4 *dst = reinterpret_cast<float4 *>(out + ch * 32);
 #pragma unroll
       for (int q = 0; q < 8; ++q) dst[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+    }
+  }
+}
+
+// bf16 output, coalesced without staging: a warp step is 4 segments of 256
+// weights (128 bytes of codes, four 64-blocks).  Lane l decodes the 8 weights of
+// code word l of each segment and stores them as one 16-byte write, so each of
+// the warp's loads and stores covers 128 or 512 contiguous bytes.  The next
+// step's codes and scales are loaded before this step's stores.
+constexpr int kDequantWarps = kDequantThreads / 32;
+__global__ void __launch_bounds__(kDequantThreads)
+nf4_dequantize_bf16_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scale_codes,
+                           const float *__restrict__ c2, int64_t nweights, __nv_bfloat16 *__restrict__ out) {
+  __shared__ float s_lv[16];
+  if (threadIdx.x < 16) s_lv[threadIdx.x] = __uint_as_float(kNf4LevelBits[threadIdx.x]);
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t nwords = nweights / 8;       // 32-bit code words (8 weights each)
+  const int64_t nsteps = (nweights + 1023) / 1024;
+  const int64_t wstride = (int64_t)gridDim.x * kDequantWarps;
+  int64_t ws = (int64_t)blockIdx.x * kDequantWarps + warp;
+  uint32_t cw[4], sq[4];
+  float cz[4];
+  auto fetch = [&](int64_t step) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int64_t w = (step * 4 + k) * 32 + lane;  // code word
+      const bool in = step < nsteps && w < nwords;
+      cw[k] = in ? __ldcs(reinterpret_cast<const uint32_t *>(codes) + w) : 0u;
+      sq[k] = in ? __ldg(scale_codes + (w >> 3)) : 0u;
+      cz[k] = in ? __ldg(c2 + (w >> 11)) : 0.0f;
+    }
+  };
+  fetch(ws);
+  for (; ws < nsteps; ws += wstride) {
+    uint32_t wv[4];
+    float S[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      wv[k] = cw[k];
+      S[k] = __fmul_rn(e4m3_to_f32(static_cast<uint8_t>(sq[k])), cz[k]);
+    }
+    const int64_t w0 = ws * 128 + lane;  // this lane's first code word of the step
+    fetch(ws + wstride);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int64_t w = w0 + 32 * k;
+      if (w < nwords) {
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t byte = (wv[k] >> (8 * j)) & 0xffu;
+          o[j] = pack_bf16x2(__fmul_rn(s_lv[byte & 0xf], S[k]), __fmul_rn(s_lv[byte >> 4], S[k]));
+        }
+        __stcs(reinterpret_cast<uint4 *>(out + w * 8), make_uint4(o[0], o[1], o[2], o[3]));
+      }
     }
   }
 }
