@@ -18,6 +18,9 @@ from .nf4_oracle import (  # noqa: F401
     BLOCK,
     GROUP,
     E4M3_MAX,
+    E5M2_MAX,
+    U8_MAX,
+    SCALE_FORMATS,
     norm_ppf,
     nf4_levels,
     uniform4_levels,
@@ -27,6 +30,12 @@ from .nf4_oracle import (  # noqa: F401
     unpack_codes,
     e4m3_decode,
     e4m3_encode,
+    e5m2_decode,
+    e5m2_encode,
+    u8_encode,
+    scale_format_max,
+    scale_decode,
+    scale_encode,
     double_quantize,
     quantize,
     dequantize_scales,

@@ -31,6 +31,11 @@ Readings where the pages are silent or loose (each also listed in the design doc):
 * The 8-bit second-level format is OCP FP8 E4M3 (the only 8-bit format a page
   names): per group of 256 consecutive blocks c2 = fl32(max S / 448) and
   q = E4M3_rne_satfinite(fl32(S / c2)); an all-zero group has c2 = 0, q = 0.
+  Two other readings of "8 bits in blocks of 256" are selectable with the same
+  structure, the group maximum mapping to the format's largest value: OCP FP8
+  E5M2 (c2 = fl32(max S / 57344), q = E5M2_rne_satfinite(fl32(S / c2))) and a
+  linear unsigned byte (c2 = fl32(max S / 255), q = rne(fl32(S / c2)) clamped
+  to 0..255, decoded value q).
 * Codes are computed from the float32 S; double quantisation is applied to the
   scales afterwards.
 * Dequantised weight: w' = bf16_rne(fl32(L[c] * fl32(dec(q) * c2))).
@@ -77,6 +82,9 @@ import numpy as np
 BLOCK = 64          # weights per first-level absmax block [UL, NF4 bullet]
 GROUP = 256         # first-level scales per second-level group [UL, double-quant bullet]
 E4M3_MAX = 448.0    # largest finite OCP FP8 E4M3 value, 1.75 * 2**8
+E5M2_MAX = 57344.0  # largest finite OCP FP8 E5M2 value, 1.75 * 2**15
+U8_MAX = 255.0      # largest linear unsigned byte
+SCALE_FORMATS = ("e4m3", "e5m2", "u8")
 NF4_OFFSET = 0.9677083  # quantile offset exactly as printed in the [UL] snippet
 
 _F32 = np.float32
@@ -251,35 +259,117 @@ def e4m3_encode(x) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
+# OCP FP8 E5M2 (IEEE-like: infinities and NaNs kept, max finite 57344), from the
+# OCP 8-bit floating point specification: 1 sign, 5 exponent (bias 15), 2
+# mantissa bits; exponent field 0 is subnormal m * 2^-16; exponent field 31 is
+# infinity (m = 0) or NaN.
+# ---------------------------------------------------------------------------
+def e5m2_decode(code) -> np.ndarray:
+    """Value (float64) of each E5M2 byte; +-inf for 0x7C / 0xFC, NaN for the rest
+    of exponent field 31."""
+    c = np.asarray(code, dtype=np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 2) & 0x1F
+    m = c & 0x3
+    with np.errstate(over="ignore"):
+        mag = np.where(e == 0, m * 2.0 ** -16, (4 + m) * np.power(2.0, e - 17))
+    mag = np.where(e == 31, np.where(m == 0, np.inf, np.nan), mag)
+    return sign * mag
+
+
+_E5M2_POS = e5m2_decode(np.arange(0x7C))  # codes 0x00..0x7B, strictly increasing
+
+
+def _encode_rne(x, table, top):
+    """Index of the nearest table value to each x in [0, table[top]] (ties to the
+    even index, which for these formats is the even last mantissa bit); values
+    above table[top] saturate to top."""
+    x = np.asarray(x, dtype=np.float64)
+    if np.any(~np.isfinite(x)) or np.any(x < 0):
+        raise ValueError("scale codes take finite non-negative values")
+    xs = np.minimum(x, table[top])
+    hi = np.minimum(np.searchsorted(table, xs, side="left"), top)  # first value >= x
+    lo = np.maximum(hi - 1, 0)
+    d_hi = table[hi] - xs                                           # exact in float64
+    d_lo = xs - table[lo]
+    pick_lo = (d_lo < d_hi) | ((d_lo == d_hi) & ((lo & 1) == 0))
+    code = np.where(pick_lo, lo, hi)
+    code = np.where(table[hi] == xs, hi, code)
+    return code.astype(np.uint8)
+
+
+def e5m2_encode(x) -> np.ndarray:
+    """E5M2 code of each non-negative finite x: round to nearest, ties to even,
+    saturating to 57344 (0x7B)."""
+    return _encode_rne(x, _E5M2_POS, 0x7B)
+
+
+def u8_encode(x) -> np.ndarray:
+    """Linear byte of each non-negative finite x: round to nearest, ties to
+    even, clamped to 255."""
+    return _encode_rne(x, np.arange(256, dtype=np.float64), 255)
+
+
+def scale_format_max(fmt: str) -> float:
+    """The value the largest scale of a group maps to."""
+    return {"e4m3": E4M3_MAX, "e5m2": E5M2_MAX, "u8": U8_MAX}[fmt]
+
+
+def scale_decode(code, fmt: str = "e4m3") -> np.ndarray:
+    """Value (float64, exact) of each 8-bit scale code in format fmt."""
+    if fmt == "e4m3":
+        return e4m3_decode(code)
+    if fmt == "e5m2":
+        return e5m2_decode(code)
+    if fmt == "u8":
+        return np.asarray(code, dtype=np.int64).astype(np.float64)
+    raise ValueError(fmt)
+
+
+def scale_encode(x, fmt: str = "e4m3") -> np.ndarray:
+    if fmt == "e4m3":
+        return e4m3_encode(x)
+    if fmt == "e5m2":
+        return e5m2_encode(x)
+    if fmt == "u8":
+        return u8_encode(x)
+    raise ValueError(fmt)
+
+
+# ---------------------------------------------------------------------------
 # Second-level ("double") quantisation [UL, double-quant bullet; VN, "Double
 # Quantization"]
 # ---------------------------------------------------------------------------
-def double_quantize(absmax: np.ndarray):
+def double_quantize(absmax: np.ndarray, fmt: str = "e4m3"):
     """Per group of 256 consecutive first-level scales (last group may be short):
-    c2 = fl32(max S / 448) and q[b] = E4M3(fl32(S[b] / c2)); an all-zero group
-    has c2 = 0 and q = 0.  Returns (q uint8[nb], c2 float32[ng])."""
+    c2 = fl32(max S / F) and q[b] = enc(fl32(S[b] / c2)), with F and enc the
+    format's largest value and encoder (E4M3: 448; E5M2: 57344; linear byte:
+    255); an all-zero group has c2 = 0 and q = 0.  Returns (q uint8[nb], c2
+    float32[ng])."""
     s = np.asarray(absmax, dtype=_F32).reshape(-1)
     nb = s.size
     ng = (nb + GROUP - 1) // GROUP
     q = np.zeros(nb, dtype=np.uint8)
     c2 = np.zeros(ng, dtype=_F32)
+    fmax = _F32(scale_format_max(fmt))
     for g in range(ng):
         sg = s[g * GROUP:(g + 1) * GROUP]
         m = sg.max()
         if m == 0:
             continue
-        c2[g] = _F32(m) / _F32(E4M3_MAX)                       # fl32(m / 448)
-        q[g * GROUP:g * GROUP + sg.size] = e4m3_encode((sg / c2[g]).astype(_F32))
+        c2[g] = _F32(m) / fmax                                  # fl32(m / F)
+        q[g * GROUP:g * GROUP + sg.size] = scale_encode((sg / c2[g]).astype(_F32), fmt)
     return q, c2
 
 
-def quantize(w: np.ndarray, rows: int, cols: int, levels: np.ndarray | None = None):
+def quantize(w: np.ndarray, rows: int, cols: int, levels: np.ndarray | None = None, scale_format: str = "e4m3"):
     """Whole quantiser: absmax per 64-block, NF4 codes, packing, double quant.
 
     ``w`` holds the rows x cols weights (float32, or bfloat16 values widened
     exactly).  Returns a dict with packed ``codes`` (rows*cols/2 bytes),
-    ``scale_codes`` (E4M3 bytes, one per block), ``c2`` (float32 per group) and
-    the first-level ``absmax`` (float32 per block, for tests).
+    ``scale_codes`` (8-bit codes in ``scale_format``, one per block), ``c2``
+    (float32 per group) and the first-level ``absmax`` (float32 per block, for
+    tests).
     """
     if cols % BLOCK:
         raise ValueError("cols must be a multiple of 64")
@@ -290,18 +380,18 @@ def quantize(w: np.ndarray, rows: int, cols: int, levels: np.ndarray | None = No
         raise ValueError("non-finite weights")
     s = block_absmax(w)
     codes = assign_codes(w, s, levels)
-    q, c2 = double_quantize(s)
-    return {"codes": pack_codes(codes), "scale_codes": q, "c2": c2, "absmax": s}
+    q, c2 = double_quantize(s, scale_format)
+    return {"codes": pack_codes(codes), "scale_codes": q, "c2": c2, "absmax": s, "scale_format": scale_format}
 
 
 # ---------------------------------------------------------------------------
 # Dequantisation [UL, forward rule: NF4 -> bfloat16 right before the matmul]
 # ---------------------------------------------------------------------------
-def dequantize_scales(scale_codes: np.ndarray, c2: np.ndarray) -> np.ndarray:
+def dequantize_scales(scale_codes: np.ndarray, c2: np.ndarray, fmt: str = "e4m3") -> np.ndarray:
     """S'[b] = fl32(dec(q[b]) * c2[b // 256])."""
     q = np.asarray(scale_codes, dtype=np.uint8).reshape(-1)
     g = np.arange(q.size) // GROUP
-    dec = e4m3_decode(q).astype(_F32)                           # exact in float32
+    dec = scale_decode(q, fmt).astype(_F32)                     # exact in float32
     return (dec * np.asarray(c2, dtype=_F32)[g]).astype(_F32)
 
 
@@ -320,13 +410,13 @@ def bf16_round(x: np.ndarray) -> np.ndarray:
 
 
 def dequantize(codes: np.ndarray, scale_codes: np.ndarray, c2: np.ndarray,
-               rows: int, cols: int, levels: np.ndarray | None = None) -> np.ndarray:
+               rows: int, cols: int, levels: np.ndarray | None = None, scale_format: str = "e4m3") -> np.ndarray:
     """W'[i] = bf16_rne(fl32(L[c_i] * S'[i // 64])), returned as float32 values
     (each exactly a bfloat16), shape (rows, cols)."""
     if levels is None:
         levels = nf4_levels()
     c = unpack_codes(codes)
-    sp = dequantize_scales(scale_codes, c2)
+    sp = dequantize_scales(scale_codes, c2, scale_format)
     prod = (levels[c].reshape(-1, BLOCK) * sp[:, None]).astype(_F32)   # fl32(L * S')
     return bf16_round(prod.reshape(-1)).reshape(rows, cols)
 
@@ -446,7 +536,7 @@ def merged_weight(w_dq: np.ndarray, a: np.ndarray, b: np.ndarray, alpha: float, 
 
 
 def merge_export(codes: np.ndarray, scale_codes: np.ndarray, c2: np.ndarray, rows: int, cols: int,
-                 a: np.ndarray, b: np.ndarray, alpha: float, r: int) -> np.ndarray:
+                 a: np.ndarray, b: np.ndarray, alpha: float, r: int, scale_format: str = "e4m3") -> np.ndarray:
     """The merged 16-bit weight, as float32 values of bf16: bf16_rne(W' + s B A).
 
     [UL] "Trade-offs": merging the adapters into the base model first needs the
@@ -454,7 +544,7 @@ def merge_export(codes: np.ndarray, scale_codes: np.ndarray, c2: np.ndarray, row
     the frozen weights for deployment.  W' + s B A is summed exactly (float64)
     and rounded to bf16 once.
     """
-    wd = dequantize(codes, scale_codes, c2, rows, cols)
+    wd = dequantize(codes, scale_codes, c2, rows, cols, scale_format=scale_format)
     return bf16_round(merged_weight(wd, a, b, alpha, r))
 
 

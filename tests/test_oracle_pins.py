@@ -387,6 +387,140 @@ def test_double_quantize_exact_rational():
     assert ties_hit >= 5  # the construction really reaches exact float32 midpoints
 
 
+# ---------------------------------------------------------------------------
+# The other readings of the 8-bit scale format: OCP FP8 E5M2 and a linear byte
+# ---------------------------------------------------------------------------
+def test_e5m2_spec_points():
+    # max normal 1.75*2^15, min normal 2^-14, min subnormal 2^-16, one, ties to even
+    assert O.e5m2_encode([57344.0])[0] == 0x7B
+    assert O.e5m2_encode([2.0 ** -14])[0] == 0x04
+    assert O.e5m2_encode([2.0 ** -16])[0] == 0x01
+    assert O.e5m2_encode([1.0])[0] == 0x3C
+    assert O.e5m2_encode([0.0])[0] == 0x00
+    assert O.e5m2_encode([1.125])[0] == 0x3C      # halfway 1 .. 1.25 -> even (1.0)
+    assert O.e5m2_encode([1.375])[0] == 0x3E      # halfway 1.25 .. 1.5 -> even (1.5)
+    assert O.e5m2_encode([2.0 ** -17])[0] == 0x00  # halfway 0 .. 2^-16 -> even (0)
+    assert O.e5m2_encode([1e6])[0] == 0x7B        # saturates
+    assert O.e5m2_decode(0x7B) == 57344.0 and O.e5m2_decode(0x7C) == np.inf and np.isnan(O.e5m2_decode(0x7D))
+    assert O.e5m2_decode(0x01) == 2.0 ** -16 and O.e5m2_decode(0xBC) == -1.0
+
+
+def test_e5m2_decode_all_codes_vs_torch():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e5m2).float().numpy().astype(np.float64)
+    got = O.e5m2_decode(codes)
+    nan = np.isnan(ref)
+    assert np.array_equal(nan, np.isnan(got))
+    assert np.array_equal(ref[~nan], got[~nan])
+
+
+def test_e5m2_encode_vs_torch():
+    pos = O.e5m2_decode(np.arange(0x7C)).astype(np.float64)
+    mids = ((pos[1:] + pos[:-1]) / 2).astype(F32)
+    around = [mids]
+    for k in range(1, 4):
+        around += [np.nextafter(mids, np.float32(1e9)), np.nextafter(mids, np.float32(-1))]
+        mids = around[-2]
+    probe = np.concatenate(around + [pos.astype(F32)])
+    rng = np.random.default_rng(7)
+    probe = np.concatenate([probe, np.exp(rng.uniform(np.log(1e-6), np.log(57344.0), 400000)).astype(F32)])
+    probe = probe[(probe >= 0) & (probe <= 57344.0)]   # torch's cast does not saturate; in range it is RNE
+    ref = torch.from_numpy(probe).to(torch.float8_e5m2).view(torch.uint8).numpy()
+    assert np.array_equal(O.e5m2_encode(probe), ref)
+
+
+def test_u8_encode_rounding():
+    k = np.arange(256, dtype=np.float64)
+    assert np.array_equal(O.u8_encode(k), k.astype(np.uint8))
+    half = k[:-1] + 0.5                                   # ties go to the even integer
+    assert np.array_equal(O.u8_encode(half), (k[:-1] + (k[:-1] % 2 == 1)).astype(np.uint8))
+    up = np.nextafter(half.astype(F32), np.float32(1e9))
+    dn = np.nextafter(half.astype(F32), np.float32(-1))
+    assert np.array_equal(O.u8_encode(up), (k[:-1] + 1).astype(np.uint8))
+    assert np.array_equal(O.u8_encode(dn), k[:-1].astype(np.uint8))
+    assert O.u8_encode([255.4999, 255.5, 300.0])[2] == 255 and O.u8_encode([255.5])[0] == 255
+
+
+def _rne_exact(x: Fraction, table) -> int:
+    """Index of the nearest table value (exact rationals, increasing) to x >= 0,
+    ties to the even index, saturating at the last entry."""
+    if x >= table[-1]:
+        return len(table) - 1
+    hi = next(i for i, v in enumerate(table) if v >= x)
+    if table[hi] == x or hi == 0:
+        return hi
+    lo = hi - 1
+    d_lo, d_hi = x - table[lo], table[hi] - x
+    if d_lo != d_hi:
+        return lo if d_lo < d_hi else hi
+    return lo if lo % 2 == 0 else hi
+
+
+@pytest.mark.parametrize("fmt", ["e5m2", "u8"])
+def test_double_quantize_exact_rational_other_formats(fmt):
+    # c2 = fl32(max S / F) and q = enc(fl32(S / c2)), re-derived in exact rational
+    # arithmetic, with scales placed where the quotient lands on or next to a
+    # rounding midpoint of the format once rounded to float32.
+    top = {"e5m2": 0x7B, "u8": 255}[fmt]
+    fmax = {"e5m2": 57344, "u8": 255}[fmt]
+    table = [Fraction(float(v)) for v in O.scale_decode(np.arange(top + 1), fmt)]
+    mids = [(a + b) / 2 for a, b in zip(table[:-1], table[1:])]
+    rng = np.random.default_rng(31)
+    groups = []
+    for size in (256, 256, 100):
+        m = np.float32(rng.uniform(0.01, 0.08))
+        c2 = F32(float(_fl32(Fraction(float(m)) / fmax)))
+        near = []
+        for mid in rng.choice(len(mids), 24, replace=False):
+            s0 = np.float32(float(mids[mid] * Fraction(float(c2))))
+            for kk in range(-3, 4):
+                sv = s0
+                for _ in range(abs(kk)):
+                    sv = np.nextafter(sv, np.float32(np.inf if kk > 0 else 0))
+                near.append(sv)
+        near = np.array(near, F32)
+        near = near[(near > 0) & (near < m)][: size - 1]
+        fill = (rng.uniform(0.0, 1.0, size - 1 - near.size) * m).astype(F32)
+        g = np.concatenate([[m], near, fill]).astype(F32)
+        rng.shuffle(g)
+        groups.append(g)
+    scales = np.concatenate(groups)
+    q, c2 = O.double_quantize(scales, fmt)
+    assert c2.size == 3 and q.size == 612
+    midset = set(mids)
+    ties_hit = 0
+    for gi, g in enumerate(groups):
+        m = max(Fraction(float(v)) for v in g)
+        c2_exact = _fl32(m / fmax)
+        assert Fraction(float(c2[gi])) == c2_exact
+        assert q[gi * 256: gi * 256 + g.size].max() == top      # the group maximum maps to the top code
+        for bi, sv in enumerate(g):
+            x = _fl32(Fraction(float(sv)) / c2_exact)
+            ties_hit += x in midset
+            assert q[gi * 256 + bi] == _rne_exact(x, table), (fmt, gi, bi, float(sv))
+    assert ties_hit >= 5
+
+
+@pytest.mark.parametrize("fmt,bound", [("e5m2", 2.0 ** -3), ("u8", None)])
+def test_other_formats_scale_error_bound(fmt, bound):
+    rng = np.random.default_rng(12)
+    w = (rng.standard_normal(64 * 256 * 3 + 64 * 17) * 0.02).astype(F32)
+    q = O.quantize(w, 1, w.size, scale_format=fmt)
+    assert q["scale_format"] == fmt
+    s, sp = q["absmax"], O.dequantize_scales(q["scale_codes"], q["c2"], fmt)
+    g = np.arange(s.size) // 256
+    if bound is not None:   # half an ulp of a 2-bit mantissa, in the normal range
+        normal_range = s / q["c2"][g] >= 2.0 ** -14
+        assert np.all((np.abs(sp - s) / s)[normal_range] <= bound * (1 + 1e-6))
+    else:                   # half a step of c2, plus float32 rounding of the product
+        assert np.all(np.abs(sp.astype(np.float64) - s) <= q["c2"][g].astype(np.float64) * (0.5 + 1e-5))
+    # the dequantised weight uses the format's scales
+    wd = O.dequantize(q["codes"], q["scale_codes"], q["c2"], 1, w.size, scale_format=fmt)
+    lv = O.nf4_levels()
+    c = O.unpack_codes(q["codes"])
+    assert np.array_equal(wd.reshape(-1), O.bf16_round((lv[c].reshape(-1, 64) * sp[:, None]).astype(F32).reshape(-1)))
+
+
 def test_storage_overhead_closed_form(golden_dir):
     figs = {f["what"]: f["value"] for f in json.load(open(os.path.join(golden_dir, "memory_figures.json")))["figures"]}
     rows, cols = 4096, 4096
