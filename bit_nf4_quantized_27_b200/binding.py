@@ -36,7 +36,11 @@ class QLoRAError(RuntimeError):
 
 class NF4TensorC(ctypes.Structure):
     _fields_ = [("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("codes", ctypes.c_void_p),
-                ("scale_codes", ctypes.c_void_p), ("c2", ctypes.c_void_p)]
+                ("scale_codes", ctypes.c_void_p), ("c2", ctypes.c_void_p), ("scale_format", ctypes.c_int32)]
+
+
+# qlora_scale_format
+SCALE_FORMATS = {"e4m3": 0, "e5m2": 1, "u8": 2}
 
 
 class LoraC(ctypes.Structure):
@@ -142,18 +146,21 @@ def workspace_bytes(m: int, n: int, k: int, r: int, backward: bool) -> int:
 class NF4Weight:
     """A quantised [rows, cols] weight: three device buffers owned by torch."""
 
-    def __init__(self, rows: int, cols: int, device="cuda"):
+    def __init__(self, rows: int, cols: int, device="cuda", scale_format: str = "e4m3"):
         total, cb, sb, gb = storage_bytes(rows, cols)
         if total == 0:
             raise ValueError("cols must be a positive multiple of 64")
+        if scale_format not in SCALE_FORMATS:
+            raise ValueError(f"scale_format must be one of {sorted(SCALE_FORMATS)}")
         self.rows, self.cols = rows, cols
+        self.scale_format = scale_format
         self.codes = torch.empty(cb, dtype=torch.uint8, device=device)
         self.scale_codes = torch.empty(sb, dtype=torch.uint8, device=device)
         self.c2 = torch.empty(gb // 4, dtype=torch.float32, device=device)
 
     def c_struct(self) -> NF4TensorC:
         return NF4TensorC(self.rows, self.cols, self.codes.data_ptr(), self.scale_codes.data_ptr(),
-                          self.c2.data_ptr())
+                          self.c2.data_ptr(), SCALE_FORMATS[self.scale_format])
 
     def nbytes(self) -> int:
         return self.codes.numel() + self.scale_codes.numel() + 4 * self.c2.numel()
@@ -166,9 +173,13 @@ def new_workspace(nbytes: int, device="cuda") -> torch.Tensor:
 
 
 def quantize(w: torch.Tensor, out: NF4Weight | None = None, ws: torch.Tensor | None = None,
-             stream=None) -> NF4Weight:
+             stream=None, scale_format: str | None = None) -> NF4Weight:
+    """NF4 codes with double-quantised block scales; scale_format (default the
+    weight's own, E4M3 for a new one) picks the 8-bit scale format."""
     assert w.is_cuda and w.is_contiguous() and w.dim() == 2
-    q = out if out is not None else NF4Weight(w.shape[0], w.shape[1], w.device)
+    q = out if out is not None else NF4Weight(w.shape[0], w.shape[1], w.device, scale_format or "e4m3")
+    if scale_format is not None:
+        q.scale_format = scale_format
     if ws is None:
         ws = new_workspace(STATUS_BYTES, w.device)
     t = q.c_struct()

@@ -58,7 +58,7 @@ __device__ __forceinline__ void ldmatrix_x2_trans(uint32_t &b0, uint32_t &b1, ui
 __global__ void __launch_bounds__(kMergeThreads) nf4_lora_merge_kernel(
     const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scale_codes, const float *__restrict__ c2,
     int64_t N, int64_t K, const __nv_bfloat16 *__restrict__ A, const __nv_bfloat16 *__restrict__ B, int r, float s,
-    __nv_bfloat16 *__restrict__ out) {
+    __nv_bfloat16 *__restrict__ out, int fmt) {
   extern __shared__ __align__(16) uint8_t merge_smem[];
   const int r16 = merge_r16(r), ldb = r16 + 8;
   constexpr int LDA = kMergeTile + 8, LDO = kMergeTile + 8;
@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(kMergeThreads) nf4_lora_merge_kernel(
   {
     const int row = tid >> 1, b = tid & 1;
     float S = 0.0f;
-    if (n0 + row < N && 64 * b < kcols) S = block_scale(scale_codes, c2, (n0 + row) * nbk + k0 / 64 + b);
+    if (n0 + row < N && 64 * b < kcols) S = block_scale(scale_codes, c2, (n0 + row) * nbk + k0 / 64 + b, fmt);
     sS[row * 2 + b] = S;
   }
   __syncthreads();

@@ -92,6 +92,7 @@ struct DecodeArgs {
   const uint8_t *codes;
   const uint8_t *scale_codes;
   const float *c2;
+  int scale_format;           // qlora_scale_format of scale_codes
   const __nv_bfloat16 *X;
   const __nv_bfloat16 *A;
   const __nv_bfloat16 *B;
@@ -334,11 +335,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       const int w = w0 + k * kDecThreads + tid;
       if (w < nwords) {
         const int row = (4 * w) / static_cast<int>(nbk), col = 4 * w - row * static_cast<int>(nbk);
-        const __half2_raw lo =
-            __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(qv[k] & 0xffffu), __NV_E4M3);
-        const __half2_raw hi =
-            __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(qv[k] >> 16), __NV_E4M3);
-        const float2 f01 = __half22float2(__half2(lo)), f23 = __half22float2(__half2(hi));
+        const float2 f01 = scale_code_value2(qv[k], a.scale_format);
+        const float2 f23 = scale_code_value2(qv[k] >> 16, a.scale_format);
         *reinterpret_cast<float4 *>(sf + row * sfs + col) =
             make_float4(__fmul_rn(f01.x, cv[k]), __fmul_rn(f01.y, cv[k]), __fmul_rn(f23.x, cv[k]),
                         __fmul_rn(f23.y, cv[k]));

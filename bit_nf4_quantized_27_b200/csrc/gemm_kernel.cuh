@@ -56,6 +56,7 @@ struct GemmArgs {
   // NF4 operand (B from dequant)
   const uint8_t *scale_codes;
   const float *c2;
+  int scale_format;  // qlora_scale_format of scale_codes
   int64_t w_rows;    // N of W
   int64_t w_cols;    // K of W
   const __nv_bfloat16 *lora_b2;  // B2 source read by the dequant warps (fwd: B [N, r]; bwd: A [r, K])
@@ -607,7 +608,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         if (++sc == C::SC) { sc = 0; pc ^= 1; }
         const uint4 c0 = half_first ? x1 : x0, c1 = half_first ? x0 : x1;
         if (qs != 0x100u) {
-          const float S = __fmul_rn(e4m3_to_f32(static_cast<uint8_t>(qs)), cs);
+          const float S = __fmul_rn(scale_code_value(qs, args.scale_format), cs);
           nf4_decode64(c0, c1, S, o);
         } else {
 #pragma unroll

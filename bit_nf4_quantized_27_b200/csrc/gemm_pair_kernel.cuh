@@ -394,8 +394,8 @@ gemm_nf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         if (b < nb && ok) {
           const uint32_t ss = static_cast<uint32_t>((cu + b) % C::SS), ps = static_cast<uint32_t>(((cu + b) / C::SS) & 1);
           if (!ptx::mbar_wait(&empty_s[ss], ps ^ 1, abort_flag)) { ok = false; break; }
-          sS[ss * C::HB + t] = __fmul_rn(e4m3_to_f32(static_cast<uint8_t>(q[b][0])), c[b][0]);
-          sS[ss * C::HB + t + 64] = __fmul_rn(e4m3_to_f32(static_cast<uint8_t>(q[b][1])), c[b][1]);
+          sS[ss * C::HB + t] = __fmul_rn(scale_code_value(q[b][0], args.scale_format), c[b][0]);
+          sS[ss * C::HB + t + 64] = __fmul_rn(scale_code_value(q[b][1], args.scale_format), c[b][1]);
           ptx::mbar_arrive(&full_s[ss]);
         }
       }

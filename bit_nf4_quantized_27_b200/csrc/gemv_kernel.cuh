@@ -57,6 +57,7 @@ struct GemvArgs {
   const uint8_t *codes;
   const uint8_t *scale_codes;
   const float *c2;
+  int scale_format;         // qlora_scale_format of scale_codes
   int64_t N, K;
   int M;
   const __nv_bfloat16 *X;   // [M, K]
@@ -256,9 +257,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1) nf4_gemv_lora_kernel(const Ge
       float S[2][4];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(cur.q[h] & 0xffffu), __NV_E4M3);
-        const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(cur.q[h] >> 16), __NV_E4M3);
-        const float2 f01 = __half22float2(__half2(lo)), f23 = __half22float2(__half2(hi));
+        const float2 f01 = scale_code_value2(cur.q[h], a.scale_format);
+        const float2 f23 = scale_code_value2(cur.q[h] >> 16, a.scale_format);
         S[h][0] = __fmul_rn(f01.x, cur.c2[h][0]);
         S[h][1] = __fmul_rn(f01.y, cur.split[h] > 1 ? cur.c2[h][0] : cur.c2[h][1]);
         S[h][2] = __fmul_rn(f23.x, cur.split[h] > 2 ? cur.c2[h][0] : cur.c2[h][1]);
@@ -652,9 +652,8 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
       float S4[2][4];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(qw[h] & 0xffffu), __NV_E4M3);
-        const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(qw[h] >> 16), __NV_E4M3);
-        const float2 f01 = __half22float2(__half2(lo)), f23 = __half22float2(__half2(hi));
+        const float2 f01 = scale_code_value2(qw[h], a.scale_format);
+        const float2 f23 = scale_code_value2(qw[h] >> 16, a.scale_format);
         S4[h][0] = __fmul_rn(f01.x, c2v[h]);
         S4[h][1] = __fmul_rn(f01.y, c2v[h]);
         S4[h][2] = __fmul_rn(f23.x, c2v[h]);

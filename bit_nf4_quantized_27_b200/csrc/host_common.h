@@ -55,6 +55,7 @@ inline qlora_status check_nf4(const qlora_nf4_tensor *t) {
   if (t->rows <= 0 || t->cols <= 0 || t->cols % QLORA_BLOCK) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (t->rows > (int64_t(1) << 31) || t->cols > (int64_t(1) << 31)) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (!aligned(t->codes, 16) || !aligned(t->c2, 4)) return QLORA_ERR_MISALIGNED;
+  if (t->scale_format < QLORA_SCALE_E4M3 || t->scale_format > QLORA_SCALE_U8) return QLORA_ERR_INVALID_ARGUMENT;
   return QLORA_OK;
 }
 

@@ -40,6 +40,13 @@ __device__ __forceinline__ void raise_status(uint32_t *status, qlora_status code
   if (status) atomicOr(status, 1u << static_cast<uint32_t>(code));
 }
 
+// Scale-code formats of the second level (qlora_scale_format): 0 OCP FP8 E4M3,
+// 1 OCP FP8 E5M2, 2 linear unsigned byte.  The group maximum maps to the
+// format's largest value.
+__host__ __device__ constexpr float scale_format_max(int fmt) {
+  return fmt == 1 ? 57344.0f : fmt == 2 ? 255.0f : 448.0f;
+}
+
 // E4M3 byte -> float32 (exact: every E4M3 value is a half value).
 __device__ __forceinline__ float e4m3_to_f32(uint8_t q) {
   __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(q), __NV_E4M3);
@@ -49,6 +56,28 @@ __device__ __forceinline__ float e4m3_to_f32(uint8_t q) {
 // float32 -> E4M3 byte, round to nearest even, saturating to +-448.
 __device__ __forceinline__ uint8_t f32_to_e4m3(float x) {
   return static_cast<uint8_t>(__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3));
+}
+
+// Exact float32 value of a scale code in format fmt (E4M3 and E5M2 values are
+// half values; a byte is an integer).
+__device__ __forceinline__ float scale_code_value(uint32_t q, int fmt) {
+  if (fmt == 2) return static_cast<float>(q & 0xffu);
+  const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(q & 0xffu),
+                                               fmt == 1 ? __NV_E5M2 : __NV_E4M3);
+  return __half2float(__half(h));
+}
+// The values of the two scale codes in the low 16 bits of q (low byte first).
+__device__ __forceinline__ float2 scale_code_value2(uint32_t q, int fmt) {
+  if (fmt == 2) return make_float2(static_cast<float>(q & 0xffu), static_cast<float>((q >> 8) & 0xffu));
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(q & 0xffffu),
+                                                   fmt == 1 ? __NV_E5M2 : __NV_E4M3);
+  return __half22float2(__half2(h));
+}
+// Scale code of a non-negative float32 in format fmt: round to nearest even,
+// saturating at the format's largest value.
+__device__ __forceinline__ uint8_t scale_code_encode(float x, int fmt) {
+  if (fmt == 2) return static_cast<uint8_t>(min(__float2uint_rn(x), 255u));
+  return static_cast<uint8_t>(__nv_cvt_float_to_fp8(x, __NV_SATFINITE, fmt == 1 ? __NV_E5M2 : __NV_E4M3));
 }
 
 // Two float32 -> packed bf16x2 (lo in bits 0..15), round to nearest even.
@@ -62,8 +91,8 @@ __device__ __forceinline__ float bf16lo_to_f32(uint32_t v) { return __uint_as_fl
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 
 // Dequantised block scale S' = fl32(E4M3(q) * c2).
-__device__ __forceinline__ float block_scale(const uint8_t *scale_codes, const float *c2, int64_t b) {
-  return __fmul_rn(e4m3_to_f32(__ldg(scale_codes + b)), __ldg(c2 + (b >> 8)));
+__device__ __forceinline__ float block_scale(const uint8_t *scale_codes, const float *c2, int64_t b, int fmt) {
+  return __fmul_rn(scale_code_value(__ldg(scale_codes + b), fmt), __ldg(c2 + (b >> 8)));
 }
 
 }  // namespace qlora

@@ -298,6 +298,7 @@ qlora_status fwd_impl(const qlora_nf4_tensor *W, const qlora_lora *ad, const voi
       g.codes = W->codes;
       g.scale_codes = W->scale_codes;
       g.c2 = W->c2;
+      g.scale_format = W->scale_format;
       g.X = static_cast<const __nv_bfloat16 *>(X);
       g.A = static_cast<const __nv_bfloat16 *>(ad->A);
       g.B = static_cast<const __nv_bfloat16 *>(ad->B);
@@ -338,7 +339,7 @@ qlora_status fwd_impl(const qlora_nf4_tensor *W, const qlora_lora *ad, const voi
                                                         th ? th + M * ad->r : nullptr, t_scale);
     if ((s = launch_status()) != QLORA_OK) return s;
     GemvArgs g{};
-    g.codes = W->codes; g.scale_codes = W->scale_codes; g.c2 = W->c2;
+    g.codes = W->codes; g.scale_codes = W->scale_codes; g.c2 = W->c2; g.scale_format = W->scale_format;
     g.N = N; g.K = K; g.M = (int)M;
     g.X = static_cast<const __nv_bfloat16 *>(X);
     g.sT = static_cast<const __nv_bfloat16 *>(sT);
@@ -377,6 +378,7 @@ qlora_status fwd_impl(const qlora_nf4_tensor *W, const qlora_lora *ad, const voi
   g.out_scale = 1.0f;
   g.scale_codes = W->scale_codes;
   g.c2 = W->c2;
+  g.scale_format = W->scale_format;
   g.w_rows = N;
   g.w_cols = K;
   g.lora_b2 = static_cast<const __nv_bfloat16 *>(ad->B);
@@ -451,6 +453,7 @@ qlora_status bwd_impl(const qlora_nf4_tensor *W, const qlora_lora *ad, const voi
     g.out_scale = 1.0f;
     g.scale_codes = W->scale_codes;
     g.c2 = W->c2;
+    g.scale_format = W->scale_format;
     g.w_rows = N;
     g.w_cols = K;
     g.lora_b2 = static_cast<const __nv_bfloat16 *>(ad->A);
@@ -574,10 +577,12 @@ qlora_status qlora_nf4_quantize(const void *W, qlora_dtype w_dtype, const qlora_
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (w_dtype == QLORA_BF16)
     nf4_quantize_kernel<__nv_bfloat16><<<(unsigned)ng, kQuantThreads, 0, st>>>(
-        static_cast<const __nv_bfloat16 *>(W), nb, out->codes, out->scale_codes, out->c2, status_ptr(ws), t);
+        static_cast<const __nv_bfloat16 *>(W), nb, out->codes, out->scale_codes, out->c2, status_ptr(ws), t,
+        out->scale_format);
   else
     nf4_quantize_kernel<float><<<(unsigned)ng, kQuantThreads, 0, st>>>(
-        static_cast<const float *>(W), nb, out->codes, out->scale_codes, out->c2, status_ptr(ws), t);
+        static_cast<const float *>(W), nb, out->codes, out->scale_codes, out->c2, status_ptr(ws), t,
+        out->scale_format);
   return launch_status();
 }
 
@@ -600,10 +605,10 @@ qlora_status qlora_nf4_dequantize(const qlora_nf4_tensor *w, void *W_out, qlora_
     const int64_t ctas = (wsteps + 2 * kDequantWarps - 1) / (2 * kDequantWarps);
     const unsigned gb = (unsigned)std::max<int64_t>(1, std::min<int64_t>(ctas, (int64_t)1 << 20));
     nf4_dequantize_bf16_kernel<<<gb, kDequantThreads, 0, st>>>(w->codes, w->scale_codes, w->c2, nweights,
-                                                               static_cast<__nv_bfloat16 *>(W_out));
+                                                               static_cast<__nv_bfloat16 *>(W_out), w->scale_format);
   } else
     nf4_dequantize_kernel<float><<<grid, kDequantThreads, 0, st>>>(w->codes, w->scale_codes, w->c2, nchunks,
-                                                                   static_cast<float *>(W_out));
+                                                                   static_cast<float *>(W_out), w->scale_format);
   return launch_status();
 }
 
@@ -754,7 +759,7 @@ qlora_status qlora_linear_fwd_multi(const qlora_nf4_tensor *W, const qlora_lora 
   lora_down_multi_kernel<<<dim3((r + 15) / 16, static_cast<unsigned>(M)), kLoraDownMultiThreads, 0, st>>>(
       static_cast<const __nv_bfloat16 *>(X), g.ml, K, r, sT);
   if ((s = launch_status()) != QLORA_OK) return s;
-  g.codes = W->codes; g.scale_codes = W->scale_codes; g.c2 = W->c2;
+  g.codes = W->codes; g.scale_codes = W->scale_codes; g.c2 = W->c2; g.scale_format = W->scale_format;
   g.N = N; g.K = K; g.M = (int)M;
   g.X = static_cast<const __nv_bfloat16 *>(X);
   g.sT = sT;
@@ -789,7 +794,8 @@ qlora_status qlora_lora_merge(const qlora_nf4_tensor *W, const qlora_lora *adapt
   const float sc = adapter->alpha / static_cast<float>(adapter->r);
   nf4_lora_merge_kernel<<<grid, kMergeThreads, bytes, reinterpret_cast<cudaStream_t>(stream)>>>(
       W->codes, W->scale_codes, W->c2, W->rows, W->cols, static_cast<const __nv_bfloat16 *>(adapter->A),
-      static_cast<const __nv_bfloat16 *>(adapter->B), adapter->r, sc, static_cast<__nv_bfloat16 *>(W_out));
+      static_cast<const __nv_bfloat16 *>(adapter->B), adapter->r, sc, static_cast<__nv_bfloat16 *>(W_out),
+      W->scale_format);
   return launch_status();
 }
 

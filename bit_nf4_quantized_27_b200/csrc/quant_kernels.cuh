@@ -101,7 +101,7 @@ template <typename TIn>
 __global__ void __launch_bounds__(kQuantThreads)
 nf4_quantize_kernel(const TIn *__restrict__ W, int64_t nblocks, uint8_t *__restrict__ codes,
                     uint8_t *__restrict__ scale_codes, float *__restrict__ c2_out,
-                    uint32_t *__restrict__ status, const CodeCellTable table) {
+                    uint32_t *__restrict__ status, const CodeCellTable table, int fmt) {
   constexpr int EPL = QuantTraits<TIn>::kElemsPerLane;
   constexpr int LPB = kBlock / EPL;                      // lanes per block
   constexpr int BPI = kQuantThreads / LPB;               // blocks per CTA iteration
@@ -182,7 +182,7 @@ nf4_quantize_kernel(const TIn *__restrict__ W, int64_t nblocks, uint8_t *__restr
   }
   __syncthreads();
 
-  // Second level: c2 = fl32(max S / 448), q = E4M3(fl32(S / c2)).
+  // Second level: c2 = fl32(max S / F), q = enc(fl32(S / c2)) in format fmt.
   float m = tid < nblk ? s_absmax[tid] : 0.0f;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -191,8 +191,8 @@ nf4_quantize_kernel(const TIn *__restrict__ W, int64_t nblocks, uint8_t *__restr
   m = s_wmax[0];
 #pragma unroll
   for (int i = 1; i < kQuantThreads / 32; ++i) m = fmaxf(m, s_wmax[i]);
-  const float c2 = m == 0.0f ? 0.0f : __fdiv_rn(m, 448.0f);
-  if (tid < nblk) scale_codes[blk0 + tid] = c2 == 0.0f ? 0 : f32_to_e4m3(__fdiv_rn(s_absmax[tid], c2));
+  const float c2 = m == 0.0f ? 0.0f : __fdiv_rn(m, scale_format_max(fmt));
+  if (tid < nblk) scale_codes[blk0 + tid] = c2 == 0.0f ? 0 : scale_code_encode(__fdiv_rn(s_absmax[tid], c2), fmt);
   if (tid == 0) c2_out[g] = c2;
 }
 
@@ -205,14 +205,14 @@ constexpr int kDequantThreads = 256;
 template <typename TOut>
 __global__ void __launch_bounds__(kDequantThreads)
 nf4_dequantize_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scale_codes,
-                      const float *__restrict__ c2, int64_t nchunks, TOut *__restrict__ out) {
+                      const float *__restrict__ c2, int64_t nchunks, TOut *__restrict__ out, int fmt) {
   __shared__ float s_lv[16];
   if (threadIdx.x < 16) s_lv[threadIdx.x] = __uint_as_float(kNf4LevelBits[threadIdx.x]);
   __syncthreads();
   for (int64_t ch = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; ch < nchunks;
        ch += (int64_t)gridDim.x * blockDim.x) {
     const uint4 cv = __ldg(reinterpret_cast<const uint4 *>(codes) + ch);
-    const float S = block_scale(scale_codes, c2, ch >> 1);
+    const float S = block_scale(scale_codes, c2, ch >> 1, fmt);
     const uint32_t words[4] = {cv.x, cv.y, cv.z, cv.w};
     if constexpr (sizeof(TOut) == 2) {
       uint32_t o[16];
@@ -250,7 +250,8 @@ nf4_dequantize_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restri
 constexpr int kDequantWarps = kDequantThreads / 32;
 __global__ void __launch_bounds__(kDequantThreads)
 nf4_dequantize_bf16_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scale_codes,
-                           const float *__restrict__ c2, int64_t nweights, __nv_bfloat16 *__restrict__ out) {
+                           const float *__restrict__ c2, int64_t nweights, __nv_bfloat16 *__restrict__ out,
+                           int fmt) {
   __shared__ float s_lv[16];
   if (threadIdx.x < 16) s_lv[threadIdx.x] = __uint_as_float(kNf4LevelBits[threadIdx.x]);
   __syncthreads();
@@ -278,7 +279,7 @@ nf4_dequantize_bf16_kernel(const uint8_t *__restrict__ codes, const uint8_t *__r
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       wv[k] = cw[k];
-      S[k] = __fmul_rn(e4m3_to_f32(static_cast<uint8_t>(sq[k])), cz[k]);
+      S[k] = __fmul_rn(scale_code_value(sq[k], fmt), cz[k]);
     }
     const int64_t w0 = ws * 128 + lane;  // this lane's first code word of the step
     fetch(ws + wstride);

@@ -59,7 +59,7 @@
 extern "C" {
 #endif
 
-#define QLORA_NF4_ABI_VERSION 1
+#define QLORA_NF4_ABI_VERSION 2
 #define QLORA_BLOCK 64          /* weights per first-level absmax block */
 #define QLORA_GROUP 256         /* first-level scales per second-level group */
 #define QLORA_STATUS_BYTES 256  /* bytes at the start of ws reserved for the status word */
@@ -87,14 +87,27 @@ typedef enum {
 
 typedef enum { QLORA_F32 = 0, QLORA_BF16 = 1 } qlora_dtype;
 
+/* Format of the 8-bit second-level scale codes.  The double-quantisation bullet
+ * of the glossary page ("How QLoRA works") says only "8 bits in blocks of 256";
+ * "Grokking QLoRA" (vnread), "Double Quantization", names FP8.  E4M3 is the
+ * default; the other two are alternative readings with the same structure:
+ * per group of 256 scales c2 = fl32(max S / F) and q = enc(fl32(S / c2)), the
+ * decoded scale S' = fl32(dec(q) * c2), with
+ *   QLORA_SCALE_E4M3  OCP FP8 E4M3, F = 448, round to nearest even, saturating
+ *   QLORA_SCALE_E5M2  OCP FP8 E5M2, F = 57344, round to nearest even, saturating
+ *   QLORA_SCALE_U8    unsigned byte q = rne(x) clamped to 255, dec(q) = q, F = 255 */
+typedef enum { QLORA_SCALE_E4M3 = 0, QLORA_SCALE_E5M2 = 1, QLORA_SCALE_U8 = 2 } qlora_scale_format;
+
 /* Quantised weight W [rows, cols]; three caller-owned device buffers, sized by
  * qlora_nf4_storage_bytes(). */
 typedef struct {
   int64_t rows;          /* N */
   int64_t cols;          /* K, a multiple of 64 */
   uint8_t *codes;        /* rows*cols/2 bytes, packed nibbles */
-  uint8_t *scale_codes;  /* nb bytes, E4M3 */
+  uint8_t *scale_codes;  /* nb bytes, in scale_format */
   float *c2;             /* ng float32 second-level constants */
+  int32_t scale_format;  /* qlora_scale_format (0, E4M3, when the struct is zero-initialised); set
+                            before qlora_nf4_quantize and kept with the buffers it wrote */
 } qlora_nf4_tensor;
 
 /* LoRA adapter: A [r, K] and B [N, r], both bf16 row-major device buffers.

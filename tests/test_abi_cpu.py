@@ -25,7 +25,7 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_abi_version(L):
-    assert L.qlora_abi_version() == 1
+    assert L.qlora_abi_version() == 2
 
 
 def test_codebook_equals_oracle_bit_for_bit(L):
@@ -66,6 +66,11 @@ def test_argument_checks_without_gpu(L):
     assert L.qlora_nf4_quantize(W, 7, ctypes.byref(good), ws, None) == 1
     assert L.qlora_nf4_quantize(ctypes.c_void_p(0x10008), 1, ctypes.byref(good), ws, None) == 3
     assert L.qlora_nf4_quantize(W, 1, ctypes.byref(_t(64, 64, codes=0x1004)), ws, None) == 3
+    bad_fmt = _t(64, 64)
+    bad_fmt.scale_format = 3
+    assert L.qlora_nf4_quantize(W, 1, ctypes.byref(bad_fmt), ws, None) == 1
+    bad_fmt.scale_format = -1
+    assert L.qlora_nf4_dequantize(ctypes.byref(bad_fmt), ws, 1, None) == 1
     ad = bd.LoraC(64, 16.0, 0x4000, 0x5000)
     X, Y = ctypes.c_void_p(0x6000), ctypes.c_void_p(0x7000)
     assert L.qlora_linear_fwd(ctypes.byref(good), ctypes.byref(bd.LoraC(12, 16.0, 0x4000, 0x5000)), X, 4, Y, 1,
