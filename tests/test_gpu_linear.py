@@ -237,6 +237,71 @@ def test_deterministic(m):
         assert torch.equal(u, v)
 
 
+def _lora_parts(c: Case, rows=None):
+    """The LoRA terms of y and dX alone: from the GPU as the call with B minus the
+    call with B = 0 (float32 outputs; the base product is the same in both), and
+    from the oracle, on all rows or on `rows`.  Returns, per term, (got, want,
+    bound): the fused kernels take the LoRA product as extra K steps with the
+    bf16 rounding of s T (or s U) as one operand, so each element is within
+    2^-8 (|s T| |B^T|) of the exact term, plus one float32 rounding of the
+    running sum per step."""
+    qg, a, b, x, dy = c.gpu()
+    y, t = bd.linear_fwd(qg, a, b, c.alpha, x, y_dtype=torch.float32)
+    y0, _ = bd.linear_fwd(qg, a, torch.zeros_like(b), c.alpha, x, y_dtype=torch.float32)
+    dx, _, _ = bd.linear_bwd(qg, a, b, c.alpha, x, dy, t, dx_dtype=torch.float32, grad_dtype=torch.float32)
+    dx0, _, _ = bd.linear_bwd(qg, a, torch.zeros_like(b), c.alpha, x, dy, t, dx_dtype=torch.float32,
+                              grad_dtype=torch.float32)
+    torch.cuda.synchronize()
+    s = O.lora_scale(c.alpha, c.r)
+    x64, dy64, a64, b64 = (np.asarray(v, np.float64) for v in (c.xf, c.dyf, c.af, c.bf))
+    wd = c.wd.astype(np.float64)
+    sel = slice(None) if rows is None else rows
+    idx = slice(None) if rows is None else torch.from_numpy(rows)
+    st = s * (x64[sel] @ a64.T)
+    su = s * (dy64[sel] @ b64)
+    y0v, dx0v = y0[idx].double().cpu().numpy(), dx0[idx].double().cpu().numpy()
+    y_term = y[idx].double().cpu().numpy() - y0v
+    dx_term = dx[idx].double().cpu().numpy() - dx0v
+    # the LoRA K steps come after the base steps in the same float32 accumulator:
+    # each 16-deep step rounds once, relative to the running sum
+    steps = c.r // 16 + 1
+    y_bound = 2.0 ** -8 * (np.abs(st) @ np.abs(b64.T)) + steps * 2.0 ** -24 * (np.abs(y0v) + np.abs(y_term))
+    dx_bound = 2.0 ** -8 * (np.abs(su) @ np.abs(a64)) + steps * 2.0 ** -24 * (np.abs(dx0v) + np.abs(dx_term))
+    return (y_term, st @ b64.T, y_bound), (dx_term, su @ a64, dx_bound)
+
+
+def _check_term(name, got, want, bound):
+    rms = float(np.sqrt(np.mean(want ** 2)))
+    assert np.all(np.isfinite(got)), name
+    worst = float(np.max(np.abs(got - want) - bound))
+    assert worst <= 1e-6 * rms, f"{name}: exceeds its bound by {worst:.3e} (term rms {rms:.3e})"
+    # and the bound itself is a small fraction of the term (2^-8 of |s U| |A|,
+    # a few percent of |s U A| for r = 64 terms of mixed signs)
+    assert float(np.sqrt(np.mean(bound ** 2))) <= 0.05 * rms, name
+
+
+@pytest.mark.parametrize("m", [17, 128, 256])
+def test_lora_term_alone_single_cta(m):
+    # 17..256 tokens run the single-CTA fused kernel; its LoRA K steps are held to
+    # their own error bound (the term is about 1.5% of y's RMS)
+    c = _custom(1024, 1024, m, 64, 4000 + m)
+    yt, dxt = _lora_parts(c)
+    _check_term(f"y lora m={m}", *yt)
+    _check_term(f"dX lora m={m}", *dxt)
+
+
+def test_lora_term_alone_65b_layer():
+    # the CTA-pair kernel at a full block shape: 8192x8192, 4096 tokens, r = 64
+    wl = I.L65B_BLOCK
+    c = Case(I.weight(wl, 0), I.activations(wl, 0), I.lora_a(wl, 0), I.lora_b(wl, 0), I.grad_output(wl, 0),
+             wl.alpha)
+    rng = np.random.default_rng(65)
+    rows = np.sort(rng.choice(c.m, 32, replace=False))
+    yt, dxt = _lora_parts(c, rows)
+    _check_term("y lora rows", *yt)
+    _check_term("dX lora rows", *dxt)
+
+
 def _sampled(wl, layer, nrows=48):
     c = Case(I.weight(wl, layer), I.activations(wl, layer), I.lora_a(wl, layer), I.lora_b(wl, layer),
              I.grad_output(wl, layer), wl.alpha)
