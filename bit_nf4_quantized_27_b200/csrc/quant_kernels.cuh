@@ -64,10 +64,12 @@ template <typename TIn>
 struct QuantTraits;
 template <>
 struct QuantTraits<__nv_bfloat16> {
-  static constexpr int kElemsPerLane = 8;  // one 16-byte vector
+  static constexpr int kVecs = 2;           // two 16-byte vectors per lane and block
+  static constexpr int kElemsPerLane = 16;
 };
 template <>
 struct QuantTraits<float> {
+  static constexpr int kVecs = 1;
   static constexpr int kElemsPerLane = 4;
 };
 
@@ -103,6 +105,8 @@ nf4_quantize_kernel(const TIn *__restrict__ W, int64_t nblocks, uint8_t *__restr
                     uint8_t *__restrict__ scale_codes, float *__restrict__ c2_out,
                     uint32_t *__restrict__ status, const CodeCellTable table, int fmt) {
   constexpr int EPL = QuantTraits<TIn>::kElemsPerLane;
+  constexpr int VPL = QuantTraits<TIn>::kVecs;
+  constexpr int EPV = EPL / VPL;                         // elements per 16-byte vector
   constexpr int LPB = kBlock / EPL;                      // lanes per block
   constexpr int BPI = kQuantThreads / LPB;               // blocks per CTA iteration
   constexpr int ITERS = kGroup / BPI;
@@ -122,16 +126,19 @@ nf4_quantize_kernel(const TIn *__restrict__ W, int64_t nblocks, uint8_t *__restr
   const int64_t blk0 = g * kGroup;
   const int nblk = static_cast<int>(nblocks - blk0 < kGroup ? nblocks - blk0 : kGroup);
 
-  // Issue every load of this thread first (ITERS x 16 bytes in flight).
-  uint4 v[ITERS];
+  // Issue every load of this thread first (ITERS x VPL x 16 bytes in flight).
+  uint4 v[ITERS][VPL];
 #pragma unroll
   for (int it = 0; it < ITERS; ++it) {
     const int lb = it * BPI + tid / LPB;  // block within group
-    if (lb < nblk) {
-      const int64_t e0 = (blk0 + lb) * kBlock + (tid % LPB) * EPL;
-      v[it] = __ldg(reinterpret_cast<const uint4 *>(W + e0));
-    } else {
-      v[it] = make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int h = 0; h < VPL; ++h) {
+      if (lb < nblk) {
+        const int64_t e0 = (blk0 + lb) * kBlock + (tid % LPB) * EPL + h * EPV;
+        v[it][h] = __ldg(reinterpret_cast<const uint4 *>(W + e0));
+      } else {
+        v[it][h] = make_uint4(0, 0, 0, 0);
+      }
     }
   }
   __syncthreads();
@@ -139,7 +146,9 @@ nf4_quantize_kernel(const TIn *__restrict__ W, int64_t nblocks, uint8_t *__restr
 #pragma unroll
   for (int it = 0; it < ITERS; ++it) {
     const int lb = it * BPI + tid / LPB;
-    uint32_t mb = absbits_max(v[it], static_cast<TIn *>(nullptr));
+    uint32_t mb = absbits_max(v[it][0], static_cast<TIn *>(nullptr));
+#pragma unroll
+    for (int h = 1; h < VPL; ++h) mb = max(mb, absbits_max(v[it][h], static_cast<TIn *>(nullptr)));
 #pragma unroll
     for (int o = LPB / 2; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
     if (lb >= nblk) continue;
@@ -149,10 +158,16 @@ nf4_quantize_kernel(const TIn *__restrict__ W, int64_t nblocks, uint8_t *__restr
     if ((tid % LPB) == 0) s_absmax[lb] = finite ? S : 0.0f;
 
     float w[EPL];
-    unpack_vec(v[it], w);
-    uint32_t packed = 0;
+#pragma unroll
+    for (int h = 0; h < VPL; ++h) {
+      float wv[EPV];
+      unpack_vec(v[it][h], wv);
+#pragma unroll
+      for (int i = 0; i < EPV; ++i) w[h * EPV + i] = wv[i];
+    }
+    uint64_t packed = 0;
     if (S == 0.0f || !finite) {
-      packed = 0x77777777u & ((1ull << (4 * EPL)) - 1);  // exact-zero level everywhere
+      packed = 0x7777777777777777ull & (EPL >= 16 ? ~0ull : ((1ull << (4 * EPL)) - 1));  // exact-zero level
     } else {
       float rS;
       asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rS) : "f"(S));
@@ -171,11 +186,14 @@ nf4_quantize_kernel(const TIn *__restrict__ W, int64_t nblocks, uint8_t *__restr
         for (int i = 0; i < EPL; ++i) c[i] = code_from_table(__fdiv_rn(w[i], S), tab_lane);
       }
 #pragma unroll
-      for (int i = 0; i < EPL; ++i) packed |= c[i] << (4 * i);
+      for (int i = 0; i < EPL; ++i) packed |= static_cast<uint64_t>(c[i]) << (4 * i);
     }
     const int64_t e0 = (blk0 + lb) * kBlock + (tid % LPB) * EPL;
-    if constexpr (EPL == 8) {
-      *reinterpret_cast<uint32_t *>(codes + e0 / 2) = packed;
+    if constexpr (EPL == 16) {
+      *reinterpret_cast<uint2 *>(codes + e0 / 2) =
+          make_uint2(static_cast<uint32_t>(packed), static_cast<uint32_t>(packed >> 32));
+    } else if constexpr (EPL == 8) {
+      *reinterpret_cast<uint32_t *>(codes + e0 / 2) = static_cast<uint32_t>(packed);
     } else {
       *reinterpret_cast<uint16_t *>(codes + e0 / 2) = static_cast<uint16_t>(packed);
     }
