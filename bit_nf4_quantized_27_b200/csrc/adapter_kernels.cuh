@@ -14,18 +14,23 @@
 namespace qlora {
 
 // ---------------------------------------------------------------------------
-// Merged export.  One CTA (8 warps) makes a 128 x 128 tile of W_merged: the
-// low-rank product s B A on mma.sync tensor cores (bf16 in, fp32 accumulate)
-// from shared-memory copies of B's 128 rows and of A's columns k0..k0+127 (both
+// Merged export.  One CTA (8 warps) makes kMergePasses consecutive 128 x 128
+// tiles of one 128-row block of W_merged: the low-rank product s B A on
+// mma.sync tensor cores (bf16 in, fp32 accumulate) from shared-memory copies of
+// B's 128 rows (staged once per CTA) and of A's columns of the tile (both
 // row-major, rows padded by 16 bytes so ldmatrix reads are conflict-free; A's
 // fragments come transposed by ldmatrix.trans); W' decoded from the tile's
 // codes and block scales staged in shared memory; the sum in fp32, rounded to
-// bf16 once, staged over the operand space and stored with 16-byte writes.
+// bf16 once, staged in shared memory and stored with 16-byte writes.  For ranks
+// up to 64 the next tile's A columns, codes and scales are loaded into
+// registers while the current tile is computed and stored.
 // HBM traffic per weight: 0.5 B of code + 1/64 B of scale + 2 B written.
 // ---------------------------------------------------------------------------
 constexpr int kMergeThreads = 256;
 constexpr int kMergeTile = 128;
 constexpr int kMergeMaxK16 = 16;  // r <= 256
+constexpr int kMergePasses = 4;   // column tiles per CTA
+constexpr int kMergePreR16 = 64;  // ranks whose next A tile fits the prefetch registers
 
 __host__ __device__ inline int merge_r16(int r) { return ((r + 15) / 16) * 16; }
 __host__ __device__ inline size_t merge_operand_bytes(int r) {
@@ -33,9 +38,8 @@ __host__ __device__ inline size_t merge_operand_bytes(int r) {
          + static_cast<size_t>(merge_r16(r)) * (kMergeTile + 8) * 2;     // A tile [r16][136]
 }
 inline size_t merge_smem_bytes(int r) {
-  const size_t ops = merge_operand_bytes(r);
   const size_t outb = static_cast<size_t>(kMergeTile) * (kMergeTile + 8) * 2;  // bf16 [128][136]
-  return (ops > outb ? ops : outb) + kMergeTile * 64 + kMergeTile * 2 * 4 + 16 * 4;
+  return merge_operand_bytes(r) + outb + kMergeTile * 64 + kMergeTile * 2 * 4 + 16 * 4;
 }
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -55,7 +59,7 @@ __device__ __forceinline__ void ldmatrix_x2_trans(uint32_t &b0, uint32_t &b1, ui
   asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];" : "=r"(b0), "=r"(b1) : "r"(addr));
 }
 
-__global__ void __launch_bounds__(kMergeThreads) nf4_lora_merge_kernel(
+__global__ void __launch_bounds__(kMergeThreads, 2) nf4_lora_merge_kernel(
     const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scale_codes, const float *__restrict__ c2,
     int64_t N, int64_t K, const __nv_bfloat16 *__restrict__ A, const __nv_bfloat16 *__restrict__ B, int r, float s,
     __nv_bfloat16 *__restrict__ out, int fmt) {
@@ -64,17 +68,19 @@ __global__ void __launch_bounds__(kMergeThreads) nf4_lora_merge_kernel(
   constexpr int LDA = kMergeTile + 8, LDO = kMergeTile + 8;
   __nv_bfloat16 *sB = reinterpret_cast<__nv_bfloat16 *>(merge_smem);  // [128][ldb]: B rows n0..
   __nv_bfloat16 *sA = sB + kMergeTile * ldb;                         // [r16][LDA]: A columns k0..
-  __nv_bfloat16 *sOut = sB;                                          // [128][LDO], after the MMAs
-  const size_t ops = merge_operand_bytes(r), outb = static_cast<size_t>(kMergeTile) * LDO * 2;
-  uint8_t *sCodes = merge_smem + (ops > outb ? ops : outb);          // [128][64]
-  float *sS = reinterpret_cast<float *>(sCodes + kMergeTile * 64);   // [128][2]
+  __nv_bfloat16 *sOut = sA + r16 * LDA;                              // [128][LDO]
+  uint8_t *sCodes = reinterpret_cast<uint8_t *>(sOut + kMergeTile * LDO);  // [128][64]
+  float *sS = reinterpret_cast<float *>(sCodes + kMergeTile * 64);         // [128][2]
   float *sLv = sS + kMergeTile * 2;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, q = lane & 3;
-  const int64_t n0 = (int64_t)blockIdx.y * kMergeTile, k0 = (int64_t)blockIdx.x * kMergeTile;
+  const int64_t n0 = (int64_t)blockIdx.y * kMergeTile;
+  const int64_t kt0 = (int64_t)blockIdx.x * kMergePasses;           // first column tile of this CTA
+  const int64_t ktiles = (K + kMergeTile - 1) / kMergeTile;
+  const int passes = static_cast<int>(ktiles - kt0 < kMergePasses ? ktiles - kt0 : kMergePasses);
   const int64_t nbk = K / 64;
-  const int kcols = static_cast<int>(K - k0 < kMergeTile ? K - k0 : kMergeTile);  // 64 or 128
+  const bool pre = r16 <= kMergePreR16;
 
   if (tid < 16) sLv[tid] = __uint_as_float(kNf4LevelBits[tid]);
   for (int i = tid; i < kMergeTile * (r16 / 8); i += kMergeThreads) {  // B rows (zero past N and r)
@@ -83,73 +89,120 @@ __global__ void __launch_bounds__(kMergeThreads) nf4_lora_merge_kernel(
     if (n0 + row < N && c8 < r) v = __ldg(reinterpret_cast<const uint4 *>(B + (n0 + row) * r + c8));
     *reinterpret_cast<uint4 *>(sB + row * ldb + c8) = v;
   }
-  for (int i = tid; i < r16 * (kMergeTile / 8); i += kMergeThreads) {  // A columns (zero past K and r)
-    const int j = i / (kMergeTile / 8), c8 = (i % (kMergeTile / 8)) * 8;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (j < r && c8 < kcols) v = __ldg(reinterpret_cast<const uint4 *>(A + (int64_t)j * K + k0 + c8));
-    *reinterpret_cast<uint4 *>(sA + j * LDA + c8) = v;
-  }
-  for (int i = tid; i < kMergeTile * 4; i += kMergeThreads) {  // codes (zero past N / K)
-    const int row = i >> 2, c16 = (i & 3) * 16;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (n0 + row < N && 2 * c16 < kcols)
-      v = __ldg(reinterpret_cast<const uint4 *>(codes + (n0 + row) * (K / 2) + k0 / 2 + c16));
-    *reinterpret_cast<uint4 *>(sCodes + row * 64 + c16) = v;
-  }
-  {
+
+  // One tile's A columns, codes and block scales: loaded into registers
+  // (ranks <= 64) and stored to shared memory when its space is free.
+  uint4 pa[kMergePreR16 / 16];  // A: r16 x 128 bf16 = 16 r16 bytes, 16 bytes per thread per 16 ranks
+  uint4 pc[2];                  // codes: 128 rows x 64 bytes, 32 bytes per thread
+  float ps;                     // block scale of (row tid / 2, block tid % 2)
+  auto load_tile = [&](int64_t kt) {
+    const int64_t k0 = kt * kMergeTile;
+    const int kcols = static_cast<int>(K - k0 < kMergeTile ? K - k0 : kMergeTile);
+#pragma unroll
+    for (int u = 0; u < kMergePreR16 / 16; ++u) {
+      const int i = tid + u * kMergeThreads;  // 16-byte piece i of the A tile
+      const int j = i / (kMergeTile / 8), c8 = (i % (kMergeTile / 8)) * 8;
+      pa[u] = make_uint4(0, 0, 0, 0);
+      if (j < r16 && j < r && c8 < kcols) pa[u] = __ldg(reinterpret_cast<const uint4 *>(A + (int64_t)j * K + k0 + c8));
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int i = tid + u * kMergeThreads;
+      const int row = i >> 2, c16 = (i & 3) * 16;
+      pc[u] = make_uint4(0, 0, 0, 0);
+      if (n0 + row < N && 2 * c16 < kcols)
+        pc[u] = __ldg(reinterpret_cast<const uint4 *>(codes + (n0 + row) * (K / 2) + k0 / 2 + c16));
+    }
     const int row = tid >> 1, b = tid & 1;
-    float S = 0.0f;
-    if (n0 + row < N && 64 * b < kcols) S = block_scale(scale_codes, c2, (n0 + row) * nbk + k0 / 64 + b, fmt);
-    sS[row * 2 + b] = S;
-  }
+    ps = 0.0f;
+    if (n0 + row < N && 64 * b < kcols) ps = block_scale(scale_codes, c2, (n0 + row) * nbk + k0 / 64 + b, fmt);
+  };
+  auto store_tile = [&]() {
+#pragma unroll
+    for (int u = 0; u < kMergePreR16 / 16; ++u) {
+      const int i = tid + u * kMergeThreads;
+      const int j = i / (kMergeTile / 8), c8 = (i % (kMergeTile / 8)) * 8;
+      if (j < r16) *reinterpret_cast<uint4 *>(sA + j * LDA + c8) = pa[u];
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int i = tid + u * kMergeThreads;
+      *reinterpret_cast<uint4 *>(sCodes + (i >> 2) * 64 + (i & 3) * 16) = pc[u];
+    }
+    sS[tid] = ps;
+  };
+  // ranks above 64: the A tile straight to shared memory (no prefetch)
+  auto direct_a = [&](int64_t kt) {
+    const int64_t k0 = kt * kMergeTile;
+    const int kcols = static_cast<int>(K - k0 < kMergeTile ? K - k0 : kMergeTile);
+    for (int i = tid; i < r16 * (kMergeTile / 8); i += kMergeThreads) {
+      const int j = i / (kMergeTile / 8), c8 = (i % (kMergeTile / 8)) * 8;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (j < r && c8 < kcols) v = __ldg(reinterpret_cast<const uint4 *>(A + (int64_t)j * K + k0 + c8));
+      *reinterpret_cast<uint4 *>(sA + j * LDA + c8) = v;
+    }
+  };
+
+  load_tile(kt0);
+  store_tile();
+  if (!pre) direct_a(kt0);
   __syncthreads();
 
-  // warp w: rows [16w, 16w + 16) of the tile, all 128 columns (16 n8 tiles)
   const uint32_t sB0 = static_cast<uint32_t>(__cvta_generic_to_shared(sB));
   const uint32_t sA0 = static_cast<uint32_t>(__cvta_generic_to_shared(sA));
-  float acc[kMergeTile / 8][4];
-#pragma unroll
-  for (int t = 0; t < kMergeTile / 8; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.0f;
   // A-fragment rows: lanes 0-15 rows 0..15 at column kk, lanes 16-31 the same rows at kk + 8
   const uint32_t a_row = static_cast<uint32_t>(warp * 16 + (lane & 15));
   const uint32_t a_col = static_cast<uint32_t>((lane >> 4) * 8);
+  for (int p = 0; p < passes; ++p) {
+    const int64_t k0 = (kt0 + p) * kMergeTile;
+    const int kcols = static_cast<int>(K - k0 < kMergeTile ? K - k0 : kMergeTile);
+    if (p + 1 < passes) load_tile(kt0 + p + 1);  // in flight during this tile's work
+
+    // warp w: rows [16w, 16w + 16) of the tile, all 128 columns (16 n8 tiles)
+    float acc[kMergeTile / 8][4];
 #pragma unroll
-  for (int k16 = 0; k16 < kMergeMaxK16; ++k16) {
-    if (16 * k16 >= r16) break;
-    uint32_t af[4];
-    ldmatrix_x4(af, sB0 + (a_row * ldb + 16 * k16 + a_col) * 2);
-    // B fragments: lanes 0-15 give rows kk + (lane & 15) of A's tile at column 8t
-    const uint32_t b_row = sA0 + ((16 * k16 + (lane & 15)) * LDA) * 2;
+    for (int t = 0; t < kMergeTile / 8; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.0f;
+#pragma unroll
+    for (int k16 = 0; k16 < kMergeMaxK16; ++k16) {
+      if (16 * k16 >= r16) break;
+      uint32_t af[4];
+      ldmatrix_x4(af, sB0 + (a_row * ldb + 16 * k16 + a_col) * 2);
+      // B fragments: lanes 0-15 give rows kk + (lane & 15) of A's tile at column 8t
+      const uint32_t b_row = sA0 + ((16 * k16 + (lane & 15)) * LDA) * 2;
+#pragma unroll
+      for (int t = 0; t < kMergeTile / 8; ++t) {
+        uint32_t b0, b1;
+        ldmatrix_x2_trans(b0, b1, b_row + t * 16);
+        mma_bf16_16816(acc[t], af[0], af[1], af[2], af[3], b0, b1);
+      }
+    }
+    const int r0 = warp * 16 + g, r1 = r0 + 8;
 #pragma unroll
     for (int t = 0; t < kMergeTile / 8; ++t) {
-      uint32_t b0, b1;
-      ldmatrix_x2_trans(b0, b1, b_row + t * 16);
-      mma_bf16_16816(acc[t], af[0], af[1], af[2], af[3], b0, b1);
-    }
-  }
-  __syncthreads();  // the operands are read; their space now holds the output tile
-
-  const int r0 = warp * 16 + g, r1 = r0 + 8;
+      const int c = t * 8 + 2 * q;  // C fragment: rows r0 / r1, columns c, c + 1
 #pragma unroll
-  for (int t = 0; t < kMergeTile / 8; ++t) {
-    const int c = t * 8 + 2 * q;  // C fragment: rows r0 / r1, columns c, c + 1
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int row = h ? r1 : r0;
-      const uint8_t byte = sCodes[row * 64 + (c >> 1)];
-      const float S = sS[row * 2 + (c >> 6)];
-      const float w0 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(sLv[byte & 15], S)));
-      const float w1 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(sLv[byte >> 4], S)));
-      const float v0 = __fmaf_rn(s, acc[t][2 * h], w0), v1 = __fmaf_rn(s, acc[t][2 * h + 1], w1);
-      *reinterpret_cast<uint32_t *>(sOut + row * LDO + c) = pack_bf16x2(v0, v1);
+      for (int h = 0; h < 2; ++h) {
+        const int row = h ? r1 : r0;
+        const uint8_t byte = sCodes[row * 64 + (c >> 1)];
+        const float S = sS[row * 2 + (c >> 6)];
+        const float w0 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(sLv[byte & 15], S)));
+        const float w1 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(sLv[byte >> 4], S)));
+        const float v0 = __fmaf_rn(s, acc[t][2 * h], w0), v1 = __fmaf_rn(s, acc[t][2 * h + 1], w1);
+        *reinterpret_cast<uint32_t *>(sOut + row * LDO + c) = pack_bf16x2(v0, v1);
+      }
     }
-  }
-  __syncthreads();
-  for (int i = tid; i < kMergeTile * (kMergeTile / 8); i += kMergeThreads) {
-    const int row = i / (kMergeTile / 8), c8 = (i % (kMergeTile / 8)) * 8;
-    if (n0 + row < N && c8 < kcols)
-      *reinterpret_cast<uint4 *>(out + (n0 + row) * K + k0 + c8) =
-          *reinterpret_cast<const uint4 *>(sOut + row * LDO + c8);
+    __syncthreads();  // the tile is in sOut; sA, sCodes and sS are read
+    for (int i = tid; i < kMergeTile * (kMergeTile / 8); i += kMergeThreads) {
+      const int row = i / (kMergeTile / 8), c8 = (i % (kMergeTile / 8)) * 8;
+      if (n0 + row < N && c8 < kcols)
+        *reinterpret_cast<uint4 *>(out + (n0 + row) * K + k0 + c8) =
+            *reinterpret_cast<const uint4 *>(sOut + row * LDO + c8);
+    }
+    if (p + 1 < passes) {
+      store_tile();
+      if (!pre) direct_a(kt0 + p + 1);
+    }
+    __syncthreads();  // the next tile is staged; sOut is stored
   }
 }
 

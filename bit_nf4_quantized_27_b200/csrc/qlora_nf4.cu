@@ -789,7 +789,8 @@ qlora_status qlora_lora_merge(const qlora_nf4_tensor *W, const qlora_lora *adapt
   if ((s = set_smem(nf4_lora_merge_kernel, static_cast<int>(merge_smem_bytes(QLORA_MAX_RANK)), dev, flags,
                     results)) != QLORA_OK)
     return s;
-  const dim3 grid(static_cast<unsigned>((W->cols + kMergeTile - 1) / kMergeTile),
+  const int64_t ktiles = (W->cols + kMergeTile - 1) / kMergeTile;
+  const dim3 grid(static_cast<unsigned>((ktiles + kMergePasses - 1) / kMergePasses),
                   static_cast<unsigned>((W->rows + kMergeTile - 1) / kMergeTile));
   const float sc = adapter->alpha / static_cast<float>(adapter->r);
   nf4_lora_merge_kernel<<<grid, kMergeThreads, bytes, reinterpret_cast<cudaStream_t>(stream)>>>(
