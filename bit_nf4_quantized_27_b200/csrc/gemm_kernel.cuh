@@ -267,6 +267,8 @@ __device__ __forceinline__ void store_chunk32(const GemmArgs &args, int row, int
 // writes the outputs exactly as the GEMM epilogue does (out = v * out_scale;
 // hi = bf16(v * hl_scale), lo = bf16(v * hl_scale - hi)).  Two columns per thread.
 __global__ void splitk_finish_kernel(const GemmArgs args) {
+  ptx::griddep_launch();
+  ptx::griddep_wait();  // the partial planes are complete
   const int64_t pairs = (int64_t)args.M_rows * args.N_cols / 2;
   const int64_t plane = (int64_t)args.M_rows * args.N_cols;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < pairs; i += (int64_t)gridDim.x * blockDim.x) {
@@ -352,6 +354,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // The set-up above overlaps the preceding kernel's tail; every global read and
+  // write below comes after that kernel has completed.
+  ptx::griddep_launch();
+  ptx::griddep_wait();
 
   const int tile_n = args.hilo_cols ? BN / 2 : BN;  // output columns per tile
   const int num_m = (args.M_rows + C::BM * MT - 1) / (C::BM * MT);

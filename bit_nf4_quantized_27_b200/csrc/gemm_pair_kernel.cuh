@@ -108,6 +108,10 @@ gemm_nf4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
   ptx::cluster_sync();  // both CTAs' barriers are initialised before any cross-CTA signal
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // The set-up above overlaps the preceding kernel's tail; every global read and
+  // write below comes after that kernel has completed.
+  ptx::griddep_launch();
+  ptx::griddep_wait();
 
   // Tiles of 2*128*MT tokens x 256 columns, handed out round-robin to the
   // clusters.  When the last round would leave at least half of the clusters

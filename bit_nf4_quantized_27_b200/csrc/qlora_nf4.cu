@@ -102,6 +102,28 @@ bool tmap_bf16(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer, 
   return make_tmap(m, ptr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, inner, outer, inner, box_inner, box_outer, true);
 }
 
+// Launch with programmatic dependent launch allowed: the kernel's set-up
+// overlaps the preceding kernel's tail, and the kernel waits for that kernel
+// (griddepcontrol.wait) before it touches global memory.
+template <typename... KArgs, typename... Args>
+qlora_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, int smem, cudaStream_t st, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) != cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  return QLORA_OK;
+}
+
 // Once per device and kernel: allow the kernel's dynamic shared memory.
 template <typename F>
 qlora_status set_smem(F kernel, int bytes, int dev, std::once_flag *flags, qlora_status *results) {
@@ -128,16 +150,18 @@ qlora_status launch_gemm_pair(const CUtensorMap &tmA, const CUtensorMap &tmA2, c
   qlora_status s = set_smem(kernel, C::SMEM_BYTES, dev, flags, results);
   if (s != QLORA_OK) return s;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(C::THREADS);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = st;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 1;  // the cluster shape alone for the occupancy query
   std::call_once(occ_flags[dev], [&] {
     cudaLaunchConfig_t q = cfg;
     q.gridDim = dim3(2);
@@ -151,6 +175,7 @@ qlora_status launch_gemm_pair(const CUtensorMap &tmA, const CUtensorMap &tmA2, c
   const int num_n = (args.N_cols + C::BN - 1) / C::BN;
   const int clusters = std::max(1, std::min(num_m * num_n, max_clusters[dev]));
   cfg.gridDim = dim3(2 * clusters);
+  cfg.numAttrs = 2;  // and programmatic dependent launch
   if (cudaLaunchKernelEx(&cfg, kernel, tmA, tmA2, tmCodes, args) != cudaSuccess) {
     cudaGetLastError();
     return QLORA_ERR_CUDA;
@@ -176,8 +201,7 @@ qlora_status launch_gemm(const CUtensorMap &tmA, const CUtensorMap &tmB, const C
   const int num_n = (args.N_cols + tile_n - 1) / tile_n;
   const int tiles = num_m * num_n * std::max(1, args.ksplit);
   const int grid = std::max(1, std::min(tiles, sms));
-  kernel<<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tmA, tmB, tmA2, tmB2, tmCodes, args);
-  return launch_status();
+  return launch_pdl(kernel, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, st, tmA, tmB, tmA2, tmB2, tmCodes, args);
 }
 
 uint32_t *status_ptr(void *ws) { return reinterpret_cast<uint32_t *>(ws); }
@@ -220,8 +244,7 @@ qlora_status launch_rank_gemm(const CUtensorMap &tmA, const CUtensorMap &tmB, Ge
   if (s != QLORA_OK) return s;
   const int64_t pairs = (int64_t)g.M_rows * g.N_cols / 2;
   const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>((pairs + 255) / 256, (int64_t)sms * 8));
-  splitk_finish_kernel<<<grid, 256, 0, st>>>(g);
-  return launch_status();
+  return launch_pdl(splitk_finish_kernel, dim3(grid), dim3(256), 0, st, g);
 }
 
 qlora_status run_lora_down(const void *X, const qlora_lora *ad, int64_t M, int64_t K, float s, void *sT,
