@@ -744,26 +744,54 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   }
   __syncthreads();
   const __nv_bfloat16 *const sT = a.sT + griddep_wait_token();
-  if (lora_rg >= 0 && a.multi) {
-    // one adapter per token: row (lane & 15) of this row group, half of the
-    // rank range per half-warp, combined by a shuffle (fixed order)
-    const int64_t n = (int64_t)(rg0 + lora_rg) * 16 + (lane & 15);
+  if (a.multi) {
+    // one adapter per token: tasks (row group, token) spread over all warps, two
+    // tasks in flight per warp with every load of a round issued before its
+    // products.  Lane
+    // = row (lane & 15) of the row group, half of the rank range per half-warp,
+    // combined by a shuffle (fixed order); each task adds its own token's column.
     const int half = lane >> 4, hr = a.r / 2;  // r % 8 == 0: hr is a multiple of 4
-    float *rb = red_at(lora_rg);  // warp 0's slot
-    for (int t = 0; t < a.M; ++t) {
-      const __nv_bfloat16 *bt = a.ml.B[t] + n * a.r + half * hr;
-      const __nv_bfloat16 *st = sT + (int64_t)t * a.r + half * hr;
-      float acc = 0.0f;
-      for (int j = 0; j < hr; j += 4) {
-        const uint2 bv = __ldg(reinterpret_cast<const uint2 *>(bt + j));
-        const uint2 sv = __ldca(reinterpret_cast<const uint2 *>(st + j));
-        acc = fmaf(bf16lo_to_f32(bv.x), bf16lo_to_f32(sv.x), acc);
-        acc = fmaf(bf16hi_to_f32(bv.x), bf16hi_to_f32(sv.x), acc);
-        acc = fmaf(bf16lo_to_f32(bv.y), bf16lo_to_f32(sv.y), acc);
-        acc = fmaf(bf16hi_to_f32(bv.y), bf16hi_to_f32(sv.y), acc);
+    const int ntask = my_rg * a.M;
+    for (int k0 = warp; k0 < ntask; k0 += 2 * kGemvWarps) {
+      float acc[2] = {0.0f, 0.0f};
+      // 16 ranks per round: four 8-byte loads of B and of s T per task (the half
+      // rank range starts 8-byte aligned: r % 8 == 0)
+      for (int j = 0; j < hr; j += 16) {
+        uint2 bv[2][4], sv[2][4];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int k = k0 + u * kGemvWarps;
+          const bool live = k < ntask;
+          const int i = live ? k / a.M : 0, t = live ? k - i * a.M : 0;
+          const int64_t n = (int64_t)(rg0 + i) * 16 + (lane & 15);
+          const __nv_bfloat16 *bt = a.ml.B[t] + n * a.r + half * hr + j;
+          const __nv_bfloat16 *st = sT + (int64_t)t * a.r + half * hr + j;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const bool in = live && j + 4 * c < hr;
+            bv[u][c] = in ? __ldg(reinterpret_cast<const uint2 *>(bt + 4 * c)) : make_uint2(0, 0);
+            sv[u][c] = in ? __ldca(reinterpret_cast<const uint2 *>(st + 4 * c)) : make_uint2(0, 0);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            acc[u] = fmaf(bf16lo_to_f32(bv[u][c].x), bf16lo_to_f32(sv[u][c].x), acc[u]);
+            acc[u] = fmaf(bf16hi_to_f32(bv[u][c].x), bf16hi_to_f32(sv[u][c].x), acc[u]);
+            acc[u] = fmaf(bf16lo_to_f32(bv[u][c].y), bf16lo_to_f32(sv[u][c].y), acc[u]);
+            acc[u] = fmaf(bf16hi_to_f32(bv[u][c].y), bf16hi_to_f32(sv[u][c].y), acc[u]);
+          }
       }
-      acc += __shfl_xor_sync(0xffffffffu, acc, 16);
-      if (half == 0) rb[(lane & 15) * TR + t] += acc;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int k = k0 + u * kGemvWarps;
+        const float v = acc[u] + __shfl_xor_sync(0xffffffffu, acc[u], 16);
+        if (k < ntask && half == 0) {
+          const int i = k / a.M, t = k - i * a.M;
+          red_at(i)[(lane & 15) * TR + t] += v;  // warp 0's slot of row group i
+        }
+      }
     }
   }
   if (lora_rg >= 0 && !a.multi) {
