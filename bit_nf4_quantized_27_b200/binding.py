@@ -87,6 +87,7 @@ def lib():
         "qlora_selftest_bounded_wait": (ctypes.c_int, [vp, ctypes.c_uint32, vp]),
         "qlora_clear_status": (ctypes.c_int, [vp, vp]),
         "qlora_read_status": (ctypes.c_int, [vp, vp]),
+        "qlora_read_library_status": (ctypes.c_int, [vp]),
         "qlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     }
     for name, (res, args) in sigs.items():
@@ -256,6 +257,12 @@ def clear_status(ws: torch.Tensor, stream=None):
 def read_status(ws: torch.Tensor, stream=None) -> int:
     """Synchronises the stream and returns the device status code (0 = ok)."""
     return int(lib().qlora_read_status(_ptr(ws), _stream(stream)))
+
+
+def read_library_status(stream=None) -> int:
+    """Synchronises the stream, returns and clears the status code of the calls
+    without a workspace (the merged export) on the current device (0 = ok)."""
+    return int(lib().qlora_read_library_status(_stream(stream)))
 
 
 class QLoRALinearFunction(torch.autograd.Function):

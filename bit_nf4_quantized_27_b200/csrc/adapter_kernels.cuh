@@ -9,200 +9,295 @@
 //   the update is decoupled-weight-decay Adam with bias correction.
 #pragma once
 
+#include "gemm_kernel.cuh"
 #include "nf4_device.cuh"
+#include "sm100_ptx.cuh"
 
 namespace qlora {
 
 // ---------------------------------------------------------------------------
-// Merged export.  One CTA (8 warps) makes kMergePasses consecutive 128 x 128
-// tiles of one 128-row block of W_merged: the low-rank product s B A on
-// mma.sync tensor cores (bf16 in, fp32 accumulate) from shared-memory copies of
-// B's 128 rows (staged once per CTA) and of A's columns of the tile (both
-// row-major, rows padded by 16 bytes so ldmatrix reads are conflict-free; A's
-// fragments come transposed by ldmatrix.trans); W' decoded from the tile's
-// codes and block scales staged in shared memory; the sum in fp32, rounded to
-// bf16 once, staged in shared memory and stored with 16-byte writes.  For ranks
-// up to 64 the next tile's A columns, codes and scales are loaded into
-// registers while the current tile is computed and stored.
-// HBM traffic per weight: 0.5 B of code + 1/64 B of scale + 2 B written.
+// Merged export on the tensor cores (tcgen05, accumulators in TMEM).  Persistent
+// CTAs walk the 128-row x 256-column tiles of W_merged.  Per tile:
+//   * warp 0 (one thread) loads by TMA, per 64 ranks, B's 128 rows (K-major)
+//     and A's 64 x 256 block (MN-major); warp 2 (one thread) loads the tile's
+//     NF4 codes (128 rows x 128 bytes, 128-byte swizzle) up to four tiles ahead;
+//   * warp 1 (one thread) issues tcgen05.mma M = 128, N = 256, K = 16 into one
+//     of two TMEM accumulators: (B A)[n0.., k0..] in float32;
+//   * warps 4..19 (TMEM lane quadrant warp % 4, 64-column quarter (warp - 4) / 4
+//     of the tile) read accumulator rows with tcgen05.ld, decode W' from the
+//     codes and the block scale, form fma(s, (B A), W') in float32, round once
+//     to bf16 and write the tile through a swizzled shared-memory buffer that a
+//     TMA store copies out (clipped at the matrix edge).  Sixteen epilogue warps
+//     (four per scheduler) keep the decode, which is the longest step, fed.
+// Loads, products, the epilogue and the stores of consecutive tiles overlap.
+// HBM traffic per weight: 0.5 B of code + 1/64 B of scale + 2 B written; the
+// adapter's tiles come from L2.  Every wait is bounded; one that gives up
+// records QLORA_ERR_TIMEOUT in the status word, the other roles leave, copies
+// and products in flight are drained and TMEM is freed.
 // ---------------------------------------------------------------------------
-constexpr int kMergeThreads = 256;
-constexpr int kMergeTile = 128;
-constexpr int kMergeMaxK16 = 16;  // r <= 256
-constexpr int kMergePasses = 4;   // column tiles per CTA
-constexpr int kMergePreR16 = 64;  // ranks whose next A tile fits the prefetch registers
+constexpr int kMergeBM = 128;
+constexpr int kMergeBN = 256;
+constexpr int kMergeThreads = 640;
+constexpr int kMergeEpiWarps = 16;
+constexpr int kMergeSAB = 2;  // stages of (B rows, A block) per 64 ranks
+constexpr int kMergeSC = 4;   // stages of codes
+constexpr uint32_t kMergeAStage = kMergeBM * 64 * 2;  // B rows: 128 x 64 ranks
+constexpr uint32_t kMergeBStage = 64 * kMergeBN * 2;  // A block: 64 ranks x 256 columns
+constexpr uint32_t kMergeABStage = kMergeAStage + kMergeBStage;
+constexpr uint32_t kMergeCStage = kMergeBM * 128;  // codes: 128 rows x 256 columns / 2
+constexpr uint32_t kMergeOutBuf = 32 * 128;         // 32 rows x 64 columns of bf16
+constexpr uint32_t kMergeOutBytes = kMergeEpiWarps * kMergeOutBuf;
+constexpr uint32_t kMergeSmemBytes =
+    kMergeSAB * kMergeABStage + kMergeSC * kMergeCStage + kMergeOutBytes + 1024 /*align*/ + 256 /*barriers*/;
+constexpr uint32_t kMergeTmemCols = 2 * kMergeBN;
+constexpr uint32_t kMergeIdesc = ptx::idesc_bf16(kMergeBM, kMergeBN, 0, 1);
+static_assert(kMergeSmemBytes <= 227 * 1024, "shared memory");
 
-__host__ __device__ inline int merge_r16(int r) { return ((r + 15) / 16) * 16; }
-__host__ __device__ inline size_t merge_operand_bytes(int r) {
-  return static_cast<size_t>(kMergeTile) * (merge_r16(r) + 8) * 2        // B rows [128][r16 + 8]
-         + static_cast<size_t>(merge_r16(r)) * (kMergeTile + 8) * 2;     // A tile [r16][136]
-}
-inline size_t merge_smem_bytes(int r) {
-  const size_t outb = static_cast<size_t>(kMergeTile) * (kMergeTile + 8) * 2;  // bf16 [128][136]
-  return merge_operand_bytes(r) + outb + kMergeTile * 64 + kMergeTile * 2 * 4 + 16 * 4;
-}
+struct MergeArgs {
+  const uint8_t *scale_codes;
+  const float *c2;
+  int64_t N, K;
+  int r;
+  float s;  // alpha / r
+  int fmt;  // qlora_scale_format
+  uint32_t *status;
+};
 
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                               uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-      "{%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldmatrix_x2_trans(uint32_t &b0, uint32_t &b1, uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];" : "=r"(b0), "=r"(b1) : "r"(addr));
-}
+__global__ void __launch_bounds__(kMergeThreads, 1)
+    nf4_lora_merge_kernel(const __grid_constant__ CUtensorMap tmCodes, const __grid_constant__ CUtensorMap tmB,
+                          const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmOut,
+                          const MergeArgs a) {
+  extern __shared__ uint8_t merge_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(merge_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sAB = smem;
+  uint8_t *sC = sAB + kMergeSAB * kMergeABStage;
+  uint8_t *sOut = sC + kMergeSC * kMergeCStage;
+  uint64_t *full_ab = reinterpret_cast<uint64_t *>(sOut + kMergeOutBytes);
+  uint64_t *empty_ab = full_ab + kMergeSAB;
+  uint64_t *full_c = empty_ab + kMergeSAB;
+  uint64_t *empty_c = full_c + kMergeSC;
+  uint64_t *acc_full = empty_c + kMergeSC;
+  uint64_t *acc_empty = acc_full + 2;
+  uint64_t *drain = acc_empty + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
-__global__ void __launch_bounds__(kMergeThreads, 2) nf4_lora_merge_kernel(
-    const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scale_codes, const float *__restrict__ c2,
-    int64_t N, int64_t K, const __nv_bfloat16 *__restrict__ A, const __nv_bfloat16 *__restrict__ B, int r, float s,
-    __nv_bfloat16 *__restrict__ out, int fmt) {
-  extern __shared__ __align__(16) uint8_t merge_smem[];
-  const int r16 = merge_r16(r), ldb = r16 + 8;
-  constexpr int LDA = kMergeTile + 8, LDO = kMergeTile + 8;
-  __nv_bfloat16 *sB = reinterpret_cast<__nv_bfloat16 *>(merge_smem);  // [128][ldb]: B rows n0..
-  __nv_bfloat16 *sA = sB + kMergeTile * ldb;                         // [r16][LDA]: A columns k0..
-  __nv_bfloat16 *sOut = sA + r16 * LDA;                              // [128][LDO]
-  uint8_t *sCodes = reinterpret_cast<uint8_t *>(sOut + kMergeTile * LDO);  // [128][64]
-  float *sS = reinterpret_cast<float *>(sCodes + kMergeTile * 64);         // [128][2]
-  float *sLv = sS + kMergeTile * 2;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kMergeSAB; ++i) { ptx::mbar_init(&full_ab[i], 1); ptx::mbar_init(&empty_ab[i], 1); }
+    for (int i = 0; i < kMergeSC; ++i) {
+      ptx::mbar_init(&full_c[i], 1);
+      ptx::mbar_init(&empty_c[i], kMergeEpiWarps);
+    }
+    for (int i = 0; i < 2; ++i) { ptx::mbar_init(&acc_full[i], 1); ptx::mbar_init(&acc_empty[i], kMergeEpiWarps); }
+    ptx::mbar_init(drain, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    ptx::prefetch_tmap(&tmCodes);
+    ptx::prefetch_tmap(&tmB);
+    ptx::prefetch_tmap(&tmA);
+    ptx::prefetch_tmap(&tmOut);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, kMergeTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, q = lane & 3;
-  const int64_t n0 = (int64_t)blockIdx.y * kMergeTile;
-  const int64_t kt0 = (int64_t)blockIdx.x * kMergePasses;           // first column tile of this CTA
-  const int64_t ktiles = (K + kMergeTile - 1) / kMergeTile;
-  const int passes = static_cast<int>(ktiles - kt0 < kMergePasses ? ktiles - kt0 : kMergePasses);
-  const int64_t nbk = K / 64;
-  const bool pre = r16 <= kMergePreR16;
+  const int64_t N = a.N, K = a.K;
+  const int64_t ncol = (K + kMergeBN - 1) / kMergeBN;
+  const int64_t tiles = ((N + kMergeBM - 1) / kMergeBM) * ncol;
+  const int rsteps = (a.r + 63) / 64;
+  auto tile_of = [&](int64_t t, int64_t &n0, int64_t &k0) {
+    n0 = (t / ncol) * kMergeBM;
+    k0 = (t % ncol) * kMergeBN;
+  };
+  auto fail = [&]() {
+    raise_status(a.status, QLORA_ERR_TIMEOUT);
+    *abort_flag = 1;
+  };
 
-  if (tid < 16) sLv[tid] = __uint_as_float(kNf4LevelBits[tid]);
-  for (int i = tid; i < kMergeTile * (r16 / 8); i += kMergeThreads) {  // B rows (zero past N and r)
-    const int row = i / (r16 / 8), c8 = (i % (r16 / 8)) * 8;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (n0 + row < N && c8 < r) v = __ldg(reinterpret_cast<const uint4 *>(B + (n0 + row) * r + c8));
-    *reinterpret_cast<uint4 *>(sB + row * ldb + c8) = v;
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer: adapter tiles
+    if (ptx::elect_one()) {
+      uint32_t sab = 0, pab = 0;
+      int issued_ab = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+        int64_t n0, k0;
+        tile_of(t, n0, k0);
+        for (int j = 0; j < rsteps; ++j) {
+          if (!ptx::mbar_wait(&empty_ab[sab], pab ^ 1, abort_flag)) { ok = false; break; }
+          ptx::mbar_arrive_expect_tx(&full_ab[sab], kMergeABStage);
+          uint8_t *d = sAB + sab * kMergeABStage;
+          ptx::tma_load_2d(d, &tmB, &full_ab[sab], 64 * j, static_cast<int32_t>(n0));
+          for (int u = 0; u < kMergeBN / 64; ++u)
+            ptx::tma_load_2d(d + kMergeAStage + u * 8192, &tmA, &full_ab[sab], static_cast<int32_t>(k0 + 64 * u),
+                             64 * j);
+          ++issued_ab;
+          if (++sab == kMergeSAB) { sab = 0; pab ^= 1; }
+        }
+      }
+      if (!ok) fail();
+      // the last (up to) kMergeSAB copies must land before the CTA exits
+      for (int i = 0; i < kMergeSAB && i < issued_ab; ++i) {
+        if (sab == 0) { sab = kMergeSAB - 1; pab ^= 1; } else { --sab; }
+        ptx::mbar_wait(&full_ab[sab], pab, nullptr);
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ TMA producer: codes
+    if (ptx::elect_one()) {
+      uint32_t sc = 0, pc = 0;
+      int issued_c = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
+        int64_t n0, k0;
+        tile_of(t, n0, k0);
+        if (!ptx::mbar_wait(&empty_c[sc], pc ^ 1, abort_flag)) { ok = false; break; }
+        ptx::mbar_arrive_expect_tx(&full_c[sc], kMergeCStage);
+        ptx::tma_load_2d(sC + sc * kMergeCStage, &tmCodes, &full_c[sc], static_cast<int32_t>(k0 / 2),
+                         static_cast<int32_t>(n0));
+        ++issued_c;
+        if (++sc == kMergeSC) { sc = 0; pc ^= 1; }
+      }
+      if (!ok) fail();
+      for (int i = 0; i < kMergeSC && i < issued_c; ++i) {
+        if (sc == 0) { sc = kMergeSC - 1; pc ^= 1; } else { --sc; }
+        ptx::mbar_wait(&full_c[sc], pc, nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (ptx::elect_one()) {
+      uint32_t sab = 0, pab = 0;
+      int it = 0;
+      bool ok = true;
+      const uint32_t sAB0 = ptx::smem_addr(sAB);
+      for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++it) {
+        const int acc = it & 1;
+        if (!ptx::mbar_wait(&acc_empty[acc], ((it >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * kMergeBN;
+        for (int j = 0; j < rsteps; ++j) {
+          if (!ptx::mbar_wait(&full_ab[sab], pab, abort_flag)) { ok = false; break; }
+          ptx::tc_fence_after();
+          const uint32_t a_base = sAB0 + sab * kMergeABStage, b_base = a_base + kMergeAStage;
+#pragma unroll
+          for (int k16 = 0; k16 < 4; ++k16)
+            ptx::mma_bf16(d_tmem, ptx::smem_desc_sw128(a_base + k16 * 32, 16, 1024),
+                          ptx::smem_desc_sw128(b_base + k16 * 2048, 8192, 1024), kMergeIdesc, (j | k16) ? 1u : 0u);
+          ptx::mma_commit(&empty_ab[sab]);
+          if (++sab == kMergeSAB) { sab = 0; pab ^= 1; }
+        }
+        if (ok) ptx::mma_commit(&acc_full[acc]);
+      }
+      if (!ok) fail();
+      ptx::mma_commit(drain);  // every product issued has completed
+      ptx::mbar_wait(drain, 0, nullptr);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue
+    const int e = warp - 4, qd = warp & 3, cq = e >> 2;
+    const int row_t = qd * 32 + lane;  // tile row of this thread (TMEM lane)
+    uint8_t *buf = sOut + e * kMergeOutBuf;
+    const int64_t nbk = K / 64;
+    // scale code and second-level constant of this thread's row in its 64-column
+    // block of tile t: loaded one tile ahead (the raw values, so that nothing
+    // waits for the loads until the tile that uses them)
+    auto scale_src = [&](int64_t t, uint32_t &qv, float &cv) {
+      qv = 0u;
+      cv = 0.0f;
+      if (t >= tiles) return;
+      int64_t n0, k0;
+      tile_of(t, n0, k0);
+      const int64_t n = n0 + row_t, kb = k0 / 64 + cq;
+      if (n < N && kb < nbk) {
+        const int64_t b = n * nbk + kb;
+        qv = __ldg(a.scale_codes + b);
+        cv = __ldg(a.c2 + (b >> 8));
+      }
+    };
+    uint32_t qv;
+    float cv;
+    scale_src(blockIdx.x, qv, cv);
+    uint32_t sc = 0, pc = 0;
+    int it = 0;
+    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
+      int64_t n0, k0;
+      tile_of(t, n0, k0);
+      const float S = __fmul_rn(scale_code_value(qv, a.fmt), cv);  // S' = fl32(code value * c2)
+      scale_src(t + gridDim.x, qv, cv);
+      const int acc = it & 1;
+      const bool ready = ptx::mbar_wait(&full_c[sc], pc, abort_flag) &&
+                         ptx::mbar_wait(&acc_full[acc], (it >> 1) & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, ready)) {  // the warp leaves together (its TMEM loads are warp-wide)
+        if (lane == 0) fail();
+        break;
+      }
+      ptx::tc_fence_after();
+      // codes of columns 64 cq .. +63 of the row: 16-byte chunks 2 cq, 2 cq + 1
+      const uint8_t *crow = sC + sc * kMergeCStage + row_t * 128;
+      const uint4 c0 = *reinterpret_cast<const uint4 *>(crow + (((2 * cq) ^ (row_t & 7)) << 4));
+      const uint4 c1 = *reinterpret_cast<const uint4 *>(crow + (((2 * cq + 1) ^ (row_t & 7)) << 4));
+      uint32_t lo[4], hi[4];
+      nf4_planes(S, lo, hi);
+      const uint32_t tcol = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) + acc * kMergeBN + cq * 64;
+      // the store that last read the buffer (one tile back) has finished reading it
+      if (lane == 0) ptx::bulk_wait_read0();
+      __syncwarp();
+#pragma unroll
+      for (int qi = 0; qi < 2; ++qi) {  // 32 columns at a time
+        uint32_t v[32];
+        ptx::tmem_ld32(tcol + 32 * qi, v);
+        const uint32_t cw[4] = {qi ? c1.x : c0.x, qi ? c1.y : c0.y, qi ? c1.z : c0.z, qi ? c1.w : c0.w};
+        uint32_t w[16];  // W' of columns 32 qi + 2i, + 1 (bf16 pairs)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) nf4_word(cw[j], lo, hi, w + 4 * j);
+        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {  // 8 columns per 16-byte chunk
+          uint32_t pk[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t wp = w[4 * c + i];
+            pk[i] = pack_bf16x2(__fmaf_rn(a.s, __uint_as_float(v[8 * c + 2 * i]), bf16lo_to_f32(wp)),
+                                __fmaf_rn(a.s, __uint_as_float(v[8 * c + 2 * i + 1]), bf16hi_to_f32(wp)));
+          }
+          const int chunk = 4 * qi + c;
+          *reinterpret_cast<uint4 *>(buf + lane * 128 + ((chunk ^ (lane & 7)) << 4)) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+      }
+      // this tile's codes and accumulator are read
+      ptx::tc_fence_before();
+      ptx::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        ptx::mbar_arrive(&empty_c[sc]);
+        ptx::mbar_arrive(&acc_empty[acc]);
+        const int64_t x = k0 + cq * 64, y = n0 + qd * 32;
+        if (x < K && y < N) {
+          ptx::tma_store_2d(&tmOut, buf, static_cast<int32_t>(x), static_cast<int32_t>(y));
+          ptx::bulk_commit();
+        }
+      }
+      if (++sc == kMergeSC) { sc = 0; pc ^= 1; }
+    }
+    if (lane == 0) ptx::bulk_wait_all();  // the stores have completed
+    __syncwarp();
   }
 
-  // One tile's A columns, codes and block scales: loaded into registers
-  // (ranks <= 64) and stored to shared memory when its space is free.
-  uint4 pa[kMergePreR16 / 16];  // A: r16 x 128 bf16 = 16 r16 bytes, 16 bytes per thread per 16 ranks
-  uint4 pc[2];                  // codes: 128 rows x 64 bytes, 32 bytes per thread
-  float ps;                     // block scale of (row tid / 2, block tid % 2)
-  auto load_tile = [&](int64_t kt) {
-    const int64_t k0 = kt * kMergeTile;
-    const int kcols = static_cast<int>(K - k0 < kMergeTile ? K - k0 : kMergeTile);
-#pragma unroll
-    for (int u = 0; u < kMergePreR16 / 16; ++u) {
-      const int i = tid + u * kMergeThreads;  // 16-byte piece i of the A tile
-      const int j = i / (kMergeTile / 8), c8 = (i % (kMergeTile / 8)) * 8;
-      pa[u] = make_uint4(0, 0, 0, 0);
-      if (j < r16 && j < r && c8 < kcols) pa[u] = __ldg(reinterpret_cast<const uint4 *>(A + (int64_t)j * K + k0 + c8));
-    }
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int i = tid + u * kMergeThreads;
-      const int row = i >> 2, c16 = (i & 3) * 16;
-      pc[u] = make_uint4(0, 0, 0, 0);
-      if (n0 + row < N && 2 * c16 < kcols)
-        pc[u] = __ldg(reinterpret_cast<const uint4 *>(codes + (n0 + row) * (K / 2) + k0 / 2 + c16));
-    }
-    const int row = tid >> 1, b = tid & 1;
-    ps = 0.0f;
-    if (n0 + row < N && 64 * b < kcols) ps = block_scale(scale_codes, c2, (n0 + row) * nbk + k0 / 64 + b, fmt);
-  };
-  auto store_tile = [&]() {
-#pragma unroll
-    for (int u = 0; u < kMergePreR16 / 16; ++u) {
-      const int i = tid + u * kMergeThreads;
-      const int j = i / (kMergeTile / 8), c8 = (i % (kMergeTile / 8)) * 8;
-      if (j < r16) *reinterpret_cast<uint4 *>(sA + j * LDA + c8) = pa[u];
-    }
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int i = tid + u * kMergeThreads;
-      *reinterpret_cast<uint4 *>(sCodes + (i >> 2) * 64 + (i & 3) * 16) = pc[u];
-    }
-    sS[tid] = ps;
-  };
-  // ranks above 64: the A tile straight to shared memory (no prefetch)
-  auto direct_a = [&](int64_t kt) {
-    const int64_t k0 = kt * kMergeTile;
-    const int kcols = static_cast<int>(K - k0 < kMergeTile ? K - k0 : kMergeTile);
-    for (int i = tid; i < r16 * (kMergeTile / 8); i += kMergeThreads) {
-      const int j = i / (kMergeTile / 8), c8 = (i % (kMergeTile / 8)) * 8;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (j < r && c8 < kcols) v = __ldg(reinterpret_cast<const uint4 *>(A + (int64_t)j * K + k0 + c8));
-      *reinterpret_cast<uint4 *>(sA + j * LDA + c8) = v;
-    }
-  };
-
-  load_tile(kt0);
-  store_tile();
-  if (!pre) direct_a(kt0);
+  ptx::tc_fence_before();
   __syncthreads();
-
-  const uint32_t sB0 = static_cast<uint32_t>(__cvta_generic_to_shared(sB));
-  const uint32_t sA0 = static_cast<uint32_t>(__cvta_generic_to_shared(sA));
-  // A-fragment rows: lanes 0-15 rows 0..15 at column kk, lanes 16-31 the same rows at kk + 8
-  const uint32_t a_row = static_cast<uint32_t>(warp * 16 + (lane & 15));
-  const uint32_t a_col = static_cast<uint32_t>((lane >> 4) * 8);
-  for (int p = 0; p < passes; ++p) {
-    const int64_t k0 = (kt0 + p) * kMergeTile;
-    const int kcols = static_cast<int>(K - k0 < kMergeTile ? K - k0 : kMergeTile);
-    if (p + 1 < passes) load_tile(kt0 + p + 1);  // in flight during this tile's work
-
-    // warp w: rows [16w, 16w + 16) of the tile, all 128 columns (16 n8 tiles)
-    float acc[kMergeTile / 8][4];
-#pragma unroll
-    for (int t = 0; t < kMergeTile / 8; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.0f;
-#pragma unroll
-    for (int k16 = 0; k16 < kMergeMaxK16; ++k16) {
-      if (16 * k16 >= r16) break;
-      uint32_t af[4];
-      ldmatrix_x4(af, sB0 + (a_row * ldb + 16 * k16 + a_col) * 2);
-      // B fragments: lanes 0-15 give rows kk + (lane & 15) of A's tile at column 8t
-      const uint32_t b_row = sA0 + ((16 * k16 + (lane & 15)) * LDA) * 2;
-#pragma unroll
-      for (int t = 0; t < kMergeTile / 8; ++t) {
-        uint32_t b0, b1;
-        ldmatrix_x2_trans(b0, b1, b_row + t * 16);
-        mma_bf16_16816(acc[t], af[0], af[1], af[2], af[3], b0, b1);
-      }
-    }
-    const int r0 = warp * 16 + g, r1 = r0 + 8;
-#pragma unroll
-    for (int t = 0; t < kMergeTile / 8; ++t) {
-      const int c = t * 8 + 2 * q;  // C fragment: rows r0 / r1, columns c, c + 1
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int row = h ? r1 : r0;
-        const uint8_t byte = sCodes[row * 64 + (c >> 1)];
-        const float S = sS[row * 2 + (c >> 6)];
-        const float w0 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(sLv[byte & 15], S)));
-        const float w1 = __bfloat162float(__float2bfloat16_rn(__fmul_rn(sLv[byte >> 4], S)));
-        const float v0 = __fmaf_rn(s, acc[t][2 * h], w0), v1 = __fmaf_rn(s, acc[t][2 * h + 1], w1);
-        *reinterpret_cast<uint32_t *>(sOut + row * LDO + c) = pack_bf16x2(v0, v1);
-      }
-    }
-    __syncthreads();  // the tile is in sOut; sA, sCodes and sS are read
-    for (int i = tid; i < kMergeTile * (kMergeTile / 8); i += kMergeThreads) {
-      const int row = i / (kMergeTile / 8), c8 = (i % (kMergeTile / 8)) * 8;
-      if (n0 + row < N && c8 < kcols)
-        *reinterpret_cast<uint4 *>(out + (n0 + row) * K + k0 + c8) =
-            *reinterpret_cast<const uint4 *>(sOut + row * LDO + c8);
-    }
-    if (p + 1 < passes) {
-      store_tile();
-      if (!pre) direct_a(kt0 + p + 1);
-    }
-    __syncthreads();  // the next tile is staged; sOut is stored
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, kMergeTmemCols);
   }
 }
 

@@ -92,36 +92,46 @@ __device__ __forceinline__ uint32_t sw128_row_chunk(uint32_t row, uint32_t c) {
   return (row & 7u) * 128u + ((c ^ (row & 7u)) << 4);
 }
 
-// Decode 64 NF4 codes (two uint4 of packed nibbles) with block scale S into 32
-// packed bf16x2 words, via a per-block table of the 16 products split into byte
-// planes and looked up with byte permutes.
-__device__ __forceinline__ void nf4_decode64(const uint4 &c0, const uint4 &c1, float S, uint32_t (&o)[32]) {
+// Table of the 16 products bf16(L[c] * S) of one block, split into byte planes:
+// lo[j] / hi[j] hold the low / high bytes of entries 4j .. 4j + 3.
+__device__ __forceinline__ void nf4_planes(float S, uint32_t (&lo)[4], uint32_t (&hi)[4]) {
   uint32_t p[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) p[j] = pack_bf16x2(__fmul_rn(nf4_level(2 * j), S), __fmul_rn(nf4_level(2 * j + 1), S));
-  // lo/hi byte planes of entries 0-3, 4-7, 8-11, 12-15
-  uint32_t lo[4], hi[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     lo[j] = __byte_perm(p[2 * j], p[2 * j + 1], 0x6420);
     hi[j] = __byte_perm(p[2 * j], p[2 * j + 1], 0x7531);
   }
+}
+
+// The eight codes of one 32-bit word (low nibble first) -> four packed bf16x2
+// words o[0..3] (code 2i in the low half of o[i]), looked up in the byte planes
+// with byte permutes: the low three bits of a code pick an entry in each half of
+// the table, the fourth bit picks the half.
+__device__ __forceinline__ void nf4_word(uint32_t w, const uint32_t (&lo)[4], const uint32_t (&hi)[4], uint32_t *o) {
+  const uint32_t sel32 = w & 0x77777777u;
+  const uint32_t msel32 = 0x32103210u | ((w >> 1) & 0x44444444u);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t sel = h ? (sel32 >> 16) : sel32;
+    const uint32_t msel = h ? (msel32 >> 16) : msel32;
+    const uint32_t la = __byte_perm(lo[0], lo[1], sel), lb = __byte_perm(lo[2], lo[3], sel);
+    const uint32_t ha = __byte_perm(hi[0], hi[1], sel), hb = __byte_perm(hi[2], hi[3], sel);
+    const uint32_t l = __byte_perm(la, lb, msel), hh = __byte_perm(ha, hb, msel);
+    o[h * 2 + 0] = __byte_perm(l, hh, 0x5140);
+    o[h * 2 + 1] = __byte_perm(l, hh, 0x7362);
+  }
+}
+
+// Decode 64 NF4 codes (two uint4 of packed nibbles) with block scale S into 32
+// packed bf16x2 words.
+__device__ __forceinline__ void nf4_decode64(const uint4 &c0, const uint4 &c1, float S, uint32_t (&o)[32]) {
+  uint32_t lo[4], hi[4];
+  nf4_planes(S, lo, hi);
   const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    const uint32_t sel32 = w[q] & 0x77777777u;
-    const uint32_t msel32 = 0x32103210u | ((w[q] >> 1) & 0x44444444u);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint32_t sel = h ? (sel32 >> 16) : sel32;
-      const uint32_t msel = h ? (msel32 >> 16) : msel32;
-      const uint32_t la = __byte_perm(lo[0], lo[1], sel), lb = __byte_perm(lo[2], lo[3], sel);
-      const uint32_t ha = __byte_perm(hi[0], hi[1], sel), hb = __byte_perm(hi[2], hi[3], sel);
-      const uint32_t l = __byte_perm(la, lb, msel), hh = __byte_perm(ha, hb, msel);
-      o[q * 4 + h * 2 + 0] = __byte_perm(l, hh, 0x5140);
-      o[q * 4 + h * 2 + 1] = __byte_perm(l, hh, 0x7362);
-    }
-  }
+  for (int q = 0; q < 8; ++q) nf4_word(w[q], lo, hi, o + 4 * q);
 }
 
 __device__ __forceinline__ void store_row128(uint8_t *atom_base, uint32_t row, const uint32_t (&o)[32]) {

@@ -28,6 +28,8 @@ using namespace qlora;
 constexpr int kFusedMT = QLORA_FUSED_MT;
 
 namespace {
+// Device address of the library status word on device `dev` (defined below).
+qlora_status library_status_addr(int dev, uint32_t **out);
 
 // ---------------------------------------------------------------------------
 // Tensor maps (driver entry point fetched through the runtime: no link-time
@@ -806,20 +808,34 @@ qlora_status qlora_lora_merge(const qlora_nf4_tensor *W, const qlora_lora *adapt
   if (!aligned(W_out, 16)) return QLORA_ERR_MISALIGNED;
   int dev, sms;
   if ((s = check_device(&dev, &sms)) != QLORA_OK) return s;
-  const int bytes = static_cast<int>(merge_smem_bytes(adapter->r));
+  uint32_t *status = nullptr;
+  if ((s = library_status_addr(dev, &status)) != QLORA_OK) return s;
   static std::once_flag flags[64];
   static qlora_status results[64];
-  if ((s = set_smem(nf4_lora_merge_kernel, static_cast<int>(merge_smem_bytes(QLORA_MAX_RANK)), dev, flags,
-                    results)) != QLORA_OK)
+  if ((s = set_smem(nf4_lora_merge_kernel, static_cast<int>(kMergeSmemBytes), dev, flags, results)) != QLORA_OK)
     return s;
-  const int64_t ktiles = (W->cols + kMergeTile - 1) / kMergeTile;
-  const dim3 grid(static_cast<unsigned>((ktiles + kMergePasses - 1) / kMergePasses),
-                  static_cast<unsigned>((W->rows + kMergeTile - 1) / kMergeTile));
-  const float sc = adapter->alpha / static_cast<float>(adapter->r);
-  nf4_lora_merge_kernel<<<grid, kMergeThreads, bytes, reinterpret_cast<cudaStream_t>(stream)>>>(
-      W->codes, W->scale_codes, W->c2, W->rows, W->cols, static_cast<const __nv_bfloat16 *>(adapter->A),
-      static_cast<const __nv_bfloat16 *>(adapter->B), adapter->r, sc, static_cast<__nv_bfloat16 *>(W_out),
-      W->scale_format);
+  const int64_t N = W->rows, K = W->cols;
+  const int r = adapter->r;
+  // codes [N][K/2 bytes], box 128 B x 128 rows; B [N, r], box 64 ranks x 128 rows;
+  // A [r, K], box 64 columns x 64 ranks; W_out [N, K], box 64 columns x 32 rows
+  CUtensorMap tmCodes, tmB, tmA, tmOut;
+  if (!make_tmap(&tmCodes, W->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, K / 2, 128, 128, true) ||
+      !tmap_bf16(&tmB, adapter->B, r, N, 64, 128) || !tmap_bf16(&tmA, adapter->A, K, r, 64, 64) ||
+      !tmap_bf16(&tmOut, W_out, K, N, 64, 32))
+    return QLORA_ERR_CUDA;
+  const int64_t tiles = ((N + kMergeBM - 1) / kMergeBM) * ((K + kMergeBN - 1) / kMergeBN);
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  MergeArgs ma;
+  ma.scale_codes = W->scale_codes;
+  ma.c2 = W->c2;
+  ma.N = N;
+  ma.K = K;
+  ma.r = r;
+  ma.s = adapter->alpha / static_cast<float>(r);
+  ma.fmt = W->scale_format;
+  ma.status = status;
+  nf4_lora_merge_kernel<<<grid, kMergeThreads, kMergeSmemBytes, reinterpret_cast<cudaStream_t>(stream)>>>(
+      tmCodes, tmB, tmA, tmOut, ma);
   return launch_status();
 }
 
@@ -860,6 +876,10 @@ qlora_status qlora_adamw_step(float *param, void *param_bf16, const float *grad,
 // once per device with cudaGetSymbolAddress.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[QLORA_NOALLOC_SCRATCH_BYTES];
 
+// Status word of the calls that take no workspace (qlora_lora_merge): one static
+// device word per GPU, looked up like the scratch array.
+static __device__ uint32_t g_library_status;
+
 namespace {
 // Only a successful lookup is cached: a lookup that fails (for example one made
 // during a stream capture) is retried by the next call on that device.
@@ -874,6 +894,21 @@ qlora_status noalloc_scratch(int dev, void **out) {
       return QLORA_ERR_CUDA;
     }
     addr[dev] = p;
+  }
+  *out = addr[dev];
+  return QLORA_OK;
+}
+qlora_status library_status_addr(int dev, uint32_t **out) {
+  static std::mutex mu;
+  static uint32_t *addr[64];
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_library_status) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return QLORA_ERR_CUDA;
+    }
+    addr[dev] = static_cast<uint32_t *>(p);
   }
   *out = addr[dev];
   return QLORA_OK;
@@ -925,6 +960,22 @@ qlora_status qlora_read_status(const void *ws, qlora_stream_t stream) {
   if (cudaStreamSynchronize(st) != cudaSuccess) return QLORA_ERR_CUDA;
   uint32_t word = 0;
   if (cudaMemcpy(&word, ws, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return QLORA_ERR_CUDA;
+  for (int code = 1; code < 32; ++code)
+    if (word & (1u << code)) return static_cast<qlora_status>(code);
+  return QLORA_OK;
+}
+
+qlora_status qlora_read_library_status(qlora_stream_t stream) {
+  int dev;
+  qlora_status s;
+  if ((s = check_device(&dev, nullptr)) != QLORA_OK) return s;
+  uint32_t *word_d = nullptr;
+  if ((s = library_status_addr(dev, &word_d)) != QLORA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return QLORA_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpy(&word, word_d, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (word && cudaMemset(word_d, 0, sizeof(word)) != cudaSuccess) return QLORA_ERR_CUDA;
   for (int code = 1; code < 32; ++code)
     if (word & (1u << code)) return static_cast<qlora_status>(code);
   return QLORA_OK;

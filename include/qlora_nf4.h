@@ -252,9 +252,12 @@ QLORA_API qlora_status qlora_linear_fwd_multi(const qlora_nf4_tensor *W, const q
  * (IBM): the low-rank update merges into the frozen weights for deployment):
  *   W_out [N, K] bf16 = bf16_rne(W' + s B A),  s = alpha / r,
  * with W' the dequantised NF4 weight, s B A from the bf16 adapter on tensor
- * cores with float32 accumulation, the sum in float32, rounded to bf16 once.
- * W_out: device, 16-byte aligned, caller-owned, overwritten.  Errors as for
- * qlora_linear_fwd (invalid tensor or adapter, misalignment, no device). */
+ * cores (tcgen05) with float32 accumulation, the sum in float32, rounded to
+ * bf16 once.  W_out: device, 16-byte aligned, caller-owned, overwritten.  Errors
+ * as for qlora_linear_fwd (invalid tensor or adapter, misalignment, no device).
+ * Takes no workspace: a device-side error (a bounded wait that gave up) is
+ * recorded in the library status word of the device, read by
+ * qlora_read_library_status. */
 QLORA_API qlora_status qlora_lora_merge(const qlora_nf4_tensor *W, const qlora_lora *adapter, void *W_out,
                                         qlora_stream_t stream);
 
@@ -302,6 +305,11 @@ QLORA_API qlora_status qlora_selftest_bounded_wait(void *ws, uint32_t limit_us, 
 /* Synchronise `stream`, read the status word at the start of ws and return the
  * first error it records (QLORA_OK if none).  The word is left unchanged. */
 QLORA_API qlora_status qlora_read_status(const void *ws, qlora_stream_t stream);
+
+/* Synchronise `stream`, read the status word that the library holds on the
+ * current device for the calls that take no workspace (qlora_lora_merge), clear
+ * it and return the first error it recorded (QLORA_OK if none). */
+QLORA_API qlora_status qlora_read_library_status(qlora_stream_t stream);
 
 /* Static, human-readable name of a status code. */
 QLORA_API const char *qlora_status_string(qlora_status status);

@@ -22,7 +22,7 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("n,k,r", [(256, 256, 8), (1000, 320, 16), (328, 576, 128), (520, 1088, 72),
-                                   (4096, 4096, 64)])
+                                   (4096, 4096, 64), (1, 512, 8), (136, 64, 256), (300, 1344, 200)])
 def test_merge_matches_oracle(n, k, r):
     w, _, a, b, _ = I.custom(n, k, 1, r, 40 * n + k + r)
     q = O.quantize(w.float().numpy(), n, k)
@@ -39,6 +39,7 @@ def test_merge_matches_oracle(n, k, r):
     bound = ulp + r * 2.0 ** -24 * terms
     assert np.all(err <= bound), f"{n}x{k} r={r}: max {np.max(err / bound):.2f} of the bound"
     assert np.mean(gv == rv) > 0.999
+    assert bd.read_library_status() == 0
 
 
 def test_merge_with_b_zero_is_the_dequantised_weight():
