@@ -110,12 +110,27 @@ __global__ void __launch_bounds__(kMergeThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   const int64_t N = a.N, K = a.K;
-  const int64_t ncol = (K + kMergeBN - 1) / kMergeBN;
-  const int64_t tiles = ((N + kMergeBM - 1) / kMergeBM) * ncol;
+  // tile t = row block rb * ncol + column block cb (fewer than 2^31 tiles); a
+  // CTA's tiles t, t + G, ... are walked by steps of (G / ncol, G % ncol)
+  const int ncol = static_cast<int>((K + kMergeBN - 1) / kMergeBN);
+  const int tiles = static_cast<int>((N + kMergeBM - 1) / kMergeBM) * ncol;
+  const int G = gridDim.x, step_r = G / ncol, step_c = G - step_r * ncol;
   const int rsteps = (a.r + 63) / 64;
-  auto tile_of = [&](int64_t t, int64_t &n0, int64_t &k0) {
-    n0 = (t / ncol) * kMergeBM;
-    k0 = (t % ncol) * kMergeBN;
+  struct TilePos {
+    int t, rb, cb;
+  };
+  auto first_tile = [&]() {
+    const int t = blockIdx.x, rb = t / ncol;
+    return TilePos{t, rb, t - rb * ncol};
+  };
+  auto next_tile = [&](TilePos &p) {
+    p.t += G;
+    p.rb += step_r;
+    p.cb += step_c;
+    if (p.cb >= ncol) {
+      p.cb -= ncol;
+      ++p.rb;
+    }
   };
   auto fail = [&]() {
     raise_status(a.status, QLORA_ERR_TIMEOUT);
@@ -128,9 +143,8 @@ __global__ void __launch_bounds__(kMergeThreads, 1)
       uint32_t sab = 0, pab = 0;
       int issued_ab = 0;
       bool ok = true;
-      for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-        int64_t n0, k0;
-        tile_of(t, n0, k0);
+      for (TilePos p = first_tile(); p.t < tiles && ok; next_tile(p)) {
+        const int64_t n0 = static_cast<int64_t>(p.rb) * kMergeBM, k0 = static_cast<int64_t>(p.cb) * kMergeBN;
         for (int j = 0; j < rsteps; ++j) {
           if (!ptx::mbar_wait(&empty_ab[sab], pab ^ 1, abort_flag)) { ok = false; break; }
           ptx::mbar_arrive_expect_tx(&full_ab[sab], kMergeABStage);
@@ -156,9 +170,8 @@ __global__ void __launch_bounds__(kMergeThreads, 1)
       uint32_t sc = 0, pc = 0;
       int issued_c = 0;
       bool ok = true;
-      for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
-        int64_t n0, k0;
-        tile_of(t, n0, k0);
+      for (TilePos p = first_tile(); p.t < tiles; next_tile(p)) {
+        const int64_t n0 = static_cast<int64_t>(p.rb) * kMergeBM, k0 = static_cast<int64_t>(p.cb) * kMergeBN;
         if (!ptx::mbar_wait(&empty_c[sc], pc ^ 1, abort_flag)) { ok = false; break; }
         ptx::mbar_arrive_expect_tx(&full_c[sc], kMergeCStage);
         ptx::tma_load_2d(sC + sc * kMergeCStage, &tmCodes, &full_c[sc], static_cast<int32_t>(k0 / 2),
@@ -179,7 +192,7 @@ __global__ void __launch_bounds__(kMergeThreads, 1)
       int it = 0;
       bool ok = true;
       const uint32_t sAB0 = ptx::smem_addr(sAB);
-      for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++it) {
+      for (int t = blockIdx.x; t < tiles && ok; t += G, ++it) {
         const int acc = it & 1;
         if (!ptx::mbar_wait(&acc_empty[acc], ((it >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
         ptx::tc_fence_after();
@@ -210,13 +223,11 @@ __global__ void __launch_bounds__(kMergeThreads, 1)
     // scale code and second-level constant of this thread's row in its 64-column
     // block of tile t: loaded one tile ahead (the raw values, so that nothing
     // waits for the loads until the tile that uses them)
-    auto scale_src = [&](int64_t t, uint32_t &qv, float &cv) {
+    auto scale_src = [&](const TilePos &p, uint32_t &qv, float &cv) {
       qv = 0u;
       cv = 0.0f;
-      if (t >= tiles) return;
-      int64_t n0, k0;
-      tile_of(t, n0, k0);
-      const int64_t n = n0 + row_t, kb = k0 / 64 + cq;
+      if (p.t >= tiles) return;
+      const int64_t n = static_cast<int64_t>(p.rb) * kMergeBM + row_t, kb = static_cast<int64_t>(p.cb) * 4 + cq;
       if (n < N && kb < nbk) {
         const int64_t b = n * nbk + kb;
         qv = __ldg(a.scale_codes + b);
@@ -225,14 +236,15 @@ __global__ void __launch_bounds__(kMergeThreads, 1)
     };
     uint32_t qv;
     float cv;
-    scale_src(blockIdx.x, qv, cv);
+    TilePos ahead = first_tile();  // the tile whose scale is loaded next
+    scale_src(ahead, qv, cv);
     uint32_t sc = 0, pc = 0;
     int it = 0;
-    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
-      int64_t n0, k0;
-      tile_of(t, n0, k0);
+    for (TilePos p = first_tile(); p.t < tiles; next_tile(p), ++it) {
+      const int64_t n0 = static_cast<int64_t>(p.rb) * kMergeBM, k0 = static_cast<int64_t>(p.cb) * kMergeBN;
       const float S = __fmul_rn(scale_code_value(qv, a.fmt), cv);  // S' = fl32(code value * c2)
-      scale_src(t + gridDim.x, qv, cv);
+      next_tile(ahead);
+      scale_src(ahead, qv, cv);
       const int acc = it & 1;
       const bool ready = ptx::mbar_wait(&full_c[sc], pc, abort_flag) &&
                          ptx::mbar_wait(&acc_full[acc], (it >> 1) & 1, abort_flag);

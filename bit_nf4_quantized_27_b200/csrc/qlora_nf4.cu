@@ -824,6 +824,7 @@ qlora_status qlora_lora_merge(const qlora_nf4_tensor *W, const qlora_lora *adapt
       !tmap_bf16(&tmOut, W_out, K, N, 64, 32))
     return QLORA_ERR_CUDA;
   const int64_t tiles = ((N + kMergeBM - 1) / kMergeBM) * ((K + kMergeBN - 1) / kMergeBN);
+  if (tiles >= (int64_t(1) << 31)) return QLORA_ERR_UNSUPPORTED_SHAPE;
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
   MergeArgs ma;
   ma.scale_codes = W->scale_codes;
