@@ -538,6 +538,11 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   __syncthreads();
   if (tid == 0)
     for (int u = 0; u < S && u < total; ++u) issue(u);
+  // per-token adapters: each token's B rows of this CTA's row groups (contiguous,
+  // my_rg * 16 rows of r ranks) start moving into L2 now, behind the weight stream,
+  // so that the LoRA step after the main loop reads them from L2
+  if (a.multi && warp == 1 && lane < a.M && my_rg > 0)
+    ptx::bulk_prefetch_l2(a.ml.B[lane] + (int64_t)rg0 * 16 * a.r, static_cast<uint32_t>(my_rg * 16 * a.r * 2));
 
   // this warp's slice of X for a chunk (raw bf16)
   uint4 xraw[NG][4][2];
@@ -745,53 +750,105 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   __syncthreads();
   const __nv_bfloat16 *const sT = a.sT + griddep_wait_token();
   if (a.multi) {
-    // one adapter per token: tasks (row group, token) spread over all warps, two
-    // tasks in flight per warp with every load of a round issued before its
-    // products.  Lane
-    // = row (lane & 15) of the row group, half of the rank range per half-warp,
-    // combined by a shuffle (fixed order); each task adds its own token's column.
-    const int half = lane >> 4, hr = a.r / 2;  // r % 8 == 0: hr is a multiple of 4
-    const int ntask = my_rg * a.M;
-    for (int k0 = warp; k0 < ntask; k0 += 2 * kGemvWarps) {
-      float acc[2] = {0.0f, 0.0f};
-      // 16 ranks per round: four 8-byte loads of B and of s T per task (the half
-      // rank range starts 8-byte aligned: r % 8 == 0)
-      for (int j = 0; j < hr; j += 16) {
-        uint2 bv[2][4], sv[2][4];
+    // one adapter per token.  s T (all tokens) is copied to shared memory (the
+    // pair table's space, unused after the main loop).  Each token's B rows of
+    // this CTA's row groups are one contiguous block of 16-byte pieces (P = r / 8
+    // per row).
+    uint4 *sts = reinterpret_cast<uint4 *>(at(lut_addr));
+    const int P = a.r / 8;  // r % 8 == 0
+    const int n16 = a.M * P;
+    for (int i = tid; i < n16; i += kGemvThreads) sts[i] = __ldcg(reinterpret_cast<const uint4 *>(sT) + i);
+    __syncthreads();
+    if ((P & (P - 1)) == 0) {
+      // P a power of two (r = 8, 16, 32, 64, 128, 256): every warp reads 32
+      // consecutive pieces per load (coalesced), eight loads in flight per lane;
+      // the P lanes of a row (an aligned group, never split across rows or
+      // tokens) combine their partial dots by a butterfly in fixed order, and the
+      // first adds the row's sum to its token's column.
+      constexpr int U = 8;
+      const int lgP = __ffs(P) - 1;
+      const int per_t = (my_rg * 16) << lgP;  // pieces per token (at most 5 * 16 * 32)
+      const int total = a.M * per_t;           // below 2^16
+      // piece / per_t as a multiply-high: exact while piece * per_t < 2^32
+      const uint32_t inv_t = 0xffffffffu / static_cast<uint32_t>(max(per_t, 1)) + 1u;
+      for (int b0 = warp * 32 + lane; b0 - lane < total; b0 += kGemvThreads * U) {  // warp-uniform test
+        uint4 bv[U];
+        int tk[U], pr[U];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int k = k0 + u * kGemvWarps;
-          const bool live = k < ntask;
-          const int i = live ? k / a.M : 0, t = live ? k - i * a.M : 0;
-          const int64_t n = (int64_t)(rg0 + i) * 16 + (lane & 15);
-          const __nv_bfloat16 *bt = a.ml.B[t] + n * a.r + half * hr + j;
-          const __nv_bfloat16 *st = sT + (int64_t)t * a.r + half * hr + j;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const bool in = live && j + 4 * c < hr;
-            bv[u][c] = in ? __ldg(reinterpret_cast<const uint2 *>(bt + 4 * c)) : make_uint2(0, 0);
-            sv[u][c] = in ? __ldca(reinterpret_cast<const uint2 *>(st + 4 * c)) : make_uint2(0, 0);
-          }
+        for (int u = 0; u < U; ++u) {
+          const int pp = b0 + u * kGemvThreads;
+          const int pc = pp < total ? pp : total - 1;  // past the end: the last piece again, not summed
+          const int t = static_cast<int>(__umulhi(static_cast<uint32_t>(pc), inv_t));
+          tk[u] = t;
+          pr[u] = pc - t * per_t;
+          bv[u] = __ldg(reinterpret_cast<const uint4 *>(a.ml.B[t] + (int64_t)rg0 * 16 * a.r) + pr[u]);
         }
 #pragma unroll
-        for (int u = 0; u < 2; ++u)
+        for (int u = 0; u < U; ++u) {
+          const int ch = pr[u] & (P - 1);
+          const uint4 sv = sts[tk[u] * P + ch];
+          const uint32_t bw[4] = {bv[u].x, bv[u].y, bv[u].z, bv[u].w};
+          const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
+          float v = 0.0f;
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            acc[u] = fmaf(bf16lo_to_f32(bv[u][c].x), bf16lo_to_f32(sv[u][c].x), acc[u]);
-            acc[u] = fmaf(bf16hi_to_f32(bv[u][c].x), bf16hi_to_f32(sv[u][c].x), acc[u]);
-            acc[u] = fmaf(bf16lo_to_f32(bv[u][c].y), bf16lo_to_f32(sv[u][c].y), acc[u]);
-            acc[u] = fmaf(bf16hi_to_f32(bv[u][c].y), bf16hi_to_f32(sv[u][c].y), acc[u]);
+          for (int e = 0; e < 4; ++e) {
+            v = fmaf(bf16lo_to_f32(bw[e]), bf16lo_to_f32(sw[e]), v);
+            v = fmaf(bf16hi_to_f32(bw[e]), bf16hi_to_f32(sw[e]), v);
           }
+          for (int o = 1; o < P; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          const int rrow = pr[u] >> lgP;
+          if (ch == 0 && b0 + u * kGemvThreads < total)
+            red_at(rrow >> 4)[(rrow & 15) * TR + tk[u]] += v;  // warp 0's slot of the row group
+        }
       }
+    } else {
+    const int row = lane & 15, nh = 2 * kGemvWarps;
+    const int ntask = my_rg * a.M;
+    for (int k0 = 2 * warp + (lane >> 4); k0 < ntask; k0 += 2 * nh) {
+      int ti[2], tt[2];
+      bool live[2];
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        const int k = k0 + u * kGemvWarps;
-        const float v = acc[u] + __shfl_xor_sync(0xffffffffu, acc[u], 16);
-        if (k < ntask && half == 0) {
-          const int i = k / a.M, t = k - i * a.M;
-          red_at(i)[(lane & 15) * TR + t] += v;  // warp 0's slot of row group i
+        const int k = k0 + u * nh;
+        live[u] = k < ntask;
+        ti[u] = live[u] ? k / a.M : 0;  // a task past the end reads row group 0 of token 0, unused
+        tt[u] = live[u] ? k - ti[u] * a.M : 0;
+      }
+      float acc[2] = {0.0f, 0.0f};
+      for (int j0 = 0; j0 < a.r; j0 += 64) {
+        // 64 ranks per round: eight 16-byte loads per task, all issued before the
+        // products; loads past rank r re-read the round's last piece (in bounds)
+        // and are not summed
+        const int cl = min(8, (a.r - j0) / 8) - 1;
+        uint4 bv[2][8];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int64_t n = (int64_t)(rg0 + ti[u]) * 16 + row;
+          const uint4 *src = reinterpret_cast<const uint4 *>(a.ml.B[tt[u]] + n * a.r + j0);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) bv[u][c] = __ldg(src + min(c, cl));
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const uint4 *st = sts + (tt[u] * a.r + j0) / 8;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            if (c > cl) break;
+            const uint4 sv = st[c];
+            const uint32_t bw[4] = {bv[u][c].x, bv[u][c].y, bv[u][c].z, bv[u][c].w};
+            const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              acc[u] = fmaf(bf16lo_to_f32(bw[e]), bf16lo_to_f32(sw[e]), acc[u]);
+              acc[u] = fmaf(bf16hi_to_f32(bw[e]), bf16hi_to_f32(sw[e]), acc[u]);
+            }
+          }
         }
       }
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+        if (live[u]) red_at(ti[u])[row * TR + tt[u]] += acc[u];  // warp 0's slot of row group ti
+    }
     }
   }
   if (lora_rg >= 0 && !a.multi) {
@@ -953,55 +1010,59 @@ __global__ void __launch_bounds__(kLoraDownThreads, 1) lora_down_small_kernel(
   }
 }
 
-// s_t T_t = s_t (x_t A_t^T) for decode tokens that each use their own adapter:
-// CTA (16-rank tile, token t), 256 threads splitting K in 8-element slices with
-// all 16 ranks' loads of a slice in flight; warp-shuffle then cross-warp sums
-// in a fixed order.  Writes s*T (bf16).
-constexpr int kLoraDownMultiThreads = 256;
-__global__ void __launch_bounds__(kLoraDownMultiThreads) lora_down_multi_kernel(
-    const __nv_bfloat16 *__restrict__ X, const MultiLora ml, int64_t K, int r, __nv_bfloat16 *__restrict__ sT) {
+// s T for per-token adapters (multi-adapter decode): row k = t * r + j of s T
+// is s_t * (X_t . A_t[j]) with token t's own adapter.  One warp per row: all of
+// a round's sixteen 16-byte loads of A's row are issued before its products (X
+// is read through L1, shared by the warps on the same token), then a butterfly
+// sum.  The launcher sizes the grid to the SMs the decode GEMV that follows
+// leaves free, so that this kernel runs beside it (programmatic dependent
+// launch) instead of delaying its CTAs.
+constexpr int kLoraDownMultiThreads = 512;
+__global__ void __launch_bounds__(kLoraDownMultiThreads, 1) lora_down_multi_kernel(
+    const __nv_bfloat16 *__restrict__ X, const MultiLora ml, int M, int64_t K, int r, __nv_bfloat16 *__restrict__ sT) {
   griddep_launch_dependents();
-  __shared__ float red[kLoraDownMultiThreads / 32][16];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int t = blockIdx.y, j0 = blockIdx.x * 16;
-  const __nv_bfloat16 *A = ml.A[t];
-  const __nv_bfloat16 *x = X + (int64_t)t * K;
-  float acc[16];
+  constexpr int kWarps = kLoraDownMultiThreads / 32, U = 16;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int rows = M * r;
+  const int64_t n16 = K / 8;  // 16-byte pieces per row (a multiple of 32)
+  for (int k = blockIdx.x * kWarps + warp; k < rows; k += gridDim.x * kWarps) {
+    const int t = k / r, j = k - t * r;
+    const uint4 *arow = reinterpret_cast<const uint4 *>(ml.A[t] + (int64_t)j * K);
+    const uint4 *xrow = reinterpret_cast<const uint4 *>(X + (int64_t)t * K);
+    float acc = 0.0f;
+    for (int64_t c0 = lane; c0 < n16; c0 += 32 * U) {
+      uint4 av[U];
 #pragma unroll
-  for (int jj = 0; jj < 16; ++jj) acc[jj] = 0.0f;
-  for (int64_t k = (int64_t)tid * 8; k < K; k += kLoraDownMultiThreads * 8) {
-    const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(x + k));
-    const float xf[8] = {bf16lo_to_f32(xv.x), bf16hi_to_f32(xv.x), bf16lo_to_f32(xv.y), bf16hi_to_f32(xv.y),
-                         bf16lo_to_f32(xv.z), bf16hi_to_f32(xv.z), bf16lo_to_f32(xv.w), bf16hi_to_f32(xv.w)};
-    uint4 av[16];
+      for (int u = 0; u < U; ++u) {
+        const int64_t c = c0 + 32 * u;
+        av[u] = c < n16 ? __ldg(arow + c) : make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll
-    for (int jj = 0; jj < 16; ++jj)
-      av[jj] = (j0 + jj < r) ? __ldg(reinterpret_cast<const uint4 *>(A + (int64_t)(j0 + jj) * K + k))
-                             : make_uint4(0, 0, 0, 0);
+      for (int u = 0; u < U; ++u) {
+        const int64_t c = c0 + 32 * u;
+        const uint4 xv = c < n16 ? __ldg(xrow + c) : make_uint4(0, 0, 0, 0);
+        const uint32_t aw[4] = {av[u].x, av[u].y, av[u].z, av[u].w};
+        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
-    for (int jj = 0; jj < 16; ++jj) {
-      const uint32_t w[4] = {av[jj].x, av[jj].y, av[jj].z, av[jj].w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        acc[jj] = fmaf(bf16lo_to_f32(w[e]), xf[2 * e], acc[jj]);
-        acc[jj] = fmaf(bf16hi_to_f32(w[e]), xf[2 * e + 1], acc[jj]);
+        for (int e = 0; e < 4; ++e) {
+          acc = fmaf(bf16lo_to_f32(aw[e]), bf16lo_to_f32(xw[e]), acc);
+          acc = fmaf(bf16hi_to_f32(aw[e]), bf16hi_to_f32(xw[e]), acc);
+        }
       }
     }
-  }
 #pragma unroll
-  for (int jj = 0; jj < 16; ++jj) {
-    float v = acc[jj];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0) red[warp][jj] = v;
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) sT[k] = __float2bfloat16_rn(acc * ml.s[t]);
   }
-  __syncthreads();
-  if (tid < 16 && j0 + tid < r) {
-    float v = 0.0f;
-#pragma unroll
-    for (int w = 0; w < kLoraDownMultiThreads / 32; ++w) v += red[w][tid];
-    sT[(int64_t)t * r + j0 + tid] = __float2bfloat16_rn(v * ml.s[t]);
-  }
+}
+
+// CTAs of the decode GEMV for N rows on `sms` SMs (as launch_gemv sizes it).
+inline int gemv_grid_ctas(int64_t N, int sms, bool bulk) {
+  const int num_rg = static_cast<int>((N + 15) / 16);
+  const int cap = bulk ? kBulkMaxRG : kGemvMaxRG;
+  int per = (num_rg + sms - 1) / sms;
+  if (per > cap) per = cap;
+  return (num_rg + per - 1) / per;
 }
 
 // Start of the dynamic shared-memory window of a kernel without static shared

@@ -781,8 +781,13 @@ qlora_status qlora_linear_fwd_multi(const qlora_nf4_tensor *W, const qlora_lora 
   }
   uint8_t *wsb = static_cast<uint8_t *>(ws);
   __nv_bfloat16 *sT = reinterpret_cast<__nv_bfloat16 *>(wsb + QLORA_STATUS_BYTES);
-  lora_down_multi_kernel<<<dim3((r + 15) / 16, static_cast<unsigned>(M)), kLoraDownMultiThreads, 0, st>>>(
-      static_cast<const __nv_bfloat16 *>(X), g.ml, K, r, sT);
+  // s T on the SMs the GEMV leaves free (at least eight CTAs, at most one warp per row)
+  const int rows = static_cast<int>(M) * r, warps = kLoraDownMultiThreads / 32;
+  int down = sms - gemv_grid_ctas(N, sms, true);
+  if (down < 8) down = 8;
+  if (down > (rows + warps - 1) / warps) down = (rows + warps - 1) / warps;
+  lora_down_multi_kernel<<<down, kLoraDownMultiThreads, 0, st>>>(static_cast<const __nv_bfloat16 *>(X), g.ml,
+                                                                   static_cast<int>(M), K, r, sT);
   if ((s = launch_status()) != QLORA_OK) return s;
   g.codes = W->codes; g.scale_codes = W->scale_codes; g.c2 = W->c2; g.scale_format = W->scale_format;
   g.N = N; g.K = K; g.M = (int)M;

@@ -158,6 +158,12 @@ __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.
 // Every bulk group of this thread has completed.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// Non-blocking prefetch of `bytes` (a multiple of 16, 16-byte aligned) of global
+// memory into L2.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // L2 policy for data that is read once (weights streamed by a decode step):
 // its lines are the first to be evicted, so they do not push out the small
 // operands, code and constants that the next call reads again.

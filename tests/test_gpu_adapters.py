@@ -90,7 +90,8 @@ def _check(name, got, ref):
 
 
 @pytest.mark.parametrize("n,k,m,r,count", [(11008, 4096, 1, 64, 2), (11008, 4096, 5, 64, 3), (11008, 4096, 16, 64, 16),
-                                           (1024, 1024, 9, 16, 4), (2048, 8192, 4, 128, 2), (512, 256, 3, 8, 3)])
+                                           (1024, 1024, 9, 16, 4), (2048, 8192, 4, 128, 2), (512, 256, 3, 8, 3),
+                                           (1024, 1024, 6, 24, 3), (512, 512, 16, 72, 5), (768, 2048, 7, 256, 2)])
 def test_multi_adapter_gemv_matches_oracle(n, k, m, r, count):
     w, x, _, _, _ = I.custom(n, k, m, r, 9000 + n + m)
     ads = _adapters(n, k, r, count, 9100 + k)
