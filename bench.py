@@ -48,10 +48,10 @@ def load_peaks():
 # captures of the `cases` module's fwd_8192 / fwd_65b_up / fwd_65b_down.  The
 # figure belongs to the kernel sources it was measured on: it is reported only
 # while their digest still matches, else the traffic is null.
-FUSED_FWD_TRAFFIC_BYTES = 586.63e6
+FUSED_FWD_TRAFFIC_BYTES = 592.60e6
 FUSED_FWD_TRAFFIC_SOURCES = ("gemm_pair_kernel.cuh", "gemm_kernel.cuh", "sm100_ptx.cuh", "nf4_device.cuh",
                              "qlora_nf4.cu")
-FUSED_FWD_TRAFFIC_DIGEST = "5680b2cc4129d462"
+FUSED_FWD_TRAFFIC_DIGEST = "547b26564f428911"
 
 
 def fused_fwd_traffic():
