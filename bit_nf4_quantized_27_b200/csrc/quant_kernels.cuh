@@ -122,6 +122,14 @@ nf4_quantize_kernel(const TIn *__restrict__ W, int64_t nblocks, uint8_t *__restr
   // cell k's entry from the bits of fl32(x * 32 + 32 + 1.5 * 2^23): (bits - 0x4B400000) * 256 + tab_lane,
   // one multiply-add in 32-bit arithmetic (|x'| <= 1 + 2 ulp keeps the cell in 0..64)
   const uint32_t tab_off = tab_lane - 0x4B400000u * 256u;
+  uint32_t pmul[8];  // 16^i in registers the compiler cannot see through: the packing runs as multiply-adds
+  {
+    uint32_t m16;
+    asm("mov.u32 %0, 16;" : "=r"(m16));
+    pmul[0] = 1u;
+#pragma unroll
+    for (int i = 1; i < 8; ++i) pmul[i] = pmul[i - 1] * m16;
+  }
   const int64_t g = blockIdx.x;
   const int64_t blk0 = g * kGroup;
   const int nblk = static_cast<int>(nblocks - blk0 < kGroup ? nblocks - blk0 : kGroup);
@@ -174,19 +182,25 @@ nf4_quantize_kernel(const TIn *__restrict__ W, int64_t nblocks, uint8_t *__restr
       bool slow = !(rS < 3.0e38f);  // subnormal S (flushed): every code takes the exact path
       if (slow) rS = 0.0f;          // (and the fast path's cells stay in range)
       uint32_t c[EPL];
+      uint32_t dmin = 0xffffffffu;  // smallest (bit distance of x' from its cell's switch point) + 8
 #pragma unroll
       for (int i = 0; i < EPL; ++i) {
         const float xa = __fmul_rn(w[i], rS);
         const float2 e = lds_f2(__float_as_uint(__fmaf_rn(xa, 32.0f, 12582912.0f + 32.0f)) * 256u + tab_off);
         c[i] = __float_as_uint(e.y) + (xa > e.x ? 1u : 0u);
-        slow |= (__float_as_uint(xa) - __float_as_uint(e.x) + 8u) <= 16u;
+        dmin = min(dmin, __float_as_uint(xa) - __float_as_uint(e.x) + 8u);
       }
+      slow |= dmin <= 16u;
       if (slow) {
 #pragma unroll
         for (int i = 0; i < EPL; ++i) c[i] = code_from_table(__fdiv_rn(w[i], S), tab_lane);
       }
+      uint32_t plo = 0, phi = 0;
 #pragma unroll
-      for (int i = 0; i < EPL; ++i) packed |= static_cast<uint64_t>(c[i]) << (4 * i);
+      for (int i = 0; i < EPL && i < 8; ++i) plo = c[i] * pmul[i] + plo;
+#pragma unroll
+      for (int i = 8; i < EPL; ++i) phi = c[i] * pmul[i - 8] + phi;
+      packed = static_cast<uint64_t>(plo) | (static_cast<uint64_t>(phi) << 32);
     }
     const int64_t e0 = (blk0 + lb) * kBlock + (tid % LPB) * EPL;
     if constexpr (EPL == 16) {
