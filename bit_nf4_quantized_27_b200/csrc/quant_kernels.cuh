@@ -66,11 +66,13 @@ template <>
 struct QuantTraits<__nv_bfloat16> {
   static constexpr int kVecs = 2;           // two 16-byte vectors per lane and block
   static constexpr int kElemsPerLane = 16;
+  static constexpr int kMinCtas = 4;        // resident CTAs per SM the register budget is cut for
 };
 template <>
 struct QuantTraits<float> {
   static constexpr int kVecs = 1;
   static constexpr int kElemsPerLane = 4;
+  static constexpr int kMinCtas = 1;        // sixteen 16-byte loads in flight per thread need the registers
 };
 
 // Unpacks the 16-byte vector of this lane to float32 values.
@@ -100,7 +102,7 @@ constexpr int kQuantThreads = 256;
 
 // grid.x = number of groups; one CTA per group of 256 blocks.
 template <typename TIn>
-__global__ void __launch_bounds__(kQuantThreads)
+__global__ void __launch_bounds__(kQuantThreads, QuantTraits<TIn>::kMinCtas)
 nf4_quantize_kernel(const TIn *__restrict__ W, int64_t nblocks, uint8_t *__restrict__ codes,
                     uint8_t *__restrict__ scale_codes, float *__restrict__ c2_out,
                     uint32_t *__restrict__ status, const CodeCellTable table, int fmt) {
@@ -165,14 +167,17 @@ nf4_quantize_kernel(const TIn *__restrict__ W, int64_t nblocks, uint8_t *__restr
     if (!finite && (tid % LPB) == 0) raise_status(status, QLORA_ERR_NONFINITE);
     if ((tid % LPB) == 0) s_absmax[lb] = finite ? S : 0.0f;
 
-    float w[EPL];
-#pragma unroll
-    for (int h = 0; h < VPL; ++h) {
-      float wv[EPV];
-      unpack_vec(v[it][h], wv);
-#pragma unroll
-      for (int i = 0; i < EPV; ++i) w[h * EPV + i] = wv[i];
-    }
+    // element i of this lane's vectors, as float32 (unpacked where it is used)
+    auto elem = [&](int i) -> float {
+      const uint4 &q = v[it][i / EPV];
+      const int j = i % EPV;
+      if constexpr (EPV == 8) {
+        const uint32_t wd = (j >> 1) == 0 ? q.x : (j >> 1) == 1 ? q.y : (j >> 1) == 2 ? q.z : q.w;
+        return (j & 1) ? bf16hi_to_f32(wd) : bf16lo_to_f32(wd);
+      } else {
+        return __uint_as_float(j == 0 ? q.x : j == 1 ? q.y : j == 2 ? q.z : q.w);
+      }
+    };
     uint64_t packed = 0;
     if (S == 0.0f || !finite) {
       packed = 0x7777777777777777ull & (EPL >= 16 ? ~0ull : ((1ull << (4 * EPL)) - 1));  // exact-zero level
@@ -181,25 +186,25 @@ nf4_quantize_kernel(const TIn *__restrict__ W, int64_t nblocks, uint8_t *__restr
       asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rS) : "f"(S));
       bool slow = !(rS < 3.0e38f);  // subnormal S (flushed): every code takes the exact path
       if (slow) rS = 0.0f;          // (and the fast path's cells stay in range)
-      uint32_t c[EPL];
+      uint32_t plo = 0, phi = 0;
       uint32_t dmin = 0xffffffffu;  // smallest (bit distance of x' from its cell's switch point) + 8
 #pragma unroll
       for (int i = 0; i < EPL; ++i) {
-        const float xa = __fmul_rn(w[i], rS);
+        const float xa = __fmul_rn(elem(i), rS);
         const float2 e = lds_f2(__float_as_uint(__fmaf_rn(xa, 32.0f, 12582912.0f + 32.0f)) * 256u + tab_off);
-        c[i] = __float_as_uint(e.y) + (xa > e.x ? 1u : 0u);
+        const uint32_t c = __float_as_uint(e.y) + (xa > e.x ? 1u : 0u);
         dmin = min(dmin, __float_as_uint(xa) - __float_as_uint(e.x) + 8u);
+        if (i < 8) plo = c * pmul[i & 7] + plo; else phi = c * pmul[i & 7] + phi;
       }
       slow |= dmin <= 16u;
       if (slow) {
+        plo = phi = 0;
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) c[i] = code_from_table(__fdiv_rn(w[i], S), tab_lane);
+        for (int i = 0; i < EPL; ++i) {
+          const uint32_t c = code_from_table(__fdiv_rn(elem(i), S), tab_lane);
+          if (i < 8) plo = c * pmul[i & 7] + plo; else phi = c * pmul[i & 7] + phi;
+        }
       }
-      uint32_t plo = 0, phi = 0;
-#pragma unroll
-      for (int i = 0; i < EPL && i < 8; ++i) plo = c[i] * pmul[i] + plo;
-#pragma unroll
-      for (int i = 8; i < EPL; ++i) phi = c[i] * pmul[i - 8] + phi;
       packed = static_cast<uint64_t>(plo) | (static_cast<uint64_t>(phi) << 32);
     }
     const int64_t e0 = (blk0 + lb) * kBlock + (tid % LPB) * EPL;
