@@ -373,7 +373,7 @@ def sub_gemv(device, peaks):
             (torch.randn(n, r, generator=g, device=device) * 0.01).to(torch.bfloat16), wl.alpha) for _ in range(m)]
     x = torch.randn(m, k, generator=g, device=device).to(torch.bfloat16)
     y = torch.empty(m, n, dtype=torch.bfloat16, device=device)
-    ws = bd.new_workspace(bd.workspace_bytes(m, n, k, r, False), device)
+    ws = bd.new_workspace(bd.workspace_bytes_multi(m, n, k, r), device)
     reps = 4 * copies
     idx = list(range(m))
 

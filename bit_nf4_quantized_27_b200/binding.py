@@ -70,6 +70,7 @@ def lib():
         "qlora_nf4_codebook": (None, [ctypes.POINTER(ctypes.c_float)]),
         "qlora_nf4_storage_bytes": (sz, [i64, i64, ctypes.POINTER(sz), ctypes.POINTER(sz), ctypes.POINTER(sz)]),
         "qlora_workspace_bytes": (sz, [i64, i64, i64, i32, ctypes.c_int]),
+        "qlora_workspace_bytes_multi": (sz, [i64, i64, i64, i32]),
         "qlora_nf4_quantize": (ctypes.c_int, [vp, ctypes.c_int, pT, vp, vp]),
         "qlora_nf4_dequantize": (ctypes.c_int, [pT, vp, ctypes.c_int, vp]),
         "qlora_linear_fwd": (ctypes.c_int, [pT, pL, vp, i64, vp, ctypes.c_int, vp, vp, sz, vp]),
@@ -315,12 +316,16 @@ def linear_fwd_multi(q: NF4Weight, adapters, adapter_of_token, X, y_dtype=torch.
     arr = (LoraC * len(adapters))(*[_lora(a, b, alpha) for a, b, alpha in adapters])
     idx = (ctypes.c_int32 * M)(*[int(i) for i in adapter_of_token])
     if ws is None:
-        ws = new_workspace(workspace_bytes(M, q.rows, q.cols, r, False), X.device)
+        ws = new_workspace(workspace_bytes_multi(M, q.rows, q.cols, r), X.device)
     t = q.c_struct()
     _check(lib().qlora_linear_fwd_multi(ctypes.byref(t), arr, len(adapters), idx, _ptr(X), M, _ptr(Y),
                                         _dtype_code(Y.dtype), _ptr(ws), ws.numel(), _stream(stream)),
            "qlora_linear_fwd_multi")
     return Y
+
+
+def workspace_bytes_multi(m: int, n: int, k: int, r: int) -> int:
+    return int(lib().qlora_workspace_bytes_multi(m, n, k, r))
 
 
 def workspace_bytes_dropout(m: int, n: int, k: int, r: int, backward: bool) -> int:

@@ -70,7 +70,9 @@ struct GemvArgs {
   uint32_t *status;
   int rg_per_cta;
   int stages;               // bulk kernel: depth of the shared-memory ring
-  int multi;                // 1: token t adds s[t] (x_t A_t^T) B_t^T with ml's adapters
+  int multi;                // 1: token t adds s[t] (x_t A_t^T) B_t^T with ml's adapters;
+                            // 2: per-token adapters, base product only (the LoRA term follows
+                            //    in lora_up_multi_kernel)
   BulkLayout lay;           // bulk kernel: placement computed on the host for a window at lay_base
   uint32_t lay_base;
   MultiLora ml;
@@ -541,7 +543,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   // per-token adapters: each token's B rows of this CTA's row groups (contiguous,
   // my_rg * 16 rows of r ranks) start moving into L2 now, behind the weight stream,
   // so that the LoRA step after the main loop reads them from L2
-  if (a.multi && warp == 1 && lane < a.M && my_rg > 0)
+  if (a.multi == 1 && warp == 1 && lane < a.M && my_rg > 0)
     ptx::bulk_prefetch_l2(a.ml.B[lane] + (int64_t)rg0 * 16 * a.r, static_cast<uint32_t>(my_rg * 16 * a.r * 2));
 
   // this warp's slice of X for a chunk (raw bf16)
@@ -749,7 +751,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   }
   __syncthreads();
   const __nv_bfloat16 *const sT = a.sT + griddep_wait_token();
-  if (a.multi) {
+  if (a.multi == 1) {
     // one adapter per token.  s T (all tokens) is copied to shared memory (the
     // pair table's space, unused after the main loop).  Each token's B rows of
     // this CTA's row groups are one contiguous block of 16-byte pieces (P = r / 8
@@ -1053,6 +1055,57 @@ __global__ void __launch_bounds__(kLoraDownMultiThreads, 1) lora_down_multi_kern
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (lane == 0) sT[k] = __float2bfloat16_rn(acc * ml.s[t]);
+  }
+}
+
+// LoRA term of the multi-adapter decode as its own pass over all SMs, after the
+// GEMV has written the base product Yb (float32 [M, N]) to the workspace:
+//   Y[t, n] = round(Yb[t, n] + sum_j B_t[n, j] (s T)[t, j]).
+// For ranks with P = r / 8 a power of two: a warp reads 32 consecutive 16-byte
+// pieces of B_t (32 / P rows, coalesced), each lane dots its piece with its
+// slice of s T (kept in registers), the P lanes of a row combine their partials
+// by a butterfly in fixed order and the first writes the row.  B is an input of
+// the call, so each CTA loads its pieces before waiting for the GEMV
+// (programmatic dependent launch) and overlaps the GEMV's tail where it can.
+constexpr int kLoraUpThreads = 256, kLoraUpRounds = 4;
+__global__ void __launch_bounds__(kLoraUpThreads) lora_up_multi_kernel(const float *__restrict__ Yb, const MultiLora ml,
+                                                                      const __nv_bfloat16 *__restrict__ sT, int64_t N,
+                                                                      int r, void *Y, int y_f32) {
+  griddep_launch_dependents();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t = blockIdx.y;
+  const int P = r / 8, lgP = __ffs(P) - 1, rpw = 32 >> lgP;  // rows per warp round
+  const int ch = lane & (P - 1);
+  const int64_t rows_per_cta = (int64_t)(kLoraUpThreads / 32) * rpw * kLoraUpRounds;
+  const int64_t row0 = blockIdx.x * rows_per_cta + (int64_t)warp * rpw * kLoraUpRounds + (lane >> lgP);
+  const uint4 *B = reinterpret_cast<const uint4 *>(ml.B[t]);
+  uint4 bv[kLoraUpRounds];
+#pragma unroll
+  for (int u = 0; u < kLoraUpRounds; ++u) {
+    const int64_t n = row0 + u * rpw;
+    bv[u] = n < N ? __ldg(B + n * P + ch) : make_uint4(0, 0, 0, 0);
+  }
+  ptx::griddep_wait();  // s T and Yb are complete
+  const uint4 sv = __ldcg(reinterpret_cast<const uint4 *>(sT + (int64_t)t * r) + ch);
+  const float s8[8] = {bf16lo_to_f32(sv.x), bf16hi_to_f32(sv.x), bf16lo_to_f32(sv.y), bf16hi_to_f32(sv.y),
+                       bf16lo_to_f32(sv.z), bf16hi_to_f32(sv.z), bf16lo_to_f32(sv.w), bf16hi_to_f32(sv.w)};
+#pragma unroll
+  for (int u = 0; u < kLoraUpRounds; ++u) {
+    const int64_t n = row0 + u * rpw;
+    const uint32_t bw[4] = {bv[u].x, bv[u].y, bv[u].z, bv[u].w};
+    float v = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v = fmaf(bf16lo_to_f32(bw[e]), s8[2 * e], v);
+      v = fmaf(bf16hi_to_f32(bw[e]), s8[2 * e + 1], v);
+    }
+    for (int o = 1; o < P; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (ch == 0 && n < N) {
+      const int64_t i = (int64_t)t * N + n;
+      const float y = __ldcg(Yb + i) + v;
+      if (y_f32) reinterpret_cast<float *>(Y)[i] = y;
+      else reinterpret_cast<__nv_bfloat16 *>(Y)[i] = __float2bfloat16_rn(y);
+    }
   }
 }
 

@@ -286,6 +286,9 @@ size_t min_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r, int for_b
   }
   return bytes;
 }
+// Float32 [M, N] base product of the multi-adapter decode's split path, placed
+// after the minimum workspace.
+size_t multi_base_bytes(int64_t M, int64_t N) { return align256(static_cast<size_t>(M) * N * 4); }
 // Partial planes for K splitting, placed after the minimum workspace when the
 // caller passed room for them.
 float *split_part(void *ws, size_t ws_bytes, int64_t M, int64_t N, int64_t K, int32_t r, int for_backward) {
@@ -575,6 +578,12 @@ size_t qlora_nf4_storage_bytes(int64_t rows, int64_t cols, size_t *codes_bytes, 
   return n / 2 + nb + ng * sizeof(float);
 }
 
+size_t qlora_workspace_bytes_multi(int64_t M, int64_t N, int64_t K, int32_t r) {
+  const size_t lo = min_workspace_bytes(M, N, K, r, 0);
+  if (lo == 0 || M > kGemvMaxM) return 0;
+  return lo + multi_base_bytes(M, N);
+}
+
 size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r, int for_backward) {
   const size_t lo = min_workspace_bytes(M, N, K, r, for_backward);
   if (lo == 0) return 0;
@@ -781,6 +790,13 @@ qlora_status qlora_linear_fwd_multi(const qlora_nf4_tensor *W, const qlora_lora 
   }
   uint8_t *wsb = static_cast<uint8_t *>(ws);
   __nv_bfloat16 *sT = reinterpret_cast<__nv_bfloat16 *>(wsb + QLORA_STATUS_BYTES);
+  // With room for a float32 [M, N] base product after the minimum workspace and a
+  // rank with a power-of-two number of 16-byte pieces per row, the LoRA term runs
+  // as its own pass over all SMs after the GEMV (lora_up_multi_kernel).
+  const size_t ws_lo = min_workspace_bytes(M, N, K, r, 0);
+  const int P = r / 8;
+  const bool split = (P & (P - 1)) == 0 && ws_bytes >= ws_lo + multi_base_bytes(M, N);
+  float *Yb = split ? reinterpret_cast<float *>(wsb + ws_lo) : nullptr;
   // s T on the SMs the GEMV leaves free (at least eight CTAs, at most one warp per row)
   const int rows = static_cast<int>(M) * r, warps = kLoraDownMultiThreads / 32;
   int down = sms - gemv_grid_ctas(N, sms, true);
@@ -795,13 +811,18 @@ qlora_status qlora_linear_fwd_multi(const qlora_nf4_tensor *W, const qlora_lora 
   g.sT = sT;
   g.B = g.ml.B[0];
   g.r = r;
-  g.Y = Y; g.y_f32 = y_dtype == QLORA_F32;
+  g.Y = split ? static_cast<void *>(Yb) : Y;
+  g.y_f32 = split ? 1 : (y_dtype == QLORA_F32);
   g.status = status_ptr(ws);
-  g.multi = 1;
+  g.multi = split ? 2 : 1;
   CUtensorMap tmc;
   if (!tmap_codes_gemv(&tmc, W->codes, N, K, static_cast<uint32_t>((K < 4096 ? K : 4096) / 256)))
     return QLORA_ERR_CUDA;
-  return launch_gemv(g, &tmc, dev, sms, st);
+  if ((s = launch_gemv(g, &tmc, dev, sms, st)) != QLORA_OK || !split) return s;
+  const int64_t rows_per_cta = static_cast<int64_t>(kLoraUpThreads / 32) * (32 / P) * kLoraUpRounds;
+  const dim3 grid(static_cast<unsigned>((N + rows_per_cta - 1) / rows_per_cta), static_cast<unsigned>(M));
+  return launch_pdl(lora_up_multi_kernel, grid, dim3(kLoraUpThreads), 0, st, static_cast<const float *>(Yb), g.ml,
+                    static_cast<const __nv_bfloat16 *>(sT), N, r, Y, y_dtype == QLORA_F32 ? 1 : 0);
 }
 
 qlora_status qlora_lora_merge(const qlora_nf4_tensor *W, const qlora_lora *adapter, void *W_out,

@@ -143,6 +143,11 @@ QLORA_API size_t qlora_nf4_storage_bytes(int64_t rows, int64_t cols, size_t *cod
  * float32 rounding order. */
 QLORA_API size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t r, int for_backward);
 
+/* Workspace bytes for qlora_linear_fwd_multi's faster path: the forward minimum
+ * for M tokens plus a float32 [M, N] buffer (256-byte rounded); 0 for invalid
+ * sizes or M > 16. */
+QLORA_API size_t qlora_workspace_bytes_multi(int64_t M, int64_t N, int64_t K, int32_t r);
+
 /* Quantise W [out->rows, out->cols] (float32 or bf16, row-major, device) to NF4
  * with double-quantised scales (glossary page, "How QLoRA works": NF4 and double
  * quantisation bullets).  Writes out->codes, out->scale_codes, out->c2.
@@ -239,7 +244,12 @@ QLORA_API qlora_status qlora_linear_bwd_dropout(const qlora_nf4_tensor *W, const
  *   adapters          host array of n_adapters >= 1 adapters, all of one rank r
  *   adapter_of_token  HOST int32 [M], values in [0, n_adapters)
  *   X bf16 [M, K], Y [M, N] (y_dtype) device; 1 <= M <= 16
- *   ws                device workspace, as qlora_linear_fwd's for M tokens
+ *   ws                device workspace, as qlora_linear_fwd's for M tokens; given
+ *                     qlora_workspace_bytes_multi(M, N, K, r) bytes (room for a
+ *                     float32 [M, N] base product) and r / 8 a power of two, the
+ *                     adapters' term runs as a separate pass over all SMs after
+ *                     the base GEMV (faster); results agree to float32 rounding
+ *                     order either way
  * Runs the staged decode kernel: N % 16 == 0, K % 256 == 0 and (K <= 4096 or
  * K % 4096 == 0), else QLORA_ERR_UNSUPPORTED_SHAPE.  No T is saved (decode). */
 QLORA_API qlora_status qlora_linear_fwd_multi(const qlora_nf4_tensor *W, const qlora_lora *adapters,

@@ -199,3 +199,11 @@ def test_keep_mask_generator_packs_like_the_oracle():
     g = torch.Generator().manual_seed(11)
     want = (torch.rand((5, 48), generator=g, dtype=torch.float64) >= 0.3).numpy()
     assert np.array_equal(O.unpack_keep(packed.numpy(), 5, 48), want)
+
+
+def test_multi_workspace_size(L):
+    for m, n, k, r in ((1, 11008, 4096, 64), (16, 11008, 4096, 64), (7, 1000, 512, 24)):
+        lo = L.qlora_workspace_bytes(m, n, k, r, 0)
+        assert L.qlora_workspace_bytes_multi(m, n, k, r) == lo + ((m * n * 4 + 255) // 256) * 256
+    assert L.qlora_workspace_bytes_multi(17, 1024, 1024, 16) == 0
+    assert L.qlora_workspace_bytes_multi(4, 1024, 1024, 300) == 0

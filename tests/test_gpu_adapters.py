@@ -104,6 +104,13 @@ def test_multi_adapter_gemv_matches_oracle(n, k, m, r, count):
     y = bd.linear_fwd_multi(qg, [(a.cuda(), b.cuda(), al) for a, b, al in ads], idx, x.cuda(), y_dtype=torch.float32)
     torch.cuda.synchronize()
     _check(f"y {n}x{k} m={m}", y, ref)
+    # the minimum workspace: the adapters' term inside the GEMV instead of its own pass
+    ws = bd.new_workspace(bd.workspace_bytes(m, n, k, r, False), torch.device("cuda"))
+    y_min = bd.linear_fwd_multi(qg, [(a.cuda(), b.cuda(), al) for a, b, al in ads], idx, x.cuda(),
+                                y_dtype=torch.float32, ws=ws)
+    torch.cuda.synchronize()
+    _check(f"y {n}x{k} m={m}, minimum workspace", y_min, ref)
+    assert bd.read_status(ws) == 0
     # the adapters' own contribution, alone
     y0 = bd.linear_fwd_multi(qg, [(a.cuda(), torch.zeros_like(b).cuda(), al) for a, b, al in ads], idx, x.cuda(),
                              y_dtype=torch.float32)
