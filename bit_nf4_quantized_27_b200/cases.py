@@ -64,7 +64,7 @@ def main(argv=None):
         for i in range(16):
             _, _, a, b, _ = _layer(11008, 4096, 1, seed=100 + i)
             ads.append((a, b, 16.0))
-        ws = bd.new_workspace(bd.workspace_bytes(16, 11008, 4096, 64, False))
+        ws = bd.new_workspace(bd.workspace_bytes_multi(16, 11008, 4096, 64))
         for _ in range(args.reps):
             bd.linear_fwd_multi(q, ads, list(range(16)), x, ws=ws)
         st = bd.read_status(ws)
