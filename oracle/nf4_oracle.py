@@ -20,7 +20,7 @@ Sources, cited by page title and section:
 * [EZ] "Mastering model fine-tuning" -- ezsol.ir.  Section "Low-Rank Adaptation
   (LoRA)": Delta W = B A.
 
-Readings where the pages are silent or loose (each also listed in the design doc):
+Readings where the pages are silent or loose:
 
 * The level table is built in exact arithmetic (float64, Wichura's AS241 for the
   normal quantile) and rounded to float32 once; the offset is the printed
