@@ -12,6 +12,7 @@ CASE is one of:
   gemv_multi16  decode forward of 16 tokens, each with its own r=64 adapter
   quant_11008   quantise an 11008x4096 bf16 weight
   dequant_11008 dequantise it
+  quant_4096 / dequant_4096     the same for a 4096x4096 weight
   merge_8192    merged export of an 8192x8192 NF4 weight with an r = 64 adapter
   adamw_65b     AdamW step over the adapters of the 65B-shaped block (flat fp32)
 Inputs are drawn on the device from fixed seeds; every run exits 0 on success.
@@ -76,8 +77,8 @@ def main(argv=None):
         for _ in range(args.reps):
             bd.linear_fwd(q, a, b, 16.0, x, ws=ws)
         st = bd.read_status(ws)
-    elif c in ("quant_11008", "dequant_11008"):
-        w, *_ = _layer(11008, 4096, 1)
+    elif c in ("quant_11008", "dequant_11008", "quant_4096", "dequant_4096"):
+        w, *_ = _layer(11008 if c.endswith("11008") else 4096, 4096, 1)
         ws = bd.new_workspace(bd.STATUS_BYTES)
         q = bd.quantize(w, ws=ws)
         out = torch.empty_like(w)
