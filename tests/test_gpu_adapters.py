@@ -52,6 +52,23 @@ def test_merge_with_b_zero_is_the_dequantised_weight():
     assert torch.equal(got.view(torch.int16), deq.view(torch.int16))
 
 
+@pytest.mark.parametrize("minimum_ws", [False, True])
+def test_multi_adapter_bf16_output_is_the_rounded_float32_output(minimum_ws):
+    """bf16 Y must be bf16(the float32 Y of the same call): one rounding of the sum."""
+    n, k, m, r = 2048, 1024, 6, 32
+    w, x, _, _, _ = I.custom(n, k, m, r, 4242)
+    ads = [(a.cuda(), b.cuda(), al) for a, b, al in _adapters(n, k, r, 3, 4343)]
+    idx = [t % 3 for t in range(m)]
+    qg = bd.quantize(w.cuda())
+    size = bd.workspace_bytes(m, n, k, r, False) if minimum_ws else bd.workspace_bytes_multi(m, n, k, r)
+    ws = bd.new_workspace(size, torch.device("cuda"))
+    y32 = bd.linear_fwd_multi(qg, ads, idx, x.cuda(), y_dtype=torch.float32, ws=ws)
+    y16 = bd.linear_fwd_multi(qg, ads, idx, x.cuda(), y_dtype=torch.bfloat16, ws=ws)
+    torch.cuda.synchronize()
+    assert bd.read_status(ws) == 0
+    assert torch.equal(y16.view(torch.int16), y32.to(torch.bfloat16).view(torch.int16))
+
+
 @pytest.mark.parametrize("n", [1, 7, 1000003])
 def test_adamw_matches_oracle_over_six_steps(n):
     g = torch.Generator().manual_seed(n)
