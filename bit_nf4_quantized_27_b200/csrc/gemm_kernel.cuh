@@ -314,7 +314,9 @@ template <bool A_MN, bool B_MN, bool NF4, int BN, int MT>
 __global__ void __launch_bounds__(GemmCfg<A_MN, B_MN, NF4, BN, MT>::THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-               const __grid_constant__ CUtensorMap tmCodes, const GemmArgs args) {
+               const __grid_constant__ CUtensorMap tmCodes, const GemmArgs args,
+               const __grid_constant__ CUtensorMap tmAg, const __grid_constant__ CUtensorMap tmBg,
+               const __grid_constant__ CUtensorMap tmB2g, const GemmArgs argsg) {
   using C = GemmCfg<A_MN, B_MN, NF4, BN, MT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -355,6 +357,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     if (args.hilo_cols) ptx::prefetch_tmap(&tmB2);
     if (args.lora_steps) ptx::prefetch_tmap(&tmA2);
     if (NF4) ptx::prefetch_tmap(&tmCodes);
+    if (argsg.M_rows > 0) {
+      ptx::prefetch_tmap(&tmAg);
+      ptx::prefetch_tmap(&tmBg);
+      if (args.hilo_cols) ptx::prefetch_tmap(&tmB2g);
+    }
   }
   if (warp == 1) {
     ptx::tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -374,17 +381,36 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const int num_n = (args.N_cols + tile_n - 1) / tile_n;
   const int tiles_mn = num_m * num_n;
   const int ksplit = args.ksplit > 1 ? args.ksplit : 1;
-  const int num_tiles = tiles_mn * ksplit;
+  const int num_tiles1 = tiles_mn * ksplit;
+  // A second, independent problem (argsg: its own maps, output and sizes; the
+  // same tile shape and column halves, no K split and no LoRA steps) may share
+  // the launch: its tiles follow this one's, so both run at once.
+  const int num_m_g = argsg.M_rows > 0 ? (argsg.M_rows + C::BM * MT - 1) / (C::BM * MT) : 0;
+  const int num_n_g = argsg.M_rows > 0 ? (argsg.N_cols + tile_n - 1) / tile_n : 0;
+  const int num_tiles = num_tiles1 + num_m_g * num_n_g;
   auto tile_of = [&](int w, int &m0, int &n0) {
+    if (w >= num_tiles1) {
+      const int v = w - num_tiles1;
+      m0 = (v % num_m_g) * C::BM * MT;
+      n0 = (v / num_m_g) * tile_n;
+      return;
+    }
     const int mn = w % tiles_mn;
     m0 = (mn % num_m) * C::BM * MT;
     n0 = (mn / num_m) * tile_n;
   };
   const int main_steps = args.k_steps;
   const int steps = main_steps + args.lora_steps;
+  // main (non-LoRA) K steps of tile w's problem
+  auto main_of = [&](int w) { return w >= num_tiles1 ? argsg.k_steps : main_steps; };
   // K steps [k_begin, k_end) of tile w (its share of the split)
   const int k_per = ksplit > 1 ? args.k_per : steps;
   auto k_range = [&](int w, int &kb, int &ke) {
+    if (w >= num_tiles1) {
+      kb = 0;
+      ke = argsg.k_steps;
+      return;
+    }
     const int sp = w / tiles_mn;
     kb = sp * k_per;
     ke = min(steps, kb + k_per);
@@ -405,8 +431,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         int m0, n0, kb, ke;
         tile_of(tile, m0, n0);
         k_range(tile, kb, ke);
+        const bool g2 = tile >= num_tiles1;
+        const CUtensorMap *mA = g2 ? &tmAg : &tmA, *mB = g2 ? &tmBg : &tmB, *mB2 = g2 ? &tmB2g : &tmB2;
+        const int ms = main_of(tile);
         for (int ks = kb; ks < ke && ok; ++ks) {
-          const bool lora = ks >= main_steps;
+          const bool lora = ks >= ms;
           const int kk = ks;
           if (NF4 && !lora) {
             if (!ptx::mbar_wait(&empty_c[sc], pc ^ 1, abort_flag)) { ok = false; break; }
@@ -425,21 +454,21 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             const int k2 = (ks - main_steps) * 64;
             for (int t = 0; t < MT; ++t) ptx::tma_load_2d(dA + t * 16384, &tmA2, &full_a[sa], k2, m0 + t * 128);
           } else if (!A_MN) {
-            for (int t = 0; t < MT; ++t) ptx::tma_load_2d(dA + t * 16384, &tmA, &full_a[sa], kk * 64, m0 + t * 128);
+            for (int t = 0; t < MT; ++t) ptx::tma_load_2d(dA + t * 16384, mA, &full_a[sa], kk * 64, m0 + t * 128);
           } else {
-            for (int t = 0; t < MT * 2; ++t) ptx::tma_load_2d(dA + t * 8192, &tmA, &full_a[sa], m0 + t * 64, kk * 64);
+            for (int t = 0; t < MT * 2; ++t) ptx::tma_load_2d(dA + t * 8192, mA, &full_a[sa], m0 + t * 64, kk * 64);
           }
           if (!NF4) {
             uint8_t *dB = sB + sa * C::B_STAGE;
             if (!B_MN) {
-              ptx::tma_load_2d(dB, &tmB, &full_a[sa], kk * 64, n0);
+              ptx::tma_load_2d(dB, mB, &full_a[sa], kk * 64, n0);
             } else if (!args.hilo_cols) {
-              for (int t = 0; t < BN / 64; ++t) ptx::tma_load_2d(dB + t * 8192, &tmB, &full_a[sa], n0 + t * 64, kk * 64);
+              for (int t = 0; t < BN / 64; ++t) ptx::tma_load_2d(dB + t * 8192, mB, &full_a[sa], n0 + t * 64, kk * 64);
             } else {  // columns n0.. of B, then the same columns of B2
               constexpr int kHalfBlocks = BN >= 128 ? BN / 128 : 1;  // 64-column blocks per half
               for (int t = 0; t < BN / 64; ++t) {
                 const int h = t / kHalfBlocks;
-                ptx::tma_load_2d(dB + t * 8192, h ? &tmB2 : &tmB, &full_a[sa], n0 + (t % kHalfBlocks) * 64, kk * 64);
+                ptx::tma_load_2d(dB + t * 8192, h ? mB2 : mB, &full_a[sa], n0 + (t % kHalfBlocks) * 64, kk * 64);
               }
             }
           }
@@ -471,11 +500,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const uint32_t acc_phase = (it / C::NUM_ACC) & 1;
         int kb, ke;
         k_range(tile, kb, ke);
+        const int ms = main_of(tile);
         if (!ptx::mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag)) { ok = false; break; }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * C::ACC_COLS;
         for (int ks = kb; ks < ke && ok; ++ks) {
-          const bool lora = ks >= main_steps;
+          const bool lora = ks >= ms;
           if (!ptx::mbar_wait(&full_a[sa], pa, abort_flag)) { ok = false; break; }
           if (NF4 && !ptx::mbar_wait(&full_b[sb], pb, abort_flag)) { ok = false; break; }
           ptx::tc_fence_after();
@@ -520,7 +550,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       ptx::tc_fence_after();
       int m0, n0;
       tile_of(tile, m0, n0);
-      const int sp = tile / tiles_mn;
+      const bool g2 = tile >= num_tiles1;
+      const GemmArgs &ea = g2 ? argsg : args;  // the tile's problem
+      const int sp = g2 ? 0 : tile / tiles_mn;
       for (int t = 0; t < MT; ++t) {
         const int row = m0 + t * 128 + q * 32 + lane;
         for (int cb = 0; cb < tile_n; cb += 32) {
@@ -536,15 +568,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(w2[j]));
           }
           const int col0 = n0 + cb;
-          if (row < args.M_rows && col0 < args.N_cols) {
-            if (ksplit > 1) {  // raw fp32 partial of this K share
+          if (row < ea.M_rows && col0 < ea.N_cols) {
+            if (ksplit > 1 && !g2) {  // raw fp32 partial of this K share
               float *o = args.part + ((int64_t)sp * args.M_rows + row) * args.N_cols + col0;
               const int nc = min(32, args.N_cols - col0);
 #pragma unroll
               for (int j = 0; j < 32; ++j)
                 if (j < nc) o[j] = __uint_as_float(v[j]);
             } else {
-              store_chunk32(args, row, col0, min(32, args.N_cols - col0), v);
+              store_chunk32(ea, row, col0, min(32, ea.N_cols - col0), v);
             }
           }
         }

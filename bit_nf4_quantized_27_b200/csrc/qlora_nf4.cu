@@ -188,10 +188,14 @@ qlora_status launch_gemm_pair(const CUtensorMap &tmA, const CUtensorMap &tmA2, c
 // Token counts from which the fused GEMMs run on CTA pairs (512-token tiles).
 constexpr int64_t kPairMinRows = 257;
 
+// One tcgen05 GEMM launch; with `group` (a second problem of the same tile shape,
+// no K split, no LoRA steps, maps gA / gB / gB2) both problems share the launch
+// and run at once.
 template <bool A_MN, bool B_MN, bool NF4, int BN, int MT>
 qlora_status launch_gemm(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmA2,
                          const CUtensorMap &tmB2, const CUtensorMap &tmCodes, const GemmArgs &args, int dev, int sms,
-                         cudaStream_t st) {
+                         cudaStream_t st, const GemmArgs *group = nullptr, const CUtensorMap *gA = nullptr,
+                         const CUtensorMap *gB = nullptr, const CUtensorMap *gB2 = nullptr) {
   using C = GemmCfg<A_MN, B_MN, NF4, BN, MT>;
   auto kernel = gemm_tc_kernel<A_MN, B_MN, NF4, BN, MT>;
   static std::once_flag flags[64];
@@ -201,9 +205,16 @@ qlora_status launch_gemm(const CUtensorMap &tmA, const CUtensorMap &tmB, const C
   const int tile_n = args.hilo_cols ? BN / 2 : BN;
   const int num_m = (args.M_rows + C::BM * MT - 1) / (C::BM * MT);
   const int num_n = (args.N_cols + tile_n - 1) / tile_n;
-  const int tiles = num_m * num_n * std::max(1, args.ksplit);
+  int tiles = num_m * num_n * std::max(1, args.ksplit);
+  GemmArgs none{};  // no second problem
+  if (group) {
+    if (NF4 || group->ksplit > 1 || group->lora_steps || group->hilo_cols != args.hilo_cols || group->M_rows <= 0)
+      return QLORA_ERR_INVALID_ARGUMENT;
+    tiles += ((group->M_rows + C::BM * MT - 1) / (C::BM * MT)) * ((group->N_cols + tile_n - 1) / tile_n);
+  }
   const int grid = std::max(1, std::min(tiles, sms));
-  return launch_pdl(kernel, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, st, tmA, tmB, tmA2, tmB2, tmCodes, args);
+  return launch_pdl(kernel, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, st, tmA, tmB, tmA2, tmB2, tmCodes, args,
+                    group ? *gA : tmA, group ? *gB : tmB, group ? *gB2 : tmB2, group ? *group : none);
 }
 
 uint32_t *status_ptr(void *ws) { return reinterpret_cast<uint32_t *>(ws); }
@@ -511,43 +522,37 @@ qlora_status bwd_impl(const qlora_nf4_tensor *W, const qlora_lora *ad, const voi
     if ((s = launch_gemm<false, true, false, 128, 1>(tmU, tmAl, tmU, tmU, tmU, g, dev, sms, st)) != QLORA_OK)
       return s;
   }
-  // dA^T [K, r] = X^T (s U_hi + s U_lo)  -> stored transposed into dA [r, K]
+  // dA^T [K, r] = X^T (s U_hi + s U_lo)  -> stored transposed into dA [r, K], and
+  // dB [N, r] = s dY^T (T_hi + T_lo): independent, one launch for both
   {
-    CUtensorMap tmXt, tmUh, tmUl;
+    CUtensorMap tmXt, tmUh, tmUl, tmDYt, tmTh, tmTl;
     if (!tmap_bf16(&tmXt, Xl, K, M, 64, 64) || !tmap_bf16(&tmUh, sU_hi, r, M, 64, 64) ||
-        !tmap_bf16(&tmUl, sU_lo, r, M, 64, 64))
+        !tmap_bf16(&tmUl, sU_lo, r, M, 64, 64) || !tmap_bf16(&tmDYt, dY, N, M, 64, 64) ||
+        !tmap_bf16(&tmTh, T_hi, r, M, 64, 64) || !tmap_bf16(&tmTl, T_lo, r, M, 64, 64))
       return QLORA_ERR_CUDA;
-    GemmArgs g{};
-    g.M_rows = (int)K;
-    g.N_cols = r;
-    g.k_steps = (int)((M + 63) / 64);
-    g.hilo_cols = 1;
-    g.out = dA;
-    g.ldo = K;
-    g.out_f32 = grad_dtype == QLORA_F32;
-    g.out_transpose = 1;
-    g.out_scale = t_scale;
-    g.status = status;
-    if ((s = launch_gemm<true, true, false, 128, 1>(tmXt, tmUh, tmXt, tmUl, tmXt, g, dev, sms, st)) != QLORA_OK)
-      return s;
-  }
-  // dB [N, r] = s dY^T (T_hi + T_lo)
-  {
-    CUtensorMap tmDYt, tmTh, tmTl;
-    if (!tmap_bf16(&tmDYt, dY, N, M, 64, 64) || !tmap_bf16(&tmTh, T_hi, r, M, 64, 64) ||
-        !tmap_bf16(&tmTl, T_lo, r, M, 64, 64))
-      return QLORA_ERR_CUDA;
-    GemmArgs g{};
-    g.M_rows = (int)N;
-    g.N_cols = r;
-    g.k_steps = (int)((M + 63) / 64);
-    g.hilo_cols = 1;
-    g.out = dB;
-    g.ldo = r;
-    g.out_f32 = grad_dtype == QLORA_F32;
-    g.out_scale = sc;
-    g.status = status;
-    if ((s = launch_gemm<true, true, false, 128, 1>(tmDYt, tmTh, tmDYt, tmTl, tmDYt, g, dev, sms, st)) != QLORA_OK)
+    GemmArgs ga{};
+    ga.M_rows = (int)K;
+    ga.N_cols = r;
+    ga.k_steps = (int)((M + 63) / 64);
+    ga.hilo_cols = 1;
+    ga.out = dA;
+    ga.ldo = K;
+    ga.out_f32 = grad_dtype == QLORA_F32;
+    ga.out_transpose = 1;
+    ga.out_scale = t_scale;
+    ga.status = status;
+    GemmArgs gb{};
+    gb.M_rows = (int)N;
+    gb.N_cols = r;
+    gb.k_steps = (int)((M + 63) / 64);
+    gb.hilo_cols = 1;
+    gb.out = dB;
+    gb.ldo = r;
+    gb.out_f32 = grad_dtype == QLORA_F32;
+    gb.out_scale = sc;
+    gb.status = status;
+    if ((s = launch_gemm<true, true, false, 128, 1>(tmXt, tmUh, tmXt, tmUl, tmXt, ga, dev, sms, st, &gb, &tmDYt,
+                                                     &tmTh, &tmTl)) != QLORA_OK)
       return s;
   }
   return QLORA_OK;
