@@ -51,7 +51,7 @@ def load_peaks():
 FUSED_FWD_TRAFFIC_BYTES = 592.60e6
 FUSED_FWD_TRAFFIC_SOURCES = ("gemm_pair_kernel.cuh", "gemm_kernel.cuh", "sm100_ptx.cuh", "nf4_device.cuh",
                              "qlora_nf4.cu")
-FUSED_FWD_TRAFFIC_DIGEST = "71739ba80dd663fd"
+FUSED_FWD_TRAFFIC_DIGEST = "aa961c27569a8b40"
 
 
 def fused_fwd_traffic():
