@@ -291,9 +291,10 @@ def run_step(layers, wl, flat, world, timing=None, ready=None, quant=True):
 
 def launches_per_step(nlayers):
     # per layer of the 65B-shaped block: quantise 1; forward 3 (T with split K and
-    # its finishing sum, fused GEMM); backward 5 (U with split K and its finishing
-    # sum, dX, dA, dB) -- 63 per step, as the ncu launch list of the step shows
-    return nlayers * 9
+    # its finishing sum, fused GEMM); backward 4 (U with split K and its finishing
+    # sum, dX, dA and dB in one launch) -- 56 per step, as the ncu launch list of
+    # the step shows
+    return nlayers * 8
 
 
 def graph_time_us(calls, reps=5):
