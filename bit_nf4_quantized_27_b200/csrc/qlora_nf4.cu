@@ -643,8 +643,12 @@ qlora_status qlora_nf4_dequantize(const qlora_nf4_tensor *w, void *W_out, qlora_
     const int64_t wsteps = (nweights + 1023) / 1024;
     const int64_t ctas = (wsteps + 2 * kDequantWarps - 1) / (2 * kDequantWarps);
     const unsigned gb = (unsigned)std::max<int64_t>(1, std::min<int64_t>(ctas, (int64_t)1 << 20));
-    nf4_dequantize_bf16_kernel<<<gb, kDequantThreads, 0, st>>>(w->codes, w->scale_codes, w->c2, nweights,
-                                                               static_cast<__nv_bfloat16 *>(W_out), w->scale_format);
+    if (reinterpret_cast<uintptr_t>(W_out) % 32 == 0)
+      nf4_dequantize_bf16_v8_kernel<<<gb, kDequantThreads, 0, st>>>(w->codes, w->scale_codes, w->c2, nweights,
+                                                                   static_cast<__nv_bfloat16 *>(W_out), w->scale_format);
+    else
+      nf4_dequantize_bf16_kernel<<<gb, kDequantThreads, 0, st>>>(w->codes, w->scale_codes, w->c2, nweights,
+                                                                 static_cast<__nv_bfloat16 *>(W_out), w->scale_format);
   } else
     nf4_dequantize_kernel<float><<<grid, kDequantThreads, 0, st>>>(w->codes, w->scale_codes, w->c2, nchunks,
                                                                    static_cast<float *>(W_out), w->scale_format);

@@ -336,4 +336,65 @@ nf4_dequantize_bf16_kernel(const uint8_t *__restrict__ codes, const uint8_t *__r
   }
 }
 
+
+// The same with 32-byte stores, for a 32-byte aligned output: each lane decodes
+// two consecutive code words (16 weights of one block, one block scale) and
+// writes them with one 256-bit store, so a warp instruction writes 1 KB.
+__global__ void __launch_bounds__(kDequantThreads)
+nf4_dequantize_bf16_v8_kernel(const uint8_t *__restrict__ codes, const uint8_t *__restrict__ scale_codes,
+                              const float *__restrict__ c2, int64_t nweights, __nv_bfloat16 *__restrict__ out,
+                              int fmt) {
+  __shared__ float s_lv[16];
+  if (threadIdx.x < 16) s_lv[threadIdx.x] = __uint_as_float(kNf4LevelBits[threadIdx.x]);
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t nwords = nweights / 8;  // a multiple of 8 (whole blocks)
+  const int64_t nsteps = (nweights + 1023) / 1024;
+  const int64_t wstride = (int64_t)gridDim.x * kDequantWarps;
+  int64_t ws = (int64_t)blockIdx.x * kDequantWarps + warp;
+  uint2 cw[2];
+  uint32_t sq[2];
+  float cz[2];
+  auto fetch = [&](int64_t step) {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int64_t w = step * 128 + k * 64 + 2 * lane;  // the lane's first code word of the pair
+      const bool in = step < nsteps && w < nwords;
+      cw[k] = in ? __ldcs(reinterpret_cast<const uint2 *>(codes) + w / 2) : make_uint2(0, 0);
+      sq[k] = in ? __ldg(scale_codes + (w >> 3)) : 0u;
+      cz[k] = in ? __ldg(c2 + (w >> 11)) : 0.0f;
+    }
+  };
+  fetch(ws);
+  for (; ws < nsteps; ws += wstride) {
+    uint2 wv[2];
+    float S[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      wv[k] = cw[k];
+      S[k] = __fmul_rn(scale_code_value(sq[k], fmt), cz[k]);
+    }
+    const int64_t w0 = ws * 128 + 2 * lane;
+    fetch(ws + wstride);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int64_t w = w0 + 64 * k;
+      if (w < nwords) {
+        uint32_t o[8];
+        const uint32_t ww[2] = {wv[k].x, wv[k].y};
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t byte = (ww[h] >> (8 * j)) & 0xffu;
+            o[4 * h + j] = pack_bf16x2(__fmul_rn(s_lv[byte & 0xf], S[k]), __fmul_rn(s_lv[byte >> 4], S[k]));
+          }
+        asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(out + w * 8), "r"(o[0]),
+                     "r"(o[1]), "r"(o[2]), "r"(o[3]), "r"(o[4]), "r"(o[5]), "r"(o[6]), "r"(o[7])
+                     : "memory");
+      }
+    }
+  }
+}
+
 }  // namespace qlora

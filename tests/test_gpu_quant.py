@@ -41,6 +41,21 @@ def _compare_dequant(q, ref, rows, cols):
     assert np.array_equal(got32.view(np.uint32), wd.view(np.uint32))
 
 
+def test_dequantize_into_a_16_byte_aligned_view():
+    """W_out only 16-byte aligned (not 32): the 16-byte-store kernel writes it."""
+    rows, cols = 96, 320
+    w = I.custom(rows, cols, 1, 8, 515)[0]
+    q, ref = _compare_quant(w)
+    wd = O.dequantize(ref["codes"], ref["scale_codes"], ref["c2"], rows, cols)
+    buf = torch.full((rows * cols + 8,), -1, dtype=torch.int16, device="cuda")
+    view = buf[8:].view(torch.bfloat16).view(rows, cols)  # 16 bytes past a 256-byte aligned start
+    assert view.data_ptr() % 32 == 16
+    bd.dequantize(q, torch.bfloat16, out=view)
+    got = buf.cpu().numpy().view(np.uint16)
+    assert np.all(got[:8] == 0xFFFF)  # nothing before the view is touched
+    assert np.array_equal(got[8:], O.bf16_bits(wd.reshape(-1)))
+
+
 def test_tiny_workload_fp32():
     w = I.weight(I.TINY)
     assert w.dtype == torch.float32 and w.shape == (256, 256)
